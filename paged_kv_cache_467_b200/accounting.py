@@ -1,0 +1,51 @@
+"""Byte accounting for a paged KV cache.
+
+The cache-size rule is stated in words on the KV-cache overview page (t13_4,
+cache-size paragraph): keys and values (the leading 2), times layers, KV heads,
+head dimension, retained tokens and bytes per element.  "KV Cache Engineering
+for LLM Serving", The cache formula, gives the same rule (its own copy of the
+formula did not survive extraction) and notes 2 bytes for BF16, 1 for FP8.
+"""
+from __future__ import annotations
+
+BYTES_PER_VALUE = {"f32": 4, "bf16": 2, "int8": 1, "fp8_e4m3": 1}
+
+
+def cache_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, bytes_per_value: float) -> float:
+    """Raw K+V cache bytes for one sequence."""
+    return 2 * layers * kv_heads * head_dim * tokens * bytes_per_value
+
+
+def block_bytes(block_size: int, kv_heads: int, head_dim: int, bytes_per_value: float) -> float:
+    """K+V bytes of one physical block of one layer (Chapter 18, Physical KV Block)."""
+    return cache_bytes(1, kv_heads, head_dim, block_size, bytes_per_value)
+
+
+def cached_scalars(kv_heads: int, tokens: int, head_size: int) -> int:
+    """K+V scalars held for ``tokens`` tokens of one layer ("KV Cache Engineering", section 1)."""
+    return 2 * kv_heads * tokens * head_size
+
+
+def tokens_in_pool(pool_bytes: float, bytes_per_token: float) -> int:
+    """Whole tokens that fit in a fixed pool ("KV Cache Engineering", section 10)."""
+    return int(pool_bytes // bytes_per_token)
+
+
+def scale_bytes_per_token(cache_dtype: str, kv_heads: int) -> int:
+    """Per-token scale metadata read with the codes: one fp32 per (token, head) for K and V with int8."""
+    return 2 * kv_heads * 4 if cache_dtype == "int8" else 0
+
+
+def decode_kv_bytes(w, unique: bool = True) -> int:
+    """K+V bytes one decode step must read from HBM for workload ``w``.
+
+    ``unique=True`` counts each physical block once (a shared prefix block is
+    read from DRAM once per step at best); ``unique=False`` counts the logical
+    bytes every sequence attends to.  Per-token scale bytes are included.
+    """
+    per_token = cache_bytes(1, w.n_kv, w.head_dim, 1, BYTES_PER_VALUE[w.cache_dtype])
+    per_token += scale_bytes_per_token(w.cache_dtype, w.n_kv)
+    tokens = int(w.context_lens.astype("int64").sum())
+    if unique and w.shared_prefix_tokens:
+        tokens -= (w.num_seqs - 1) * w.shared_prefix_tokens
+    return int(tokens * per_token)

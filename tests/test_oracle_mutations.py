@@ -1,0 +1,91 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin catches each.
+
+Every mutant is applied with monkeypatch, so the oracle itself is untouched
+once the test ends.
+"""
+import numpy as np
+import pytest
+
+import oracle.paged_attention as pa
+import oracle.quant as oq
+import test_oracle_attention as pins
+import test_oracle_quant as qpins
+from conftest import read_golden
+
+
+def _fails(check):
+    with pytest.raises(AssertionError):
+        check()
+
+
+def test_interleaved_gqa_mapping_is_caught(monkeypatch):
+    monkeypatch.setattr(pa, "kv_head_of", lambda h, n_q, n_kv: h % n_kv)
+    _fails(pins.check_contiguous_equals_sdpa)
+    _fails(lambda: pins.test_gqa_mapping_example(read_golden))
+
+
+def test_dropped_scale_is_caught(monkeypatch):
+    real = pa.attention_one_sequence
+    monkeypatch.setattr(pa, "attention_one_sequence", lambda q, K, V, sm_scale, **kw: real(q, K, V, 1.0, **kw))
+    _fails(pins.check_against_brute)
+
+
+def test_missing_length_truncation_is_caught(monkeypatch):
+    def whole_blocks(cache, block_row, length, block_size):
+        n_blocks = -(-length // block_size)
+        return np.concatenate([cache[int(block_row[j])] for j in range(n_blocks)], axis=0) if n_blocks else cache[:0, 0]
+
+    monkeypatch.setattr(pa, "gather_sequence", whole_blocks)
+    _fails(pins.check_against_brute)
+
+
+def test_wrong_row_order_is_caught(monkeypatch):
+    real = pa.gather_sequence
+
+    def reversed_rows(cache, block_row, length, block_size):
+        n_blocks = -(-length // block_size)
+        blocks = [cache[int(block_row[j])][::-1] for j in range(n_blocks)]
+        return np.concatenate(blocks, axis=0)[:length] if blocks else real(cache, block_row, length, block_size)
+
+    monkeypatch.setattr(pa, "gather_sequence", reversed_rows)
+    _fails(pins.check_against_brute)
+
+
+def test_swapped_key_value_is_caught(monkeypatch):
+    real = pa.attention_one_sequence
+    monkeypatch.setattr(pa, "attention_one_sequence", lambda q, K, V, s, **kw: real(q, V, K, s, **kw))
+    _fails(pins.check_against_brute)
+
+
+def test_unnormalised_softmax_is_caught(monkeypatch):
+    real = pa.attention_one_sequence
+
+    def unnormalised(q, K, V, sm_scale, **kw):
+        out, lse = real(q, K, V, sm_scale)
+        return out * np.exp(lse - lse.max())[:, None], lse
+
+    monkeypatch.setattr(pa, "attention_one_sequence", unnormalised)
+    _fails(pins.check_against_brute)
+
+
+def test_wrong_largest_code_is_caught(monkeypatch):
+    real = oq.absmax_quantize
+    monkeypatch.setattr(qpins, "absmax_quantize", lambda v, bits, ft=np.float64: real(v, bits + 1, ft))
+    _fails(lambda: qpins.test_absmax_4bit_worked_example_float64(read_golden))
+
+
+def test_truncating_rounding_is_caught(monkeypatch):
+    monkeypatch.setattr(oq.np, "rint", np.trunc)
+    _fails(lambda: qpins.test_absmax_4bit_worked_example_float64(read_golden))
+
+
+def test_int8_scale_of_wrong_head_is_caught(monkeypatch):
+    real = pa.dequantize_rows
+
+    def head0_scale(rows, cache_dtype, row_scales=None, head_scales=None):
+        if cache_dtype == "int8":
+            row_scales = np.repeat(np.asarray(row_scales)[:, :1], rows.shape[1], axis=1)
+        return real(rows, cache_dtype, row_scales, head_scales)
+
+    monkeypatch.setattr(pa, "dequantize_rows", head0_scale)
+    _fails(lambda: pins.test_quantized_decode_is_attention_over_dequantized_rows("int8"))
