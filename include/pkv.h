@@ -1,0 +1,174 @@
+/*
+ * pkv - paged KV-cache decode attention for NVIDIA B200 (sm_100a).
+ *
+ * Plain C interface of libpkv.so.  Every pointer argument marked "device" is
+ * caller-owned device memory; the library allocates nothing, frees nothing and
+ * never synchronises the stream.  Work is enqueued on `stream` (a
+ * cudaStream_t passed as void*, NULL = legacy default stream).  Argument
+ * checks run on the host before anything is launched and return a status;
+ * nothing is launched when a call returns an error.
+ *
+ * Layouts (row-major, innermost last):
+ *   key / value (new rows)   [num_tokens, n_kv, head_dim]          act dtype
+ *   key_cache / value_cache  [num_blocks, block_size, n_kv, head_dim] cache dtype
+ *   query / out              [num_seqs, n_q, head_dim]             act dtype
+ *   block_tables             int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens             int32 [num_seqs]
+ *   slot_mapping             int64 [num_tokens]
+ *   k_scale / v_scale        INT8:     float [num_blocks, block_size, n_kv]
+ *                            FP8 E4M3: float [n_kv]
+ * A physical block holds the K (or V) rows of block_size consecutive tokens
+ * for all KV heads: "Chapter 18 - KV-Cache Optimization Strategies", How
+ * PagedAttention Works (Physical KV Block figure: [block_size, G, d_k]).
+ */
+#ifndef PKV_H
+#define PKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  PKV_F32 = 0,      /* IEEE float32 */
+  PKV_BF16 = 1,     /* bfloat16 */
+  PKV_INT8 = 2,     /* int8 codes, one float scale per (token, head); cache only */
+  PKV_FP8_E4M3 = 3  /* OCP E4M3 bytes, one float scale per KV head; cache only */
+} pkv_dtype;
+
+typedef enum {
+  PKV_OK = 0,
+  PKV_ERR_INVALID_ARG = 1, /* null pointer, negative size, misaligned pointer, bad combination */
+  PKV_ERR_UNSUPPORTED = 2, /* valid but not implemented: head_dim, block_size, dtype pair, group size */
+  PKV_ERR_WORKSPACE = 3,   /* workspace missing or smaller than pkv_paged_attention_workspace_size() */
+  PKV_ERR_CUDA = 4         /* a CUDA runtime / driver call or a launch failed */
+} pkv_status;
+
+/* Bits OR-ed by the kernels into the optional int32 *device_error word.  An
+ * offending entry is skipped (never dereferenced); results of the affected
+ * sequence are then unspecified.  Kernels never trap. */
+#define PKV_DEVERR_SLOT_RANGE 0x1   /* slot < -1 or slot >= num_blocks * block_size */
+#define PKV_DEVERR_BLOCK_RANGE 0x2  /* block table entry outside [0, num_blocks) */
+#define PKV_DEVERR_CONTEXT_LEN 0x4  /* context_len < 0, > max_context_len or > max_blocks_per_seq * block_size */
+#define PKV_DEVERR_TIMEOUT 0x8      /* a bounded wait inside a kernel gave up (~1 s) */
+
+/*
+ * Append new tokens' K/V rows into their cache slots (reshape_and_cache).
+ *
+ * "Chapter 18 - KV-Cache Optimization Strategies", How PagedAttention Works:
+ * new tokens fill the current block; the block table maps logical blocks to
+ * physical ones (KV-cache overview page t13_4, block-table paragraph).  Row t
+ * goes to row slot % block_size of physical block slot / block_size, where
+ * slot = slot_mapping[t]; slot -1 skips the row.
+ *
+ *   key, value          device, [num_tokens, n_kv, head_dim], act_dtype (F32 or BF16)
+ *   key_cache, value_cache device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
+ *   k_scale, v_scale    INT8: device, written, one scale per (slot, head);
+ *                       FP8_E4M3: device, read, one scale per KV head;
+ *                       F32/BF16: must be NULL
+ *   slot_mapping        device int64 [num_tokens]
+ *   device_error        optional device int32 (NULL = not reported)
+ *
+ * Cache dtype rules: F32 cache needs F32 rows and BF16 cache needs BF16 rows
+ * (bit copies).  INT8: per (token, head) absmax quantiser of "KV Cache
+ * Engineering for LLM Serving", section 8, at 8 bits in IEEE float32:
+ * scale = max|x| / 127, code = clamp(rint(x / scale), -127, 127) (ties to
+ * even); an all-zero row stores scale 0 and codes 0.  FP8_E4M3: code =
+ * E4M3(x / scale_h) rounded to nearest-even, saturating at +-448; scale_h == 0
+ * stores code 0.  head_dim must be 64, 128 or 256; pointers 16-byte aligned.
+ * Slots of one call must be distinct, and must not lie in blocks shared by
+ * several sequences (copy-on-write is the caller's job: Chapter 18, Prefix
+ * Caching).
+ */
+pkv_status pkv_kv_cache_write(const void* key, const void* value, void* key_cache, void* value_cache, float* k_scale,
+                              float* v_scale, const int64_t* slot_mapping, int64_t num_tokens, int n_kv, int head_dim,
+                              int block_size, int64_t num_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                              int32_t* device_error, void* stream);
+
+/*
+ * Bytes of device workspace pkv_paged_attention_decode needs for this shape on
+ * the current device (0 when it needs none, e.g. an F32 cache).  Returns
+ * (size_t)-1 when the shape is unsupported or the device cannot be queried.
+ */
+size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                          pkv_dtype cache_dtype);
+
+/*
+ * Single-token decode attention over a paged KV cache (PagedAttention).
+ *
+ * For sequence s and query head h (KV head kv = h / (n_q / n_kv), consecutive
+ * grouping: "KV Cache Engineering for LLM Serving", section 1), over the
+ * L = context_lens[s] cached tokens reached through block_tables[s]
+ * (KV-cache overview page t13_4, block-table paragraph):
+ *   score_p = sm_scale * <query[s,h,:], K_p[kv,:]>
+ *   out[s,h,:] = sum_p softmax(score)_p * V_p[kv,:]
+ *   lse_out[s,h] = log(sum_p exp(score_p))             (natural log; optional)
+ * K_p / V_p are dequantised for INT8 (code * scale[block,row,kv]) and
+ * FP8_E4M3 (value * scale[kv]) caches.  L == 0 gives out = 0, lse = -inf.
+ * Entries of block_tables past ceil(L / block_size) are never read, and rows of
+ * the last block past L never enter the softmax.
+ *
+ *   out                device, [num_seqs, n_q, head_dim], act_dtype
+ *   query              device, [num_seqs, n_q, head_dim], act_dtype
+ *   k_scale, v_scale   as for pkv_kv_cache_write (read only); NULL for F32/BF16
+ *   max_context_len    host upper bound of context_lens (sizes the launch; no
+ *                      device->host read happens)
+ *   lse_out            optional device float [num_seqs, n_q]
+ *   workspace          device scratch of workspace_bytes; zero-filled once by
+ *                      the caller before its first use (the kernels leave its
+ *                      counter region zeroed after each call).  Calls that may
+ *                      run concurrently need separate workspaces.
+ *
+ * Supported: block_size 16; act F32 with an F32 cache (head_dim 32..256, a
+ * multiple of 32); act BF16 with a BF16 cache (head_dim 64 or 128); act BF16
+ * or F32 with an INT8 or FP8_E4M3 cache (head_dim 128); n_q a multiple of n_kv
+ * with n_q / n_kv <= 64.  Pointers 16-byte aligned.
+ */
+pkv_status pkv_paged_attention_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                      const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                      int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                      float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                      void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream);
+
+/*
+ * Launch shape overrides for pkv_paged_attention_decode_ex (0 = automatic).
+ * num_ctas: persistent CTAs sharing the blocks of all (sequence, KV-head group)
+ * pairs; stages: depth of the shared-memory ring of K/V blocks; heads_per_cta:
+ * KV heads a CTA streams together (a divisor of n_kv).
+ */
+typedef struct {
+  int num_ctas;
+  int stages;
+  int heads_per_cta;
+} pkv_decode_tuning;
+
+/* Workspace bytes for pkv_paged_attention_decode_ex with the given tuning. */
+size_t pkv_paged_attention_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                             pkv_dtype cache_dtype, const pkv_decode_tuning* tuning);
+
+/* pkv_paged_attention_decode with explicit launch shape (tuning may be NULL). */
+pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                         const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                         int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                         int64_t num_blocks, float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                         float* lse_out, void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                         const pkv_decode_tuning* tuning, void* stream);
+
+/* Static text for a status code. */
+const char* pkv_status_string(pkv_status status);
+
+/* Text of the last CUDA error seen by this thread's failing call ("" if none). */
+const char* pkv_last_cuda_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int pkv_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H */

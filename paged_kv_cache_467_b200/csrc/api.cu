@@ -1,0 +1,182 @@
+// C ABI of libpkv: argument validation, launch planning and status codes.
+// Every check here runs on the host before anything is enqueued.
+#include <cuda_runtime.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "internal.h"
+
+namespace pkv {
+
+static thread_local char g_last_cuda_error[256] = "";
+
+pkv_status cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
+  return PKV_ERR_CUDA;
+}
+
+pkv_status driver_fail(int code, const char* where) {
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: driver error %d", where, code);
+  return PKV_ERR_CUDA;
+}
+
+int device_sm_count() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return v;
+}
+
+int device_smem_optin() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return -1;
+  return v;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+static bool valid_dtype(int d) { return d >= PKV_F32 && d <= PKV_FP8_E4M3; }
+
+// Shape rules of the decode kernels; PKV_OK when the tensor-core path or the
+// F32 path can run it.
+static pkv_status check_decode_shape(const DecodeShape& s) {
+  if (s.num_seqs < 0 || s.n_q <= 0 || s.n_kv <= 0 || s.head_dim <= 0 || s.block_size <= 0) return PKV_ERR_INVALID_ARG;
+  if (!valid_dtype(s.act) || !valid_dtype(s.cache)) return PKV_ERR_INVALID_ARG;
+  if (s.act != PKV_F32 && s.act != PKV_BF16) return PKV_ERR_INVALID_ARG;
+  if (s.n_q % s.n_kv != 0) return PKV_ERR_INVALID_ARG;
+  if (s.block_size != kBlockSize) return PKV_ERR_UNSUPPORTED;
+  if (s.n_q / s.n_kv > 64) return PKV_ERR_UNSUPPORTED;
+  switch (s.cache) {
+    case PKV_F32:
+      if (s.act != PKV_F32) return PKV_ERR_UNSUPPORTED;
+      if (s.head_dim % 32 != 0 || s.head_dim > 256) return PKV_ERR_UNSUPPORTED;
+      return PKV_OK;
+    case PKV_BF16:
+      if (s.act != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+      if (s.head_dim != 64 && s.head_dim != 128) return PKV_ERR_UNSUPPORTED;
+      return PKV_OK;
+    default:
+      if (s.head_dim != 128) return PKV_ERR_UNSUPPORTED;
+      return PKV_OK;
+  }
+}
+
+static size_t workspace_for(const DecodeShape& s, const pkv_decode_tuning* tuning) {
+  if (check_decode_shape(s) != PKV_OK) return (size_t)-1;
+  if (s.cache == PKV_F32 || s.num_seqs == 0) return 0;
+  TcPlan plan;
+  if (plan_tc(s, tuning, &plan) != PKV_OK) return (size_t)-1;
+  return plan.ws_total;
+}
+
+static pkv_status decode_impl(void* out, const void* query, const void* key_cache, const void* value_cache,
+                              const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                              int max_blocks_per_seq, const int32_t* context_lens, int max_context_len, int num_seqs,
+                              int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks, float sm_scale,
+                              pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out, void* workspace,
+                              size_t workspace_bytes, int32_t* device_error, const pkv_decode_tuning* tuning,
+                              void* stream) {
+  const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, act_dtype, cache_dtype};
+  pkv_status st = check_decode_shape(s);
+  if (st != PKV_OK) return st;
+  if (max_blocks_per_seq < 0 || max_context_len < 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (num_blocks * (int64_t)block_size > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_INVALID_ARG;
+  const bool quant = cache_dtype == PKV_INT8 || cache_dtype == PKV_FP8_E4M3;
+  if (quant && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale))) return PKV_ERR_INVALID_ARG;
+  if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
+  if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
+
+  TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
+           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error};
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  if (cache_dtype == PKV_F32) return launch_decode_f32(s, a, strm);
+  TcPlan plan;
+  st = plan_tc(s, tuning, &plan);
+  if (st != PKV_OK) return st;
+  if (!workspace || workspace_bytes < plan.ws_total || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+  return launch_tc(s, plan, a, strm);
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+pkv_status pkv_kv_cache_write(const void* key, const void* value, void* key_cache, void* value_cache, float* k_scale,
+                              float* v_scale, const int64_t* slot_mapping, int64_t num_tokens, int n_kv, int head_dim,
+                              int block_size, int64_t num_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                              int32_t* device_error, void* stream) {
+  if (num_tokens < 0 || n_kv <= 0 || head_dim <= 0 || block_size <= 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (!valid_dtype(act_dtype) || !valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
+  if (act_dtype != PKV_F32 && act_dtype != PKV_BF16) return PKV_ERR_INVALID_ARG;
+  if (cache_dtype == PKV_F32 && act_dtype != PKV_F32) return PKV_ERR_UNSUPPORTED;
+  if (cache_dtype == PKV_BF16 && act_dtype != PKV_BF16) return PKV_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return PKV_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PKV_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
+  if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+    return PKV_ERR_INVALID_ARG;
+  const bool quant = cache_dtype == PKV_INT8 || cache_dtype == PKV_FP8_E4M3;
+  if (quant && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+  if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
+  return launch_cache_write(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping, num_tokens, n_kv,
+                            head_dim, block_size, num_blocks, act_dtype, cache_dtype, device_error,
+                            static_cast<cudaStream_t>(stream));
+}
+
+size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                          pkv_dtype cache_dtype) {
+  const pkv_dtype act = cache_dtype == PKV_F32 ? PKV_F32 : PKV_BF16;
+  return workspace_for(DecodeShape{num_seqs, n_q, n_kv, head_dim, block_size, act, cache_dtype}, nullptr);
+}
+
+size_t pkv_paged_attention_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                             pkv_dtype cache_dtype, const pkv_decode_tuning* tuning) {
+  const pkv_dtype act = cache_dtype == PKV_F32 ? PKV_F32 : PKV_BF16;
+  return workspace_for(DecodeShape{num_seqs, n_q, n_kv, head_dim, block_size, act, cache_dtype}, tuning);
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                      const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                      int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                      int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                      float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                      void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream) {
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream);
+}
+
+pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                         const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                                         int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                         int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                         int64_t num_blocks, float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                         float* lse_out, void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                         const pkv_decode_tuning* tuning, void* stream) {
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream);
+}
+
+const char* pkv_status_string(pkv_status status) {
+  switch (status) {
+    case PKV_OK: return "ok";
+    case PKV_ERR_INVALID_ARG: return "invalid argument";
+    case PKV_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case PKV_ERR_WORKSPACE: return "workspace missing or too small";
+    case PKV_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+const char* pkv_last_cuda_error(void) { return g_last_cuda_error; }
+
+int pkv_version(void) { return 100; }
+
+}  // extern "C"

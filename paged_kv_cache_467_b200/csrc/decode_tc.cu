@@ -1,0 +1,781 @@
+// Paged decode attention on the tensor-core path (BF16, INT8 and FP8 E4M3 caches).
+//
+// What it computes: for every sequence s and query head h, softmax over the
+// s-th sequence's cached keys of sm_scale * <q_h, K_p> weighting the cached
+// values, with query heads grouped onto KV heads consecutively ("KV Cache
+// Engineering for LLM Serving", section 1) and the rows found through the
+// sequence's block table (KV-cache overview page t13_4, block-table paragraph;
+// "Chapter 18 - KV-Cache Optimization Strategies", How PagedAttention Works).
+//
+// How (B200 design, not from the pages):
+//  * Work unit = (sequence, group of HPC KV heads).  All units' 16-token blocks
+//    are laid end to end and every persistent CTA takes an equal contiguous
+//    share (split-K over context with no wave quantisation).  A unit cut by a
+//    share boundary is finished by whichever CTA writes its last piece: pieces
+//    carry (normalised o, log-sum-exp) and are merged in CTA order, so the
+//    result does not depend on timing.
+//  * One producer warp streams each block's K and V tiles of the CTA's KV heads
+//    into a ring of shared-memory stages with TMA (128-byte swizzle, tile
+//    [16 tokens x 128 bytes] per box), completing on mbarriers.  Block-table
+//    entries are fetched 32 at a time by the producer's lanes.
+//  * Consumer warp (KV head, chunk of 8 query heads): S^T[16 tok x 8 heads] =
+//    K_blk * Q^T with m16n8k16 MMAs (K from ldmatrix, Q held in registers), an
+//    online base-2 softmax with warp shuffles, then O^T[d x 8] += V^T * P^T
+//    (V^T via ldmatrix.trans, P^T via movmatrix).  INT8 / FP8 codes are
+//    converted to exact f16 in registers; the per-token INT8 scales multiply the
+//    scores and the probabilities, the per-head FP8 scales fold into constants.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "internal.h"
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+struct TcParams {
+  void* out;
+  const void* query;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  float* lse_out;
+  int* counters;
+  float* part_o;
+  float* part_lse;
+  int* err;
+  long long num_blocks;
+  int max_blocks_per_seq;
+  int cap_len;  // min(max_context_len, max_blocks_per_seq * 16)
+  int max_context_len;
+  int num_seqs, n_q, n_kv;
+  int G, QC, HPC, HG, NCW, stages, units;
+  float scale_log2;
+  int act_bf16;
+  uint32_t stage_bytes, tx_bytes;
+};
+
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Attended length of sequence s, clamped to what the launch and table cover.
+__device__ __forceinline__ int seq_len(const TcParams& p, int s, bool report) {
+  int L = __ldg(p.context_lens + s);
+  if (L < 0 || L > p.cap_len) {
+    if (report) flag_error(p.err, DEVERR_CONTEXT_LEN);
+    L = L < 0 ? 0 : p.cap_len;
+  }
+  return L;
+}
+
+// First index i in [0, n) with P[i] > x (n if none).
+__device__ __forceinline__ int upper_bound_smem(const int* P, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    int mid = (lo + hi) >> 1;
+    if (P[mid] <= x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// P[u] = number of blocks of units 0..u-1, P[units] = total.  All threads call.
+__device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
+  const int nthreads = blockDim.x;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5, nwarps = nthreads >> 5;
+  const int units = p.units;
+  const int per_t = (units + nthreads - 1) / nthreads;
+  const int u0 = min(t * per_t, units), u1 = min(u0 + per_t, units);
+  int local = 0;
+  for (int u = u0; u < u1; ++u) {
+    const int s = u / p.HG;
+    local += (seq_len(p, s, (u % p.HG) == 0) + kBlockSize - 1) / kBlockSize;
+  }
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int v = lane < nwarps ? wsum[lane] : 0;
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < nwarps) wsum[lane] = incl - v;
+  }
+  __syncthreads();
+  int run = wsum[warp] + x - local;
+  for (int u = u0; u < u1; ++u) {
+    P[u] = run;
+    run += (seq_len(p, u / p.HG, false) + kBlockSize - 1) / kBlockSize;
+  }
+  if (u1 == units && u0 < u1) P[units] = run;
+  if (units == 0 && t == 0) P[0] = 0;
+  __syncthreads();
+}
+
+template <int CACHE, int D>
+struct TcTraits {
+  static constexpr int kElem = CACHE == TC_BF16 ? 2 : 1;
+  static constexpr int kChunks = D * kElem / 128;  // 128-byte chunks per head row
+  static constexpr int kTile = kChunks * 2048;     // one head's 16-row tile
+  static constexpr int kSteps = D / 16;            // k-steps of Q.K and m-tiles of P.V
+};
+
+// Write one finished (or merged) row pair: heads 2c, 2c+1 of this lane.
+template <int CACHE, int D>
+__device__ __forceinline__ int d_of(int mt, int hi, int g) {
+  if constexpr (CACHE == TC_BF16) return mt * 16 + g + 8 * hi;
+  else return g * 16 + 2 * mt + hi;
+}
+
+template <int D>
+__device__ void merge_pieces(const TcParams& p, int u, int q_local, int c0, int npieces, bool c0_slot1, int per_unused,
+                             long long out_row, int lane) {
+  const int QH = p.HPC * p.G;
+  float M = -INFINITY;
+  for (int k = lane; k < npieces; k += 32) {
+    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
+    M = fmaxf(M, __ldcg(p.part_lse + ((size_t)(c0 + k) * 2 + slot) * QH + q_local));
+  }
+  M = warp_max(M);
+  constexpr int kPer = D / 32;
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int k = 0; k < npieces; ++k) {
+    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
+    const size_t piece = ((size_t)(c0 + k) * 2 + slot) * QH + q_local;
+    const float w = ex2(__ldcg(p.part_lse + piece) - M);
+    wsum += w;
+    const float* src = p.part_o + piece * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += w * __ldcg(src + e);
+    }
+  }
+  const float inv = 1.f / wsum;
+  if (p.act_bf16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) o[e] = __float2bfloat16_rn(acc[e] * inv);
+  } else {
+    float* o = reinterpret_cast<float*>(p.out) + out_row * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) o[e] = acc[e] * inv;
+  }
+  if (p.lse_out && lane == 0) p.lse_out[out_row] = (M + log2f(wsum)) * kLn2;
+}
+
+template <int CACHE, int D, int MAXW>
+__global__ void __launch_bounds__((MAXW + 1) * 32, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                     const TcParams p) {
+  using Tr = TcTraits<CACHE, D>;
+  constexpr int KS = Tr::kSteps;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * p.stage_bytes);
+  uint64_t* empty = full + p.stages;
+  int* wsum = reinterpret_cast<int*>(empty + p.stages);
+  int* P = wsum + 32;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int units = p.units;
+
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < p.stages; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], p.NCW);
+    }
+    fence_barrier_init();
+  }
+  if (warp == p.NCW && lane == 0) {
+    prefetch_tensormap(&kmap);
+    prefetch_tensormap(&vmap);
+  }
+  build_prefix(p, P, wsum);  // ends with __syncthreads()
+
+  const int total = P[units];
+  const int per = max(1, (total + (int)gridDim.x - 1) / (int)gridDim.x);
+  const int a = min((int)blockIdx.x * per, total);
+  const int b = min(a + per, total);
+
+  // ------------------------------------------------------------ producer
+  if (warp == p.NCW) {
+    if (a >= b) return;
+    int it = 0;
+    bool abort = false;
+    for (int base = a; base < b && !abort; base += 32) {
+      const int i = base + lane;
+      int phys = -1, hg = 0;
+      if (i < b) {
+        const int u = upper_bound_smem(P, units + 1, i) - 1;
+        const int s = u / p.HG;
+        hg = u - s * p.HG;
+        phys = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + (i - P[u]));
+        if (phys < 0 || (long long)phys >= p.num_blocks) {
+          flag_error(p.err, DEVERR_BLOCK_RANGE);
+          phys = -1;
+        }
+      }
+      const int n = min(32, b - base);
+      for (int k = 0; k < n; ++k) {
+        const int ph = __shfl_sync(0xffffffffu, phys, k);
+        const int hgk = __shfl_sync(0xffffffffu, hg, k);
+        int ok = 1;
+        if (lane == 0) {
+          const int stage = it % p.stages;
+          if (it >= p.stages && !mbar_wait(&empty[stage], ((it / p.stages) & 1) ^ 1)) {
+            flag_error(p.err, DEVERR_TIMEOUT);
+            ok = 0;
+          } else {
+            uint8_t* st = smem + (size_t)stage * p.stage_bytes;
+            mbar_arrive_expect_tx(&full[stage], p.tx_bytes);
+            const int row = ph * kBlockSize;  // -16 for a rejected entry: the TMA zero-fills it
+#pragma unroll 1
+            for (int hl = 0; hl < p.HPC; ++hl) {
+#pragma unroll
+              for (int ch = 0; ch < Tr::kChunks; ++ch) {
+                const int c1 = (hgk * p.HPC + hl) * Tr::kChunks + ch;
+                tma_load_3d(st + (hl * Tr::kChunks + ch) * 2048, &kmap, 0, c1, row, &full[stage]);
+                tma_load_3d(st + (p.HPC + hl) * Tr::kTile + ch * 2048, &vmap, 0, c1, row, &full[stage]);
+              }
+            }
+            if constexpr (CACHE == TC_INT8) {
+              const size_t sb = (size_t)(ph >= 0 ? ph : 0) * kBlockSize * p.n_kv;
+              const uint32_t bytes = 64u * p.n_kv;
+              uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
+              bulk_load(sc, p.k_scale + sb, bytes, &full[stage]);
+              bulk_load(sc + bytes, p.v_scale + sb, bytes, &full[stage]);
+            }
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { abort = true; break; }
+        ++it;
+      }
+    }
+    // Never leave with copies in flight: wait for the last stages issued.
+    if (lane == 0) {
+      for (int k = max(0, it - p.stages); k < it; ++k) mbar_wait(&full[k % p.stages], (k / p.stages) & 1);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int head_local = warp / p.QC;
+  const int qc = warp - head_local * p.QC;
+  const int g = lane >> 2, c = lane & 3;
+  const int QH = p.HPC * p.G;
+  const int qbase_local = head_local * p.G + qc * 8;  // q head index inside the unit
+  const bool head0_ok = qc * 8 + 2 * c < p.G, head1_ok = qc * 8 + 2 * c + 1 < p.G;
+
+  // CTA 0 writes the sequences with no tokens: out = 0, lse = -inf.
+  if (blockIdx.x == 0) {
+    for (int u = 0; u < units; ++u) {
+      if (P[u] != P[u + 1]) continue;
+      const int s = u / p.HG, hg = u - s * p.HG;
+      for (int n = 0; n < 8; ++n) {
+        if (qc * 8 + n >= p.G) break;
+        const long long row = (long long)s * p.n_q + hg * QH + qbase_local + n;
+        for (int dd = lane; dd < D; dd += 32) {
+          if (p.act_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[row * D + dd] = __float2bfloat16_rn(0.f);
+          else reinterpret_cast<float*>(p.out)[row * D + dd] = 0.f;
+        }
+        if (p.lse_out && lane == 0) p.lse_out[row] = -INFINITY;
+      }
+    }
+  }
+  if (a >= b) return;
+
+  // Per-lane ldmatrix offsets inside a head tile (128-byte swizzle: the 16-byte
+  // chunk j of row r lives at chunk j ^ (r & 7)).
+  const int k_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const int k_cadd = lane >> 4;
+  const int v_tok = (lane & 7) + ((lane >> 4) & 1) * 8;
+  const int v_cadd = (lane >> 3) & 1;
+  const int sw = lane & 7;
+
+  const int u_first = upper_bound_smem(P, units + 1, a) - 1;
+  int u = u_first;
+  int j = a - P[u];
+  int s = 0, hg = 0, L = 0;
+  float head_k_scale = 1.f, head_v_scale = 1.f;
+
+  uint32_t qf[KS][2];
+  float acc[KS][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  int it = 0;
+  for (int i = a; i < b; ++i, ++it) {
+    if (i == a || j == 0) {
+      // ---- unit start: load this warp's 8 query rows as MMA B fragments
+      s = u / p.HG;
+      hg = u - s * p.HG;
+      L = seq_len(p, s, false);
+      const int kv = hg * p.HPC + head_local;
+      const int qh = kv * p.G + qc * 8 + g;  // query head of fragment column g
+      const bool q_ok = qc * 8 + g < p.G;
+      const size_t qoff = ((size_t)s * p.n_q + qh) * D;
+      if constexpr (CACHE == TC_BF16) {
+        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(p.query) + qoff);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qf[ks][0] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c) / 2) : 0u;
+          qf[ks][1] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c + 8) / 2) : 0u;
+        }
+      } else {
+        // k-step ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+          float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+          if (q_ok) {
+            if (p.act_bf16) {
+              const uint2 w = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.query) + qoff + d0));
+              x0 = __uint_as_float(w.x << 16); x1 = __uint_as_float(w.x & 0xFFFF0000u);
+              x2 = __uint_as_float(w.y << 16); x3 = __uint_as_float(w.y & 0xFFFF0000u);
+            } else {
+              const float4 w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
+              x0 = w.x; x1 = w.y; x2 = w.z; x3 = w.w;
+            }
+          }
+          qf[ks][0] = pack_f16(x0, x1);
+          qf[ks][1] = pack_f16(x2, x3);
+        }
+        if constexpr (CACHE == TC_FP8) {
+          head_k_scale = __ldg(p.k_scale + kv);
+          head_v_scale = __ldg(p.v_scale + kv);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+
+    const int stage = it % p.stages;
+    if (!mbar_wait(&full[stage], (it / p.stages) & 1)) {
+      flag_error(p.err, DEVERR_TIMEOUT);
+      break;
+    }
+    const uint8_t* st = smem + (size_t)stage * p.stage_bytes;
+    const uint32_t kt = smem_addr(st + head_local * Tr::kTile);
+    const uint32_t vt = smem_addr(st + (p.HPC + head_local) * Tr::kTile);
+    const int valid = min(kBlockSize, L - j * kBlockSize);
+    const int t0 = g, t1 = g + 8;
+
+    // ---- S^T = K Q^T : [16 tokens x 8 heads]
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (CACHE == TC_BF16) {
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t af[4];
+        const int chunk = (ks & 3) * 2 + k_cadd;
+        ldmatrix_x4(af, kt + (ks >> 2) * 2048 + k_row * 128 + ((chunk ^ sw) << 4));
+        if (ks & 1) mma_bf16(sb, af, qf[ks][0], qf[ks][1]);
+        else mma_bf16(sa, af, qf[ks][0], qf[ks][1]);
+      }
+    } else {
+      // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each)
+      uint4 kr[2][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        kr[0][h] = lds128(kt + t0 * 128 + (((2 * c + h) ^ g) << 4));
+        kr[1][h] = lds128(kt + t1 * 128 + (((2 * c + h) ^ g) << 4));
+      }
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int h = ks >> 2, k = ks & 3;
+        const uint32_t w0 = (&kr[0][h].x)[k], w1 = (&kr[1][h].x)[k];
+        uint32_t af[4];
+        if constexpr (CACHE == TC_INT8) {
+          const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
+          af[0] = i8x2_to_f16x2(x0, 0x4140);
+          af[1] = i8x2_to_f16x2(x1, 0x4140);
+          af[2] = i8x2_to_f16x2(x0, 0x4342);
+          af[3] = i8x2_to_f16x2(x1, 0x4342);
+        } else {
+          af[0] = e4m3x2_to_f16x2(w0);
+          af[1] = e4m3x2_to_f16x2(w1);
+          af[2] = e4m3x2_to_f16x2(w0 >> 16);
+          af[3] = e4m3x2_to_f16x2(w1 >> 16);
+        }
+        if (ks & 1) mma_f16(sb, af, qf[ks][0], qf[ks][1]);
+        else mma_f16(sa, af, qf[ks][0], qf[ks][1]);
+      }
+    }
+
+    // ---- scale, mask, online softmax (base 2)
+    float sc0 = p.scale_log2, sc1 = p.scale_log2;
+    float vs0 = 1.f, vs1 = 1.f;
+    const int kvh = hg * p.HPC + head_local;
+    if constexpr (CACHE == TC_INT8) {
+      const float* ksm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile);
+      const float* vsm = ksm + kBlockSize * p.n_kv;
+      sc0 *= ksm[t0 * p.n_kv + kvh];
+      sc1 *= ksm[t1 * p.n_kv + kvh];
+      vs0 = vsm[t0 * p.n_kv + kvh];
+      vs1 = vsm[t1 * p.n_kv + kvh];
+    } else if constexpr (CACHE == TC_FP8) {
+      sc0 *= head_k_scale;
+      sc1 *= head_k_scale;
+    }
+    const bool ok0 = t0 < valid, ok1 = t1 < valid;
+    const float s00 = ok0 ? (sa[0] + sb[0]) * sc0 : -INFINITY;  // token g,   head 2c
+    const float s01 = ok0 ? (sa[1] + sb[1]) * sc0 : -INFINITY;  // token g,   head 2c+1
+    const float s10 = ok1 ? (sa[2] + sb[2]) * sc1 : -INFINITY;  // token g+8, head 2c
+    const float s11 = ok1 ? (sa[3] + sb[3]) * sc1 : -INFINITY;  // token g+8, head 2c+1
+    float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+    m0 = mn0;
+    m1 = mn1;
+    const float p00 = ex2(s00 - mn0), p01 = ex2(s01 - mn1);
+    const float p10 = ex2(s10 - mn0), p11 = ex2(s11 - mn1);
+    l0 = l0 * al0 + (p00 + p10);
+    l1 = l1 * al1 + (p01 + p11);
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+      acc[mt][0] *= al0;
+      acc[mt][1] *= al1;
+      acc[mt][2] *= al0;
+      acc[mt][3] *= al1;
+    }
+
+    // ---- O^T += V^T P^T
+    uint32_t pb0, pb1;
+    if constexpr (CACHE == TC_BF16) {
+      pb0 = movmatrix_trans(pack_bf16(p00, p01));
+      pb1 = movmatrix_trans(pack_bf16(p10, p11));
+    } else if constexpr (CACHE == TC_INT8) {
+      pb0 = movmatrix_trans(pack_f16(ok0 ? p00 * vs0 : 0.f, ok0 ? p01 * vs0 : 0.f));
+      pb1 = movmatrix_trans(pack_f16(ok1 ? p10 * vs1 : 0.f, ok1 ? p11 * vs1 : 0.f));
+    } else {
+      pb0 = movmatrix_trans(pack_f16(p00, p01));
+      pb1 = movmatrix_trans(pack_f16(p10, p11));
+    }
+    // token pairs of the A fragments: (2c, 2c+1) and (2c+8, 2c+9)
+    uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
+    const bool partial = valid < kBlockSize;
+    if (partial) {
+      mlo = (2 * c < valid ? 0x0000FFFFu : 0u) | (2 * c + 1 < valid ? 0xFFFF0000u : 0u);
+      mhi = (2 * c + 8 < valid ? 0x0000FFFFu : 0u) | (2 * c + 9 < valid ? 0xFFFF0000u : 0u);
+    }
+    if constexpr (CACHE == TC_BF16) {
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        uint32_t af[4];
+        const int chunk = (mt & 3) * 2 + v_cadd;
+        ldmatrix_x4_trans(af, vt + (mt >> 2) * 2048 + v_tok * 128 + ((chunk ^ sw) << 4));
+        af[0] &= mlo;
+        af[1] &= mlo;
+        af[2] &= mhi;
+        af[3] &= mhi;
+        mma_bf16(acc[mt], af, pb0, pb1);
+      }
+    } else {
+      // lane (g, c) reads chunk g of token rows 2c, 2c+1, 2c+8, 2c+9
+      const uint4 x0 = lds128(vt + (2 * c) * 128 + ((g ^ ((2 * c) & 7)) << 4));
+      const uint4 y0 = lds128(vt + (2 * c + 1) * 128 + ((g ^ ((2 * c + 1) & 7)) << 4));
+      const uint4 x1 = lds128(vt + (2 * c + 8) * 128 + ((g ^ ((2 * c + 8) & 7)) << 4));
+      const uint4 y1 = lds128(vt + (2 * c + 9) * 128 + ((g ^ ((2 * c + 9) & 7)) << 4));
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int wi = mt >> 1;
+        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+        uint32_t ta = prmt((&x0.x)[wi], (&y0.x)[wi], sel);
+        uint32_t tb = prmt((&x1.x)[wi], (&y1.x)[wi], sel);
+        uint32_t af[4];
+        if constexpr (CACHE == TC_INT8) {
+          ta ^= 0x80808080u;
+          tb ^= 0x80808080u;
+          af[0] = i8x2_to_f16x2(ta, 0x4140);
+          af[1] = i8x2_to_f16x2(ta, 0x4342);
+          af[2] = i8x2_to_f16x2(tb, 0x4140);
+          af[3] = i8x2_to_f16x2(tb, 0x4342);
+        } else {
+          af[0] = e4m3x2_to_f16x2(ta);
+          af[1] = e4m3x2_to_f16x2(ta >> 16);
+          af[2] = e4m3x2_to_f16x2(tb);
+          af[3] = e4m3x2_to_f16x2(tb >> 16);
+        }
+        af[0] &= mlo;
+        af[1] &= mlo;
+        af[2] &= mhi;
+        af[3] &= mhi;
+        mma_f16(acc[mt], af, pb0, pb1);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[stage]);
+
+    // ---- unit end: finish here, or hand a piece to the merge
+    const bool unit_end = (i + 1 == P[u + 1]);
+    if (unit_end || i + 1 == b) {
+      float lt0 = l0, lt1 = l1;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
+        lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
+      }
+      const float post = (CACHE == TC_FP8) ? head_v_scale : 1.f;
+      const float inv0 = post / lt0, inv1 = post / lt1;
+      const float lse0 = m0 + log2f(lt0), lse1 = m1 + log2f(lt1);
+      const bool contained = P[u] >= a && P[u + 1] <= b;
+      const long long row0 = (long long)s * p.n_q + hg * QH + qbase_local + 2 * c;  // head 2c of this lane
+      if (contained) {
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int dd = d_of<CACHE, D>(mt, hi, g);
+            const float v0 = acc[mt][2 * hi] * inv0, v1 = acc[mt][2 * hi + 1] * inv1;
+            if (p.act_bf16) {
+              __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out);
+              if (head0_ok) o[row0 * D + dd] = __float2bfloat16_rn(v0);
+              if (head1_ok) o[(row0 + 1) * D + dd] = __float2bfloat16_rn(v1);
+            } else {
+              float* o = reinterpret_cast<float*>(p.out);
+              if (head0_ok) o[row0 * D + dd] = v0;
+              if (head1_ok) o[(row0 + 1) * D + dd] = v1;
+            }
+          }
+        }
+        if (p.lse_out && g == 0) {
+          if (head0_ok) p.lse_out[row0] = lse0 * kLn2;
+          if (head1_ok) p.lse_out[row0 + 1] = lse1 * kLn2;
+        }
+      } else {
+        const int slot = (u == u_first) ? 0 : 1;
+        const size_t pbase = ((size_t)blockIdx.x * 2 + slot) * QH + qbase_local + 2 * c;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int dd = d_of<CACHE, D>(mt, hi, g);
+            if (head0_ok) __stcg(p.part_o + pbase * D + dd, acc[mt][2 * hi] * inv0);
+            if (head1_ok) __stcg(p.part_o + (pbase + 1) * D + dd, acc[mt][2 * hi + 1] * inv1);
+          }
+        }
+        if (g == 0) {
+          if (head0_ok) __stcg(p.part_lse + pbase, lse0);
+          if (head1_ok) __stcg(p.part_lse + pbase + 1, lse1);
+        }
+        __threadfence();
+        __syncwarp();
+        const int c0 = P[u] / per, c1 = (P[u + 1] - 1) / per;
+        const int npieces = c1 - c0 + 1;
+        int last = 0;
+        if (lane == 0) {
+          int* ctr = p.counters + (size_t)u * p.NCW + warp;
+          const int old = atomicAdd(ctr, 1);
+          last = (old == npieces - 1);
+          if (last) *ctr = 0;  // leave the counter zeroed for the next call
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          const bool c0_slot1 = (P[u] % per) != 0;
+          for (int n = 0; n < 8; ++n) {
+            if (qc * 8 + n >= p.G) break;
+            const long long row = (long long)s * p.n_q + hg * QH + qbase_local + n;
+            merge_pieces<D>(p, u, qbase_local + n, c0, npieces, c0_slot1, per, row, lane);
+          }
+        }
+      }
+    }
+    ++j;
+    if (unit_end) {
+      ++u;
+      while (u < units && P[u + 1] == P[u]) ++u;
+      j = 0;
+    }
+  }
+}
+
+// ----------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Rank-3 view of a cache pool [num_blocks * 16 rows][n_kv * head_dim * elem bytes]
+// as (128-byte chunk elements, chunk index, row), box = 1 chunk x 16 rows.
+static pkv_status make_kv_map(CUtensorMap* map, const void* base, int elem, int n_kv, int head_dim, int64_t rows) {
+  auto fn = encode_fn();
+  if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
+  const cuuint64_t row_bytes = (cuuint64_t)n_kv * head_dim * elem;
+  cuuint64_t dims[3] = {(cuuint64_t)(128 / elem), row_bytes / 128, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {128, row_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem), 1, (cuuint32_t)kBlockSize};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return driver_fail((int)r, "cuTensorMapEncodeTiled");
+  return PKV_OK;
+}
+
+template <int CACHE, int D, int MAXW>
+static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const TcParams& prm,
+                                 cudaStream_t stream) {
+  auto kern = decode_tc_kernel<CACHE, D, MAXW>;
+  static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
+  if ((int)plan.smem_bytes > configured_bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    configured_bytes = (int)plan.smem_bytes;
+  }
+  kern<<<plan.num_ctas, (plan.NCW + 1) * 32, plan.smem_bytes, stream>>>(km, vm, prm);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_tc_kernel launch");
+  return PKV_OK;
+}
+
+// Up to 8 consumer warps use the variant whose launch bound leaves ~220
+// registers per thread; wider CTAs take the 16-warp variant.
+template <int CACHE, int D>
+static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const TcParams& prm,
+                             cudaStream_t stream) {
+  if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, prm, stream);
+  return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, prm, stream);
+}
+
+pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream) {
+  const int elem = plan.cache_kind == TC_BF16 ? 2 : 1;
+  const int64_t rows = a.num_blocks * kBlockSize;
+  CUtensorMap km, vm;
+  pkv_status st = make_kv_map(&km, a.key_cache, elem, s.n_kv, s.head_dim, rows);
+  if (st != PKV_OK) return st;
+  st = make_kv_map(&vm, a.value_cache, elem, s.n_kv, s.head_dim, rows);
+  if (st != PKV_OK) return st;
+
+  TcParams prm;
+  prm.out = a.out;
+  prm.query = a.query;
+  prm.k_scale = a.k_scale;
+  prm.v_scale = a.v_scale;
+  prm.block_tables = a.block_tables;
+  prm.context_lens = a.context_lens;
+  prm.lse_out = a.lse_out;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  prm.counters = reinterpret_cast<int*>(ws + plan.ws_counters);
+  prm.part_o = reinterpret_cast<float*>(ws + plan.ws_part_o);
+  prm.part_lse = reinterpret_cast<float*>(ws + plan.ws_part_lse);
+  prm.err = a.device_error;
+  prm.num_blocks = a.num_blocks;
+  prm.max_blocks_per_seq = a.max_blocks_per_seq;
+  prm.max_context_len = a.max_context_len;
+  prm.cap_len = (int)std::min<int64_t>(a.max_context_len, (int64_t)a.max_blocks_per_seq * kBlockSize);
+  prm.num_seqs = s.num_seqs;
+  prm.n_q = s.n_q;
+  prm.n_kv = s.n_kv;
+  prm.G = plan.G;
+  prm.QC = plan.QC;
+  prm.HPC = plan.HPC;
+  prm.HG = plan.HG;
+  prm.NCW = plan.NCW;
+  prm.stages = plan.stages;
+  prm.units = plan.units;
+  prm.scale_log2 = (float)((double)a.sm_scale * 1.4426950408889634);
+  prm.act_bf16 = s.act == PKV_BF16;
+  prm.stage_bytes = plan.stage_bytes;
+  prm.tx_bytes = plan.tx_bytes;
+
+  if (plan.cache_kind == TC_BF16) {
+    if (s.head_dim == 64) return launch_one<TC_BF16, 64>(plan, km, vm, prm, stream);
+    return launch_one<TC_BF16, 128>(plan, km, vm, prm, stream);
+  }
+  if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, prm, stream);
+  return launch_one<TC_FP8, 128>(plan, km, vm, prm, stream);
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan) {
+  TcPlan pl{};
+  pl.cache_kind = s.cache == PKV_BF16 ? TC_BF16 : (s.cache == PKV_INT8 ? TC_INT8 : TC_FP8);
+  const int elem = pl.cache_kind == TC_BF16 ? 2 : 1;
+  pl.chunks = s.head_dim * elem / 128;
+  pl.G = s.n_q / s.n_kv;
+  pl.QC = (pl.G + 7) / 8;
+  const int want_hpc = tuning ? tuning->heads_per_cta : 0;
+  const size_t scale_bytes = pl.cache_kind == TC_INT8 ? 2 * 64 * (size_t)s.n_kv : 0;
+  if (want_hpc > 0) {
+    if (s.n_kv % want_hpc != 0 || want_hpc * pl.QC > kMaxConsumerWarps) return PKV_ERR_INVALID_ARG;
+    pl.HPC = want_hpc;
+  } else {
+    pl.HPC = 1;
+    for (int h = s.n_kv; h >= 1; --h) {
+      if (s.n_kv % h) continue;
+      const size_t stage = 2 * (size_t)h * pl.chunks * 2048 + scale_bytes;
+      if (h * pl.QC <= kMaxConsumerWarps && stage <= 64 * 1024) {
+        pl.HPC = h;
+        break;
+      }
+    }
+  }
+  if (pl.HPC * pl.QC > kMaxConsumerWarps) return PKV_ERR_UNSUPPORTED;
+  pl.HG = s.n_kv / pl.HPC;
+  pl.NCW = pl.HPC * pl.QC;
+  pl.units = s.num_seqs * pl.HG;
+  pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * pl.chunks * 2048 + scale_bytes);
+  pl.stage_bytes = (uint32_t)align_up(pl.tx_bytes, 1024);
+
+  const int sms = device_sm_count();
+  const int optin = device_smem_optin();
+  if (sms <= 0 || optin <= 0) return PKV_ERR_CUDA;
+  const size_t fixed = align_up(2 * 8 * kMaxStages + 32 * 4 + ((size_t)pl.units + 1) * 4, 16) + 1024;
+  const int want_stages = tuning ? tuning->stages : 0;
+  int stages = want_stages > 0 ? want_stages : (int)std::min<size_t>(kMaxStages, ((size_t)optin - fixed) / pl.stage_bytes);
+  if (stages < 2 || stages > kMaxStages) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
+  pl.stages = stages;
+  pl.smem_bytes = (size_t)stages * pl.stage_bytes + fixed;
+  if (pl.smem_bytes > (size_t)optin) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
+  // CTAs resident per SM from shared memory alone (228 KB per SM, 1 KB reserved per CTA).
+  const int per_sm = std::max(1, (int)(233472 / (pl.smem_bytes + 1024)));
+  const int want_ctas = tuning ? tuning->num_ctas : 0;
+  pl.num_ctas = want_ctas > 0 ? want_ctas : sms * per_sm;
+  const size_t QH = (size_t)pl.HPC * pl.G;
+  pl.ws_counters = 0;
+  pl.ws_part_o = align_up((size_t)pl.units * pl.NCW * 4, 256);
+  pl.ws_part_lse = align_up(pl.ws_part_o + (size_t)pl.num_ctas * 2 * QH * s.head_dim * 4, 256);
+  pl.ws_total = align_up(pl.ws_part_lse + (size_t)pl.num_ctas * 2 * QH * 4, 256);
+  *plan = pl;
+  return PKV_OK;
+}
+
+}  // namespace pkv

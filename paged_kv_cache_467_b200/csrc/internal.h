@@ -1,0 +1,74 @@
+// Host-side declarations shared by the .cu files of libpkv (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/pkv.h"
+
+namespace pkv {
+
+constexpr int kBlockSize = 16;
+constexpr int kMaxStages = 8;
+constexpr int kMaxConsumerWarps = 16;
+
+// Cache kinds of the tensor-core decode kernel.
+enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2 };
+
+struct DecodeShape {
+  int num_seqs, n_q, n_kv, head_dim, block_size;
+  pkv_dtype act, cache;
+};
+
+// Launch plan of the tensor-core decode kernel; a pure function of the shape,
+// the device's SM count / shared-memory limit and the tuning overrides.
+struct TcPlan {
+  int cache_kind;   // TcCache
+  int G, QC, HPC, HG, NCW;
+  int chunks;       // 128-byte row chunks per KV head row (head_dim * elem / 128)
+  int stages;
+  int num_ctas;
+  int units;        // num_seqs * HG
+  uint32_t stage_bytes, tx_bytes;
+  size_t smem_bytes;
+  size_t ws_counters, ws_part_o, ws_part_lse, ws_total;  // byte offsets / total
+};
+
+pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
+
+struct TcArgs {
+  void* out;
+  const void* query;
+  const void* key_cache;
+  const void* value_cache;
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  const int32_t* context_lens;
+  int max_context_len;
+  int64_t num_blocks;
+  float sm_scale;
+  float* lse_out;
+  void* workspace;
+  int32_t* device_error;
+};
+
+pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);
+
+pkv_status launch_decode_f32(const DecodeShape& s, const TcArgs& a, cudaStream_t stream);
+
+pkv_status launch_cache_write(const void* key, const void* value, void* key_cache, void* value_cache, float* k_scale,
+                              float* v_scale, const int64_t* slot_mapping, int64_t num_tokens, int n_kv, int head_dim,
+                              int block_size, int64_t num_blocks, pkv_dtype act, pkv_dtype cache, int32_t* device_error,
+                              cudaStream_t stream);
+
+// Records the CUDA error text for pkv_last_cuda_error() and returns PKV_ERR_CUDA.
+pkv_status cuda_fail(cudaError_t e, const char* where);
+pkv_status driver_fail(int code, const char* where);
+
+int device_sm_count();
+int device_smem_optin();
+
+}  // namespace pkv

@@ -1,0 +1,185 @@
+"""ctypes binding of libpkv.so: same names as the C ABI in include/pkv.h.
+
+Only argument marshalling happens here (dtype codes, raw pointers, the current
+CUDA stream); every step of the computation runs in the library's kernels.
+Importing this module raises when the library has not been built, so no caller
+can end up on a silent fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpkv.so")
+
+PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3 = 0, 1, 2, 3
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype", 3: "workspace missing or too small", 4: "CUDA error"}
+DEVERR_SLOT_RANGE, DEVERR_BLOCK_RANGE, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+
+_CACHE_DTYPES = {
+    "f32": PKV_F32,
+    "bf16": PKV_BF16,
+    "int8": PKV_INT8,
+    "fp8_e4m3": PKV_FP8_E4M3,
+}
+
+
+class PkvError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if detail:
+            msg += f" ({detail})"
+        super().__init__(msg)
+
+
+class DecodeTuning(ctypes.Structure):
+    _fields_ = [("num_ctas", ctypes.c_int), ("stages", ctypes.c_int), ("heads_per_cta", ctypes.c_int)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_467_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    lib.pkv_kv_cache_write.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i32, i32, vp, vp]
+    lib.pkv_kv_cache_write.restype = i32
+    lib.pkv_paged_attention_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.pkv_paged_attention_workspace_size.restype = sz
+    lib.pkv_paged_attention_workspace_size_ex.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(DecodeTuning)]
+    lib.pkv_paged_attention_workspace_size_ex.restype = sz
+    decode_args = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i64, f32, i32, i32, vp, vp, sz, vp]
+    lib.pkv_paged_attention_decode.argtypes = decode_args + [vp]
+    lib.pkv_paged_attention_decode.restype = i32
+    lib.pkv_paged_attention_decode_ex.argtypes = decode_args + [ctypes.POINTER(DecodeTuning), vp]
+    lib.pkv_paged_attention_decode_ex.restype = i32
+    lib.pkv_status_string.argtypes = [i32]
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    lib.pkv_last_cuda_error.argtypes = []
+    lib.pkv_last_cuda_error.restype = ctypes.c_char_p
+    lib.pkv_version.argtypes = []
+    lib.pkv_version.restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        detail = lib.pkv_last_cuda_error().decode() if status == 4 else ""
+        raise PkvError(status, where, detail)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpkv must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(device=None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def act_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return PKV_F32
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    raise TypeError(f"unsupported activation dtype {t.dtype}")
+
+
+def cache_code(t: torch.Tensor, cache_dtype: str | None = None) -> int:
+    if cache_dtype is not None:
+        return _CACHE_DTYPES[cache_dtype]
+    if t.dtype == torch.float32:
+        return PKV_F32
+    if t.dtype == torch.bfloat16:
+        return PKV_BF16
+    if t.dtype == torch.int8:
+        return PKV_INT8
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return PKV_FP8_E4M3
+    raise TypeError(f"unsupported cache dtype {t.dtype}")
+
+
+def kv_cache_write(key, value, key_cache, value_cache, slot_mapping, k_scale=None, v_scale=None, device_error=None):
+    """Append rows of ``key``/``value`` [T, n_kv, d] at ``slot_mapping`` [T] (int64)."""
+    T, n_kv, d = key.shape
+    num_blocks, block_size = key_cache.shape[0], key_cache.shape[1]
+    st = lib.pkv_kv_cache_write(
+        _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping),
+        T, n_kv, d, block_size, num_blocks, act_code(key), cache_code(key_cache), _ptr(device_error), _stream(key.device),
+    )
+    _check(st, "pkv_kv_cache_write")
+
+
+def paged_attention_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, cache_dtype: int, tuning=None) -> int:
+    if tuning is None:
+        n = lib.pkv_paged_attention_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, cache_dtype)
+    else:
+        n = lib.pkv_paged_attention_workspace_size_ex(num_seqs, n_q, n_kv, head_dim, block_size, cache_dtype, ctypes.byref(tuning))
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(2, "pkv_paged_attention_workspace_size")
+    return int(n)
+
+
+_ws_lock = threading.Lock()
+_workspaces: dict = {}
+
+
+def workspace_for(nbytes: int, device) -> torch.Tensor:
+    """Zero-filled scratch reused per (device, stream); grows when needed."""
+    key = (torch.device(device).index, _stream(device))
+    with _ws_lock:
+        ws = _workspaces.get(key)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+            _workspaces[key] = ws
+        return ws
+
+
+def paged_attention_decode(
+    out,
+    query,
+    key_cache,
+    value_cache,
+    block_tables,
+    context_lens,
+    max_context_len: int,
+    sm_scale: float | None = None,
+    k_scale=None,
+    v_scale=None,
+    lse_out=None,
+    workspace=None,
+    device_error=None,
+    tuning: DecodeTuning | None = None,
+):
+    """Decode attention of ``query`` [S, n_q, d] over a paged cache into ``out``."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ccode = cache_code(key_cache)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, tuning)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    args = [
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
+        float(sm_scale), act_code(query), ccode, _ptr(lse_out), _ptr(workspace), ws_bytes, _ptr(device_error),
+    ]
+    if tuning is None:
+        st = lib.pkv_paged_attention_decode(*args, _stream(query.device))
+    else:
+        st = lib.pkv_paged_attention_decode_ex(*args, ctypes.byref(tuning), _stream(query.device))
+    _check(st, "pkv_paged_attention_decode")
+    return out

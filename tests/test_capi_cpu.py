@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad
+arguments on the host before touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_467_b200 import build
+
+    build.build()
+    from paged_kv_cache_467_b200 import ops
+
+    return ops.lib
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "pkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert "pkv_kv_cache_write" in names and "pkv_paged_attention_decode" in names
+    raw = ctypes.CDLL(os.path.join(ROOT, "paged_kv_cache_467_b200", "libpkv.so"))
+    for n in names:
+        assert hasattr(raw, n), n
+
+
+def test_status_strings_and_version(lib):
+    assert lib.pkv_status_string(0) == b"ok"
+    assert lib.pkv_status_string(3) == b"workspace missing or too small"
+    assert lib.pkv_version() >= 100
+
+
+FAKE = 0x10000  # an aligned, never dereferenced address: validation fails before any launch
+
+
+def _write(lib, **kw):
+    args = dict(key=FAKE, value=FAKE, key_cache=FAKE, value_cache=FAKE, k_scale=None, v_scale=None, slots=FAKE,
+                T=4, n_kv=2, d=128, bs=16, nb=8, act=1, cache=1, err=None)
+    args.update(kw)
+    return lib.pkv_kv_cache_write(args["key"], args["value"], args["key_cache"], args["value_cache"], args["k_scale"],
+                                  args["v_scale"], args["slots"], args["T"], args["n_kv"], args["d"], args["bs"],
+                                  args["nb"], args["act"], args["cache"], args["err"], None)
+
+
+def test_cache_write_host_validation(lib):
+    assert _write(lib, T=0) == 0  # nothing to do
+    assert _write(lib, key=None) == 1
+    assert _write(lib, key=FAKE + 4) == 1  # misaligned
+    assert _write(lib, d=96) == 2
+    assert _write(lib, act=0, cache=1) == 2  # F32 rows into a BF16 cache
+    assert _write(lib, act=2) == 1  # int8 rows are not an activation dtype
+    assert _write(lib, cache=2) == 1  # INT8 cache needs scale arrays
+    assert _write(lib, k_scale=FAKE, v_scale=FAKE) == 1  # BF16 cache takes no scales
+    assert _write(lib, cache=7) == 1
+    assert _write(lib, n_kv=0) == 1
+
+
+def _decode(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, ks=None, vs=None, bt=FAKE, mb=8, cl=FAKE, mcl=100, S=2, nq=8, nkv=2,
+             d=128, bs=16, nb=16, scale=0.1, act=1, cache=1, lse=None, ws=FAKE, wsb=1 << 20, err=None)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["mb"],
+                                          a["cl"], a["mcl"], a["S"], a["nq"], a["nkv"], a["d"], a["bs"], a["nb"],
+                                          a["scale"], a["act"], a["cache"], a["lse"], a["ws"], a["wsb"], a["err"], None)
+
+
+def test_decode_host_validation(lib):
+    assert _decode(lib, S=0) == 0
+    assert _decode(lib, nq=6, nkv=4) == 1  # query heads not a multiple of KV heads
+    assert _decode(lib, bs=32) == 2
+    assert _decode(lib, d=96) == 2
+    assert _decode(lib, nq=130, nkv=2) == 2  # group of 65
+    assert _decode(lib, out=None) == 1
+    assert _decode(lib, kc=FAKE + 8) == 1
+    assert _decode(lib, ks=FAKE, vs=FAKE) == 1  # BF16 cache takes no scales
+    assert _decode(lib, cache=2) == 1  # INT8 without scales
+    assert _decode(lib, act=0, cache=1) == 2  # F32 query with a BF16 cache
+    assert _decode(lib, act=1, cache=0, d=64) == 2  # BF16 query with an F32 cache
+    assert _decode(lib, cache=2, ks=FAKE, vs=FAKE, d=64) == 2  # quantised caches need head_dim 128
+    assert _decode(lib, nb=1 << 28) == 2  # pool rows beyond int32
+    assert _decode(lib, mcl=-1) == 1
+    assert _decode(lib, mb=0) == 1
+
+
+def test_workspace_size_host_paths(lib):
+    # an F32 cache needs no workspace and no device query
+    assert lib.pkv_paged_attention_workspace_size(4, 8, 2, 64, 16, 0) == 0
+    # unsupported shapes report (size_t)-1
+    assert lib.pkv_paged_attention_workspace_size(4, 8, 2, 96, 16, 1) == ctypes.c_size_t(-1).value
+    if not torch.cuda.is_available():
+        # sizing the tensor-core path needs the device's SM count
+        assert lib.pkv_paged_attention_workspace_size(4, 8, 2, 128, 16, 1) == ctypes.c_size_t(-1).value
