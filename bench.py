@@ -1,0 +1,473 @@
+"""Benchmark of one paged decode step: cache append + decode attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--config NAME]
+
+A step appends one token per sequence (pkv_kv_cache_write) and runs decode
+attention over every sequence's paged cache (pkv_paged_attention_decode), for
+one layer of the workload.  Default workload: the Llama-3-8B-shaped decode
+step (batch 64, 32 query / 8 KV heads, head_dim 128, BF16 cache, block 16,
+context lengths uniform in [512, 4096], shuffled pool sized to fit exactly).
+
+Under torchrun every rank runs its own replica of the workload (sequences are
+independent: weak scaling, no collective on the data path); rank 0 prints one
+JSON line.  ``--impl reference`` times the CPU float64 oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s (% of HBM peak) and decode tokens/s per step"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--config", default="llama3_8b")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_467_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """DRAM bytes per decode launch from the committed ncu summary, or None when
+    the summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"decode_{config}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples taken while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {
+            "sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "reasons": sorted(reasons),
+            "samples": len(sm),
+        }
+
+
+# ----------------------------------------------------------------- oracle
+def oracle_step_sample(w, seqs, host_rows):
+    """One oracle step (append + decode) over the sampled sequences; returns KV bytes read."""
+    import numpy as np
+
+    import oracle
+
+    kv_bytes = 0
+    for s in seqs:
+        kc, vc, K, V, q = host_rows[s]
+        L = int(w.context_lens[s])
+        oracle.kv_cache_write(K[L - 1 : L], V[L - 1 : L], kc, vc, np.array([L - 1], dtype=np.int64))
+        nb = kc.shape[0]
+        oracle.paged_attention_decode(q, kc, vc, np.arange(nb, dtype=np.int32)[None], np.array([L]), w.sm_scale)
+        kv_bytes += L * w.n_kv * w.head_dim * 2 * 2
+    return kv_bytes
+
+
+def prepare_oracle_rows(w, seqs):
+    import numpy as np
+
+    import oracle
+
+    rows = {}
+    q = w.query()
+    for s in seqs:
+        L = int(w.context_lens[s])
+        nb = -(-L // w.block_size)
+        K, V = w.sequence_kv(s)
+        kc = np.zeros((nb, w.block_size, w.n_kv, w.head_dim))
+        vc = np.zeros_like(kc)
+        oracle.kv_cache_write(K[: L - 1], V[: L - 1], kc, vc, np.arange(L - 1, dtype=np.int64))
+        rows[s] = (kc, vc, K, V, q[s : s + 1])
+    return rows
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def time_oracle(w, budget_s: float, max_seqs: int | None = None):
+    """Time oracle steps on a bounded sample of the workload's sequences."""
+    order = list(range(w.num_seqs))
+    seqs, t_total, b_total = [], 0.0, 0
+    host = {}
+    for s in order:
+        if max_seqs is not None and len(seqs) >= max_seqs:
+            break
+        host.update(prepare_oracle_rows(w, [s]))
+        t0 = time.perf_counter()
+        b = oracle_step_sample(w, [s], host)
+        t_total += time.perf_counter() - t0
+        b_total += b
+        seqs.append(s)
+        if t_total >= budget_s:
+            break
+    return b_total, t_total, seqs
+
+
+def run_reference(args, rank, world):
+    from paged_kv_cache_467_b200 import workloads
+
+    if rank != 0:
+        return
+    w = workloads.CONFIGS[args.config]()
+    # every step: the oracle over a bounded sample of the workload (its first sequence)
+    per_step = 1
+    host = prepare_oracle_rows(w, list(range(per_step)))
+    for _ in range(args.warmup):
+        oracle_step_sample(w, range(per_step), host)
+    t0 = time.perf_counter()
+    b = 0
+    for _ in range(args.steps):
+        b += oracle_step_sample(w, range(per_step), host)
+    dt = time.perf_counter() - t0
+    gbs = b / dt / 1e9
+    cores = blas_threads()
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": gbs,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic",
+        "config": config_block(w, world),
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{per_step} of {w.num_seqs} sequences per step (append + float64 decode)"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def replica_workload(base, rank):
+    """Rank r's replica: the same shape with its own seed (sequences are independent)."""
+    from paged_kv_cache_467_b200 import workloads
+
+    if rank == 0:
+        return base
+    return workloads.make_workload(
+        base.name, seed=base.seed + 1000 * rank, context_lens=base.context_lens, n_q=base.n_q, n_kv=base.n_kv,
+        head_dim=base.head_dim, cache_dtype=base.cache_dtype, shared_prefix_tokens=base.shared_prefix_tokens,
+        outlier_fraction=0.01 if base.k_outlier_channels is not None else 0.0)
+
+
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of a list of floats over all ranks (identity at world 1)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
+def whole_job_gbs(bytes_per_rank, world, ms):
+    """Bytes all ranks processed divided by the slowest rank's time, in GB/s."""
+    return bytes_per_rank * world / (ms * 1e-3) / 1e9
+
+
+def config_block(w, world):
+    from paged_kv_cache_467_b200 import accounting
+
+    kv = accounting.decode_kv_bytes(w)
+    return {
+        "workload": w.name,
+        "batch": w.num_seqs,
+        "n_q": w.n_q,
+        "n_kv": w.n_kv,
+        "head_dim": w.head_dim,
+        "block_size": w.block_size,
+        "cache_dtype": w.cache_dtype,
+        "context_tokens": int(w.context_lens.astype("int64").sum()),
+        "kv_bytes_per_step_per_gpu": kv,
+        "l2": f"inputs larger than L2 ({kv / 2**20:.0f} MiB of KV per step vs 126 MiB L2)" if kv > L2_BYTES
+        else "L2 flushed between steps",
+        "parallelism": f"replicas x{world} (independent sequences per GPU)",
+    }
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_b200(args, rank, world, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from paged_kv_cache_467_b200 import accounting, ops, workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+
+    w = replica_workload(workloads.CONFIGS[args.config](), rank)
+    S, nq, nkv, d, bs = w.num_seqs, w.n_q, w.n_kv, w.head_dim, w.block_size
+    gen = torch.Generator(device=dev).manual_seed(1234 + rank)
+    shape = (w.num_blocks, bs, nkv, d)
+    # q/K/V ~ N(0,1) synthetic cache, filled on the device (the writer is exercised by the step's append)
+    if w.cache_dtype == "bf16":
+        kc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        vc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+        ks = vs = None
+    else:
+        kc = torch.empty(shape, device=dev, dtype=torch.int8 if w.cache_dtype == "int8" else torch.uint8)
+        vc = torch.empty_like(kc)
+        if w.cache_dtype == "int8":
+            ks = torch.empty(shape[:3], device=dev)
+            vs = torch.empty(shape[:3], device=dev)
+        else:
+            ks = torch.full((nkv,), 5.0 / 448, device=dev)
+            vs = torch.full((nkv,), 5.0 / 448, device=dev)
+        slots_all = torch.arange(w.num_blocks * bs, device=dev, dtype=torch.int64)
+        for c0 in range(0, slots_all.numel(), 1 << 20):
+            sl = slots_all[c0 : c0 + (1 << 20)]
+            kk = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+            vv = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+            ops.kv_cache_write(kk, vv, kc, vc, sl, ks, vs)
+    q = torch.randn((S, nq, d), device=dev, generator=gen).to(torch.bfloat16)
+    k_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    v_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    slots = torch.from_numpy(w.new_token_slots()).to(dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc))
+    ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    kv_bytes = accounting.decode_kv_bytes(w)
+
+    def step():
+        ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+        ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                   device_error=err)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---------------- device-resident timing
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    t_spin = time.perf_counter()
+    while time.perf_counter() - t_spin < 0.4:  # keep the GPU busy while the sampler starts
+        step()
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev_start, ev_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    ev_start.record(stream)
+    for k in range(args.steps):
+        ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+        att[k][0].record(stream)
+        ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                   device_error=err)
+        att[k][1].record(stream)
+    ev_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = ev_start.elapsed_time(ev_end) / args.steps
+    att_ms = sum(a.elapsed_time(b) for a, b in att) / args.steps
+    ms, att_ms = max_over_ranks([ms, att_ms], world, dev)
+    assert int(err.item()) == 0, f"device error flag {int(err.item())}"
+
+    # ---------------- end to end through the public API with host buffers
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_q, h_k, h_v, h_slots, h_bt, h_cl = pin(q), pin(k_new), pin(v_new), pin(slots), pin(bt), pin(cl)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+    d_slots, d_bt, d_cl = torch.empty_like(slots), torch.empty_like(bt), torch.empty_like(cl)
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_cl))
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_steps = min(args.steps, 500)
+
+    def e2e_step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_slots.copy_(h_slots, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_cl.copy_(h_cl, non_blocking=True)
+        ops.kv_cache_write(d_k, d_v, kc, vc, d_slots, ks, vs, err)
+        ops.paged_attention_decode(out, d_q, kc, vc, d_bt, d_cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                   device_error=err)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()  # the host reads the step's result
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], world, dev)[0]
+
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        value = whole_job_gbs(kv_bytes, world, ms)
+        achieved = kv_bytes / (att_ms * 1e-3) / 1e9
+        traffic = profiled_traffic(args.config)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": w.cache_dtype,
+            "data": "synthetic",
+            "config": config_block(w, world),
+            "tokens_per_s": S * world / (ms * 1e-3),
+            "pct_of_hbm_peak": 100.0 * value / world / peak,
+            "roofline": {
+                "bound": "hbm",
+                "achieved": achieved,
+                "peak": peak,
+                "unit": "GB/s",
+                "frac": achieved / peak,
+                "traffic": traffic,
+                "kernel": "decode_tc_kernel (pkv_paged_attention_decode)",
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "bytes_per_launch": kv_bytes,
+                "launch_ms": att_ms,
+            },
+            "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            b, t, seqs = time_oracle(w, budget_s=12.0)
+            line["cpu_baseline"] = {
+                "value": b / t / 1e9,
+                "unit": "GB/s",
+                "cores": blas_threads(),
+                "kind": "oracle",
+                "sample": f"{len(seqs)} of {w.num_seqs} sequences (append + float64 decode), {t:.1f} s",
+            }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_b200(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -117,9 +117,12 @@ size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int h
  *                      device->host read happens)
  *   lse_out            optional device float [num_seqs, n_q]
  *   workspace          device scratch of workspace_bytes; zero-filled once by
- *                      the caller before its first use (the kernels leave its
- *                      counter region zeroed after each call).  Calls that may
- *                      run concurrently need separate workspaces.
+ *                      the caller before its first use.  Its first 256 KiB hold
+ *                      merge counters at a fixed place for every shape, and each
+ *                      call leaves them zeroed, so one workspace serves calls of
+ *                      any shape in stream order.  Calls that may run
+ *                      concurrently need separate workspaces; after a call
+ *                      reports PKV_DEVERR_TIMEOUT, zero the workspace again.
  *
  * Supported: block_size 16; act F32 with an F32 cache (head_dim 32..256, a
  * multiple of 32); act BF16 with a BF16 cache (head_dim 64 or 128); act BF16

@@ -592,7 +592,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const int npieces = c1 - c0 + 1;
         int last = 0;
         if (lane == 0) {
-          int* ctr = p.counters + (size_t)u * p.NCW + warp;
+          // A split unit's last CTA (c1) is unique to it: the unit holds c1's first block.
+          int* ctr = p.counters + (size_t)c1 * kMaxConsumerWarps + warp;
           const int old = atomicAdd(ctr, 1);
           last = (old == npieces - 1);
           if (last) *ctr = 0;  // leave the counter zeroed for the next call
@@ -738,11 +739,11 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     if (s.n_kv % want_hpc != 0 || want_hpc * pl.QC > kMaxConsumerWarps) return PKV_ERR_INVALID_ARG;
     pl.HPC = want_hpc;
   } else {
+    // Two consumer warps per CTA (2 KV heads when the group fits one warp) and
+    // several CTAs per SM measured best: each SM then streams several units.
     pl.HPC = 1;
-    for (int h = s.n_kv; h >= 1; --h) {
-      if (s.n_kv % h) continue;
-      const size_t stage = 2 * (size_t)h * pl.chunks * 2048 + scale_bytes;
-      if (h * pl.QC <= kMaxConsumerWarps && stage <= 64 * 1024) {
+    for (int h = std::min(s.n_kv, 2); h >= 1; --h) {
+      if (s.n_kv % h == 0 && h * pl.QC <= 2) {
         pl.HPC = h;
         break;
       }
@@ -760,18 +761,35 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   if (sms <= 0 || optin <= 0) return PKV_ERR_CUDA;
   const size_t fixed = align_up(2 * 8 * kMaxStages + 32 * 4 + ((size_t)pl.units + 1) * 4, 16) + 1024;
   const int want_stages = tuning ? tuning->stages : 0;
-  int stages = want_stages > 0 ? want_stages : (int)std::min<size_t>(kMaxStages, ((size_t)optin - fixed) / pl.stage_bytes);
+  int stages = want_stages;
+  if (stages <= 0) {
+    // Deepest ring (up to 4 stages) that still lets 4 CTAs share an SM; fewer
+    // CTAs per SM only when even 2 stages do not fit.
+    stages = 2;
+    for (int per = kTargetCtasPerSm; per >= 1; --per) {
+      const size_t budget = (size_t)kSmemPerSm / per - 1024;
+      if (budget < fixed) continue;
+      const int fit = (int)std::min<size_t>(4, (budget - fixed) / pl.stage_bytes);
+      if (fit >= 2) {
+        stages = fit;
+        break;
+      }
+    }
+  }
   if (stages < 2 || stages > kMaxStages) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   pl.stages = stages;
   pl.smem_bytes = (size_t)stages * pl.stage_bytes + fixed;
   if (pl.smem_bytes > (size_t)optin) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
-  // CTAs resident per SM from shared memory alone (228 KB per SM, 1 KB reserved per CTA).
-  const int per_sm = std::max(1, (int)(233472 / (pl.smem_bytes + 1024)));
+  // CTAs resident per SM from shared memory alone (1 KB reserved per CTA).
+  const int per_sm = std::max(1, std::min(kTargetCtasPerSm, (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
   const int want_ctas = tuning ? tuning->num_ctas : 0;
   pl.num_ctas = want_ctas > 0 ? want_ctas : sms * per_sm;
+  if (pl.num_ctas > kMaxCtas) return want_ctas > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   const size_t QH = (size_t)pl.HPC * pl.G;
+  // Counters sit in a fixed region whatever the shape, so one zero-filled
+  // workspace can serve calls of different shapes.
   pl.ws_counters = 0;
-  pl.ws_part_o = align_up((size_t)pl.units * pl.NCW * 4, 256);
+  pl.ws_part_o = (size_t)kMaxCtas * kMaxConsumerWarps * 4;
   pl.ws_part_lse = align_up(pl.ws_part_o + (size_t)pl.num_ctas * 2 * QH * s.head_dim * 4, 256);
   pl.ws_total = align_up(pl.ws_part_lse + (size_t)pl.num_ctas * 2 * QH * 4, 256);
   *plan = pl;

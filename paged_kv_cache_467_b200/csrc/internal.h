@@ -12,6 +12,9 @@ namespace pkv {
 constexpr int kBlockSize = 16;
 constexpr int kMaxStages = 8;
 constexpr int kMaxConsumerWarps = 16;
+constexpr int kMaxCtas = 4096;          // upper bound of persistent CTAs per launch
+constexpr int kTargetCtasPerSm = 4;
+constexpr size_t kSmemPerSm = 233472;  // 228 KB of shared memory per SM
 
 // Cache kinds of the tensor-core decode kernel.
 enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2 };

@@ -157,6 +157,19 @@ def test_pool_permutation_is_bitwise_invisible(cache):
     assert np.array_equal(out, out2) and np.array_equal(lse, lse2)
 
 
+def test_workspace_reused_across_shapes():
+    ops = _ops()
+    # one zero-filled workspace, big enough for both shapes, used by both in turn
+    w1 = _wl([3000, 2500, 40], 64, 8, 128, seed=21)  # few units, long
+    w2 = _wl([300 + 13 * i for i in range(40)], 32, 8, 128, seed=22)  # many units
+    n = max(ops.paged_attention_workspace_size(w.num_seqs, w.n_q, w.n_kv, 128, 16, ops.PKV_BF16) for w in (w1, w2))
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    for w in (w1, w2, w1):
+        st = fill_gpu(w)
+        out, lse = run_decode(w, st, workspace=ws)
+        check_all(w, st, out, lse, rows=False)
+
+
 def test_empty_sequences():
     w = _wl([0, 40, 0, 17, 0], 16, 4, 128, seed=2)
     st = fill_gpu(w)
