@@ -363,8 +363,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           qf[ks][1] = pack_f16(x2, x3);
         }
         if constexpr (CACHE == TC_FP8) {
-          head_k_scale = __ldg(p.k_scale + kv);
-          head_v_scale = __ldg(p.v_scale + kv);
+          // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256)
+          head_k_scale = __ldg(p.k_scale + kv) * 256.f;
+          head_v_scale = __ldg(p.v_scale + kv) * 256.f;
         }
       }
 #pragma unroll
@@ -415,10 +416,11 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           af[2] = i8x2_to_f16x2(x0, 0x4342);
           af[3] = i8x2_to_f16x2(x1, 0x4342);
         } else {
-          af[0] = e4m3x2_to_f16x2(w0);
-          af[1] = e4m3x2_to_f16x2(w1);
-          af[2] = e4m3x2_to_f16x2(w0 >> 16);
-          af[3] = e4m3x2_to_f16x2(w1 >> 16);
+          // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, values / 256
+          af[0] = e4m3x2_hi_to_f16x2_div256(prmt(w0, 0u, 0x1404));
+          af[1] = e4m3x2_hi_to_f16x2_div256(prmt(w1, 0u, 0x1404));
+          af[2] = e4m3x2_hi_to_f16x2_div256(prmt(w0, 0u, 0x3424));
+          af[3] = e4m3x2_hi_to_f16x2_div256(prmt(w1, 0u, 0x3424));
         }
         if (ks & 1) mma_f16(sb, af, qf[ks][0], qf[ks][1]);
         else mma_f16(sa, af, qf[ks][0], qf[ks][1]);
@@ -507,22 +509,24 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         const int wi = mt >> 1;
-        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-        uint32_t ta = prmt((&x0.x)[wi], (&y0.x)[wi], sel);
-        uint32_t tb = prmt((&x1.x)[wi], (&y1.x)[wi], sel);
         uint32_t af[4];
         if constexpr (CACHE == TC_INT8) {
-          ta ^= 0x80808080u;
-          tb ^= 0x80808080u;
+          const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+          const uint32_t ta = prmt((&x0.x)[wi], (&y0.x)[wi], sel) ^ 0x80808080u;
+          const uint32_t tb = prmt((&x1.x)[wi], (&y1.x)[wi], sel) ^ 0x80808080u;
           af[0] = i8x2_to_f16x2(ta, 0x4140);
           af[1] = i8x2_to_f16x2(ta, 0x4342);
           af[2] = i8x2_to_f16x2(tb, 0x4140);
           af[3] = i8x2_to_f16x2(tb, 0x4342);
         } else {
-          af[0] = e4m3x2_to_f16x2(ta);
-          af[1] = e4m3x2_to_f16x2(ta >> 16);
-          af[2] = e4m3x2_to_f16x2(tb);
-          af[3] = e4m3x2_to_f16x2(tb >> 16);
+          // byte A of the token-2c row into bits [15:8], of the token-2c+1 row into [31:24]
+          const uint32_t A = 2 * (mt & 1);
+          const uint32_t s0 = ((4 + A) << 12) | ((4 + A) << 8) | (A << 4) | A;
+          const uint32_t s1 = s0 + 0x1111u;
+          af[0] = e4m3x2_hi_to_f16x2_div256(prmt((&x0.x)[wi], (&y0.x)[wi], s0));
+          af[1] = e4m3x2_hi_to_f16x2_div256(prmt((&x0.x)[wi], (&y0.x)[wi], s1));
+          af[2] = e4m3x2_hi_to_f16x2_div256(prmt((&x1.x)[wi], (&y1.x)[wi], s0));
+          af[3] = e4m3x2_hi_to_f16x2_div256(prmt((&x1.x)[wi], (&y1.x)[wi], s1));
         }
         af[0] &= mlo;
         af[1] &= mlo;

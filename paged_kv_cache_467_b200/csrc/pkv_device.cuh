@@ -160,10 +160,13 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t biased_word, uint32_t
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two E4M3 bytes (low 16 bits of w) -> f16x2 (exact: every E4M3 value is an f16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w16) {
-  __half2_raw r = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w16 & 0xFFFFu), __NV_E4M3);
-  return static_cast<uint32_t>(r.x) | (static_cast<uint32_t>(r.y) << 16);
+// Two E4M3 bytes held in bits [15:8] and [31:24] of t (other bits ignored) ->
+// f16x2 equal to the E4M3 values times 2^-8, exactly.  The E4M3 magnitude bits
+// EEEE.MMM moved to f16 bits [13:7] read as an f16 with exponent field EEEE and
+// mantissa MMM0000000: the exponent biases differ by 8 (15 vs 7), subnormals
+// included, so the f16 value is the E4M3 value scaled by 2^-8.
+__device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2_div256(uint32_t t) {
+  return ((t >> 1) & 0x3F803F80u) | (t & 0x80008000u);
 }
 
 __device__ __forceinline__ float warp_max(float v) {
