@@ -161,10 +161,45 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
                                          float* lse_out, void* workspace, size_t workspace_bytes, int32_t* device_error,
                                          const pkv_decode_tuning* tuning, void* stream);
 
+/*
+ * pkv_paged_attention_decode for callers that cannot allocate device memory.
+ * This entry point has no counterpart in the paper; it exists for the callers
+ * of this library.
+ *
+ * Some callers cannot give the library a workspace: a library loaded into a
+ * host runtime that owns every device allocation and offers plug-ins no
+ * allocator, or a serving loop that must never call cudaMalloc because it can
+ * synchronise the device.  This call takes the same arguments as
+ * pkv_paged_attention_decode minus the workspace and runs the same kernels.
+ * Its scratch is a 16 MiB array that is part of libpkv itself.  Every GPU that
+ * loads the library holds that array until the process exits.  The call itself
+ * allocates nothing.
+ *
+ *   - Shapes needing more scratch than 16 MiB (see
+ *     pkv_paged_attention_workspace_size) are rejected with PKV_ERR_WORKSPACE
+ *     before anything is launched; pkv_last_cuda_error() then says how many
+ *     bytes the shape needs.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress).  Make that first call before any stream capture
+ *     on that device.
+ *   - Every call on a device shares the one array.  Each call clears the array's
+ *     merge counters (cudaMemsetAsync on `stream`) before launching.  Calls whose
+ *     work can overlap on the GPU (different streams, no ordering between them)
+ *     race on the array and give wrong results; keep such calls in one stream.
+ */
+pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const void* key_cache,
+                                             const void* value_cache, const float* k_scale, const float* v_scale,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                             int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                             float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                             float* lse_out, int32_t* device_error, void* stream);
+
 /* Static text for a status code. */
 const char* pkv_status_string(pkv_status status);
 
-/* Text of the last CUDA error seen by this thread's failing call ("" if none). */
+/* Text describing this thread's last failing CUDA call, or the last scratch-size
+ * rejection of pkv_paged_attention_decode_static ("" if none). */
 const char* pkv_last_cuda_error(void);
 
 /* Library version: major * 10000 + minor * 100 + patch. */

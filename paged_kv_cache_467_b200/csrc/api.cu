@@ -1,6 +1,7 @@
 // C ABI of libpkv: argument validation, launch planning and status codes.
 // Every check here runs on the host before anything is enqueued.
 #include <cuda_runtime.h>
+#include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -13,6 +14,13 @@ static thread_local char g_last_cuda_error[256] = "";
 pkv_status cuda_fail(cudaError_t e, const char* where) {
   snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", where, cudaGetErrorString(e));
   return PKV_ERR_CUDA;
+}
+
+void note_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_cuda_error, sizeof(g_last_cuda_error), fmt, ap);
+  va_end(ap);
 }
 
 pkv_status driver_fail(int code, const char* where) {

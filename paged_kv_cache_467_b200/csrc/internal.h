@@ -70,6 +70,8 @@ pkv_status launch_cache_write(const void* key, const void* value, void* key_cach
 // Records the CUDA error text for pkv_last_cuda_error() and returns PKV_ERR_CUDA.
 pkv_status cuda_fail(cudaError_t e, const char* where);
 pkv_status driver_fail(int code, const char* where);
+// Sets the text pkv_last_cuda_error() returns for this thread.
+void note_error(const char* fmt, ...);
 
 int device_sm_count();
 int device_smem_optin();

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attention_decode.restype = i32
     lib.pkv_paged_attention_decode_ex.argtypes = decode_args + [ctypes.POINTER(DecodeTuning), vp]
     lib.pkv_paged_attention_decode_ex.restype = i32
+    lib.pkv_paged_attention_decode_static.argtypes = decode_args[:20] + [vp, vp]
+    lib.pkv_paged_attention_decode_static.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_cuda_error.argtypes = []
@@ -182,4 +184,23 @@ def paged_attention_decode(
     else:
         st = lib.pkv_paged_attention_decode_ex(*args, ctypes.byref(tuning), _stream(query.device))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_static(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
+                                  sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None,
+                                  device_error=None):
+    """pkv_paged_attention_decode_static: decode with the library's own scratch (no workspace argument)."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    st = lib.pkv_paged_attention_decode_static(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
+        float(sm_scale), act_code(query), cache_code(key_cache), _ptr(lse_out), _ptr(device_error),
+        _stream(query.device),
+    )
+    if st != 0:
+        raise PkvError(st, "pkv_paged_attention_decode_static", lib.pkv_last_cuda_error().decode())
     return out
