@@ -60,6 +60,8 @@ struct TcParams {
 };
 
 constexpr float kLn2 = 0.6931471805599453f;
+// Slack (log2 units) of the running softmax maximum before it is moved.
+constexpr float kLazyLog2 = 8.f;
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -143,46 +145,73 @@ __device__ __forceinline__ int d_of(int mt, int hi, int g) {
   else return g * 16 + 2 * mt + hi;
 }
 
+// Merge the pieces of one unit for this warp's query heads (up to 8).  Lane
+// owns dims [lane * D/32, (lane + 1) * D/32) of every head, so all loads of one
+// piece are independent and each piece costs about one L2 round trip.  Pieces
+// are combined in CTA order: M = max lse_k, w_k = 2^(lse_k - M),
+// o = sum w_k o_k / sum w_k, lse = M + log2(sum w_k) (base-2 log-sum-exp).
 template <int D>
-__device__ void merge_pieces(const TcParams& p, int u, int q_local, int c0, int npieces, bool c0_slot1, int per_unused,
-                             long long out_row, int lane) {
+__device__ void merge_pieces(const TcParams& p, int qbase_local, int nh, int c0, int npieces, bool c0_slot1,
+                             long long out_row0, int lane) {
   const int QH = p.HPC * p.G;
-  float M = -INFINITY;
-  for (int k = lane; k < npieces; k += 32) {
-    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-    M = fmaxf(M, __ldcg(p.part_lse + ((size_t)(c0 + k) * 2 + slot) * QH + q_local));
-  }
-  M = warp_max(M);
   constexpr int kPer = D / 32;
-  float acc[kPer];
+  float M[8], wsum[8], acc[8][kPer];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
+  for (int n = 0; n < 8; ++n) {
+    M[n] = -INFINITY;
+    wsum[n] = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[n][e] = 0.f;
+  }
+#pragma unroll 1
   for (int k = 0; k < npieces; ++k) {
     const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-    const size_t piece = ((size_t)(c0 + k) * 2 + slot) * QH + q_local;
-    const float w = ex2(__ldcg(p.part_lse + piece) - M);
-    wsum += w;
-    const float* src = p.part_o + piece * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-    } else {
+    const float* lse = p.part_lse + ((size_t)(c0 + k) * 2 + slot) * QH + qbase_local;
 #pragma unroll
-      for (int e = 0; e < kPer; ++e) acc[e] += w * __ldcg(src + e);
+    for (int n = 0; n < 8; ++n)
+      if (n < nh) M[n] = fmaxf(M[n], __ldcg(lse + n));
+  }
+#pragma unroll 1
+  for (int k = 0; k < npieces; ++k) {
+    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
+    const size_t piece = ((size_t)(c0 + k) * 2 + slot) * QH + qbase_local;
+    const float* lse = p.part_lse + piece;
+    const float* src = p.part_o + piece * D + lane * kPer;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+      if (n < nh) {
+        const float w = ex2(__ldcg(lse + n) - M[n]);
+        wsum[n] += w;
+        if constexpr (kPer == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)n * D));
+          acc[n][0] += w * v.x;
+          acc[n][1] += w * v.y;
+          acc[n][2] += w * v.z;
+          acc[n][3] += w * v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src + (size_t)n * D));
+          acc[n][0] += w * v.x;
+          acc[n][1] += w * v.y;
+        }
+      }
     }
   }
-  const float inv = 1.f / wsum;
-  if (p.act_bf16) {
-    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + out_row * D + lane * kPer;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) o[e] = __float2bfloat16_rn(acc[e] * inv);
-  } else {
-    float* o = reinterpret_cast<float*>(p.out) + out_row * D + lane * kPer;
+  for (int n = 0; n < 8; ++n) {
+    if (n >= nh) break;
+    const long long row = out_row0 + n;
+    const float inv = 1.f / wsum[n];
+    if (p.act_bf16) {
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * D + lane * kPer;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) o[e] = acc[e] * inv;
+      for (int e = 0; e < kPer; ++e) o[e] = __float2bfloat16_rn(acc[n][e] * inv);
+    } else {
+      float* o = reinterpret_cast<float*>(p.out) + row * D + lane * kPer;
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) o[e] = acc[n][e] * inv;
+    }
+    if (p.lse_out && lane == 0) p.lse_out[row] = (M[n] + log2f(wsum[n])) * kLn2;
   }
-  if (p.lse_out && lane == 0) p.lse_out[out_row] = (M + log2f(wsum)) * kLn2;
 }
 
 template <int CACHE, int D, int MAXW>
@@ -314,6 +343,19 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const int v_tok = (lane & 7) + ((lane >> 4) & 1) * 8;
   const int v_cadd = (lane >> 3) & 1;
   const int sw = lane & 7;
+  // Byte offset of this lane's first 16-byte piece inside a head tile.  The
+  // swizzle XORs address bits [6:4] with the row's low bits, so the piece for
+  // chunk (base ^ x) sits at offset koff ^ (x << 4): one XOR per access.
+  //  bf16: ldmatrix rows k_row / v_tok, chunk pair (ks & 3) * 2 (+ lane's half)
+  //  int8/fp8: K rows g (+8 rows = +1024 B), chunks 2c (+1); V rows 2c (+1, +8, +9), chunk g
+  uint32_t koff, voff;
+  if constexpr (CACHE == TC_BF16) {
+    koff = k_row * 128 + ((k_cadd ^ sw) << 4);
+    voff = v_tok * 128 + ((v_cadd ^ sw) << 4);
+  } else {
+    koff = g * 128 + (((2 * c) ^ g) << 4);
+    voff = (2 * c) * 128 + ((g ^ (2 * c)) << 4);
+  }
 
   const int u_first = upper_bound_smem(P, units + 1, a) - 1;
   int u = u_first;
@@ -325,49 +367,79 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   float acc[KS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
+  // Query words of a unit as loaded (bf16 pairs) and the FP8 head scales.
+  uint32_t qraw[KS][2];
+  float raw_k_scale = 1.f, raw_v_scale = 1.f;
+  auto fetch_query = [&](int uu) {
+    const int ss = uu / p.HG, hh = uu - ss * p.HG;
+    const int kv = hh * p.HPC + head_local;
+    const bool q_ok = qc * 8 + g < p.G;
+    const size_t qoff = ((size_t)ss * p.n_q + kv * p.G + qc * 8 + g) * D;  // query head of fragment column g
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(p.query) + qoff);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      if constexpr (CACHE == TC_BF16) {
+        // MMA B fragment: dims ks*16 + 2c, +1 and ks*16 + 2c + 8, +9
+        qraw[ks][0] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c) / 2) : 0u;
+        qraw[ks][1] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c + 8) / 2) : 0u;
+      } else {
+        // k-step ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
+        const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+        const uint2 w = q_ok ? __ldg(reinterpret_cast<const uint2*>(q32 + d0 / 2)) : make_uint2(0u, 0u);
+        qraw[ks][0] = w.x;
+        qraw[ks][1] = w.y;
+      }
+    }
+    if constexpr (CACHE == TC_FP8) {
+      // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256)
+      raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
+      raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
+    }
+  };
+
   int it = 0;
   for (int i = a; i < b; ++i, ++it) {
     if (i == a || j == 0) {
-      // ---- unit start: load this warp's 8 query rows as MMA B fragments
+      // ---- unit start: this warp's 8 query rows as MMA B fragments
       s = u / p.HG;
       hg = u - s * p.HG;
       L = seq_len(p, s, false);
-      const int kv = hg * p.HPC + head_local;
-      const int qh = kv * p.G + qc * 8 + g;  // query head of fragment column g
-      const bool q_ok = qc * 8 + g < p.G;
-      const size_t qoff = ((size_t)s * p.n_q + qh) * D;
       if constexpr (CACHE == TC_BF16) {
-        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(p.query) + qoff);
+        fetch_query(u);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
-          qf[ks][0] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c) / 2) : 0u;
-          qf[ks][1] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c + 8) / 2) : 0u;
+          qf[ks][0] = qraw[ks][0];
+          qf[ks][1] = qraw[ks][1];
         }
       } else {
-        // k-step ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
+        if (p.act_bf16) {
+          fetch_query(u);
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
-          float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
-          if (q_ok) {
-            if (p.act_bf16) {
-              const uint2 w = __ldg(reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(p.query) + qoff + d0));
-              x0 = __uint_as_float(w.x << 16); x1 = __uint_as_float(w.x & 0xFFFF0000u);
-              x2 = __uint_as_float(w.y << 16); x3 = __uint_as_float(w.y & 0xFFFF0000u);
-            } else {
-              const float4 w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
-              x0 = w.x; x1 = w.y; x2 = w.z; x3 = w.w;
-            }
+          for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = pack_f16(__uint_as_float(qraw[ks][0] << 16), __uint_as_float(qraw[ks][0] & 0xFFFF0000u));
+            qf[ks][1] = pack_f16(__uint_as_float(qraw[ks][1] << 16), __uint_as_float(qraw[ks][1] & 0xFFFF0000u));
           }
-          qf[ks][0] = pack_f16(x0, x1);
-          qf[ks][1] = pack_f16(x2, x3);
-        }
-        if constexpr (CACHE == TC_FP8) {
-          // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256)
-          head_k_scale = __ldg(p.k_scale + kv) * 256.f;
-          head_v_scale = __ldg(p.v_scale + kv) * 256.f;
+        } else {
+          // float32 queries: loaded and rounded to f16 here (not prefetched)
+          const int kv = hg * p.HPC + head_local;
+          const bool q_ok = qc * 8 + g < p.G;
+          const size_t qoff = ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q_ok) w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
+            qf[ks][0] = pack_f16(w.x, w.y);
+            qf[ks][1] = pack_f16(w.z, w.w);
+          }
+          if constexpr (CACHE == TC_FP8) {
+            raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
+            raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
+          }
         }
       }
+      head_k_scale = raw_k_scale;
+      head_v_scale = raw_v_scale;
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
@@ -391,8 +463,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t af[4];
-        const int chunk = (ks & 3) * 2 + k_cadd;
-        ldmatrix_x4(af, kt + (ks >> 2) * 2048 + k_row * 128 + ((chunk ^ sw) << 4));
+        ldmatrix_x4(af, kt + (koff ^ ((ks & 3) << 5)) + (ks >> 2) * 2048);
         if (ks & 1) mma_bf16(sb, af, qf[ks][0], qf[ks][1]);
         else mma_bf16(sa, af, qf[ks][0], qf[ks][1]);
       }
@@ -401,8 +472,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       uint4 kr[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        kr[0][h] = lds128(kt + t0 * 128 + (((2 * c + h) ^ g) << 4));
-        kr[1][h] = lds128(kt + t1 * 128 + (((2 * c + h) ^ g) << 4));
+        kr[0][h] = lds128(kt + (koff ^ (h << 4)));
+        kr[1][h] = lds128(kt + (koff ^ (h << 4)) + 1024);
       }
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
@@ -447,27 +518,35 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     const float s01 = ok0 ? (sa[1] + sb[1]) * sc0 : -INFINITY;  // token g,   head 2c+1
     const float s10 = ok1 ? (sa[2] + sb[2]) * sc1 : -INFINITY;  // token g+8, head 2c
     const float s11 = ok1 ? (sa[3] + sb[3]) * sc1 : -INFINITY;  // token g+8, head 2c+1
+    // The reference max m of each head moves only when some score exceeds it by
+    // more than kLazyLog2, so probabilities stay <= 2^kLazyLog2 and most blocks
+    // skip the cross-lane max and the rescale of the accumulators; the final
+    // o / l and lse = m + log2(l) do not depend on which m was used.
     float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
+    if (__any_sync(0xffffffffu, mx0 > m0 + kLazyLog2 || mx1 > m1 + kLazyLog2)) {
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-    const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const float p00 = ex2(s00 - mn0), p01 = ex2(s01 - mn1);
-    const float p10 = ex2(s10 - mn0), p11 = ex2(s11 - mn1);
-    l0 = l0 * al0 + (p00 + p10);
-    l1 = l1 * al1 + (p01 + p11);
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= al0;
+      l1 *= al1;
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt) {
-      acc[mt][0] *= al0;
-      acc[mt][1] *= al1;
-      acc[mt][2] *= al0;
-      acc[mt][3] *= al1;
+      for (int mt = 0; mt < KS; ++mt) {
+        acc[mt][0] *= al0;
+        acc[mt][1] *= al1;
+        acc[mt][2] *= al0;
+        acc[mt][3] *= al1;
+      }
     }
+    const float p00 = ex2(s00 - m0), p01 = ex2(s01 - m1);
+    const float p10 = ex2(s10 - m0), p11 = ex2(s11 - m1);
+    l0 += p00 + p10;
+    l1 += p01 + p11;
 
     // ---- O^T += V^T P^T
     uint32_t pb0, pb1;
@@ -492,8 +571,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         uint32_t af[4];
-        const int chunk = (mt & 3) * 2 + v_cadd;
-        ldmatrix_x4_trans(af, vt + (mt >> 2) * 2048 + v_tok * 128 + ((chunk ^ sw) << 4));
+        ldmatrix_x4_trans(af, vt + (voff ^ ((mt & 3) << 5)) + (mt >> 2) * 2048);
         af[0] &= mlo;
         af[1] &= mlo;
         af[2] &= mhi;
@@ -502,10 +580,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       }
     } else {
       // lane (g, c) reads chunk g of token rows 2c, 2c+1, 2c+8, 2c+9
-      const uint4 x0 = lds128(vt + (2 * c) * 128 + ((g ^ ((2 * c) & 7)) << 4));
-      const uint4 y0 = lds128(vt + (2 * c + 1) * 128 + ((g ^ ((2 * c + 1) & 7)) << 4));
-      const uint4 x1 = lds128(vt + (2 * c + 8) * 128 + ((g ^ ((2 * c + 8) & 7)) << 4));
-      const uint4 y1 = lds128(vt + (2 * c + 9) * 128 + ((g ^ ((2 * c + 9) & 7)) << 4));
+      const uint4 x0 = lds128(vt + voff);
+      const uint4 y0 = lds128(vt + (voff ^ 16) + 128);
+      const uint4 x1 = lds128(vt + voff + 1024);
+      const uint4 y1 = lds128(vt + (voff ^ 16) + 1152);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
         const int wi = mt >> 1;
@@ -606,11 +684,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         if (last) {
           __threadfence();
           const bool c0_slot1 = (P[u] % per) != 0;
-          for (int n = 0; n < 8; ++n) {
-            if (qc * 8 + n >= p.G) break;
-            const long long row = (long long)s * p.n_q + hg * QH + qbase_local + n;
-            merge_pieces<D>(p, u, qbase_local + n, c0, npieces, c0_slot1, per, row, lane);
-          }
+          const int nh = min(8, p.G - qc * 8);
+          merge_pieces<D>(p, qbase_local, nh, c0, npieces, c0_slot1, (long long)s * p.n_q + hg * QH + qbase_local, lane);
         }
       }
     }
