@@ -30,6 +30,7 @@
 
 #include <algorithm>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "pkv_device.cuh"
@@ -397,66 +398,13 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     }
   };
 
-  int it = 0;
-  for (int i = a; i < b; ++i, ++it) {
-    if (i == a || j == 0) {
-      // ---- unit start: this warp's 8 query rows as MMA B fragments
-      s = u / p.HG;
-      hg = u - s * p.HG;
-      L = seq_len(p, s, false);
-      if constexpr (CACHE == TC_BF16) {
-        fetch_query(u);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qf[ks][0] = qraw[ks][0];
-          qf[ks][1] = qraw[ks][1];
-        }
-      } else {
-        if (p.act_bf16) {
-          fetch_query(u);
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            qf[ks][0] = pack_f16(__uint_as_float(qraw[ks][0] << 16), __uint_as_float(qraw[ks][0] & 0xFFFF0000u));
-            qf[ks][1] = pack_f16(__uint_as_float(qraw[ks][1] << 16), __uint_as_float(qraw[ks][1] & 0xFFFF0000u));
-          }
-        } else {
-          // float32 queries: loaded and rounded to f16 here (not prefetched)
-          const int kv = hg * p.HPC + head_local;
-          const bool q_ok = qc * 8 + g < p.G;
-          const size_t qoff = ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
-#pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
-            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (q_ok) w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
-            qf[ks][0] = pack_f16(w.x, w.y);
-            qf[ks][1] = pack_f16(w.z, w.w);
-          }
-          if constexpr (CACHE == TC_FP8) {
-            raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
-            raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
-          }
-        }
-      }
-      head_k_scale = raw_k_scale;
-      head_v_scale = raw_v_scale;
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      m0 = m1 = -INFINITY;
-      l0 = l1 = 0.f;
-    }
-
-    const int stage = it % p.stages;
-    if (!mbar_wait(&full[stage], (it / p.stages) & 1)) {
-      flag_error(p.err, DEVERR_TIMEOUT);
-      break;
-    }
-    const uint8_t* st = smem + (size_t)stage * p.stage_bytes;
+  // Scores of one 16-token block held in stage memory st: S^T = K Q^T
+  // [16 tokens x 8 heads] in log2 units, -inf past the sequence end.
+  // sv = (token g, head 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); vsc = int8 V
+  // scales of tokens g and g+8 (1 otherwise).
+  auto block_scores = [&](const uint8_t* st, int valid, float (&sv)[4], float (&vsc)[2]) {
     const uint32_t kt = smem_addr(st + head_local * Tr::kTile);
-    const uint32_t vt = smem_addr(st + (p.HPC + head_local) * Tr::kTile);
-    const int valid = min(kBlockSize, L - j * kBlockSize);
     const int t0 = g, t1 = g + 8;
-
     // ---- S^T = K Q^T : [16 tokens x 8 heads]
     float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
     if constexpr (CACHE == TC_BF16) {
@@ -498,67 +446,41 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       }
     }
 
-    // ---- scale, mask, online softmax (base 2)
     float sc0 = p.scale_log2, sc1 = p.scale_log2;
-    float vs0 = 1.f, vs1 = 1.f;
+    vsc[0] = vsc[1] = 1.f;
     const int kvh = hg * p.HPC + head_local;
     if constexpr (CACHE == TC_INT8) {
       const float* ksm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile);
       const float* vsm = ksm + kBlockSize * p.n_kv;
       sc0 *= ksm[t0 * p.n_kv + kvh];
       sc1 *= ksm[t1 * p.n_kv + kvh];
-      vs0 = vsm[t0 * p.n_kv + kvh];
-      vs1 = vsm[t1 * p.n_kv + kvh];
+      vsc[0] = vsm[t0 * p.n_kv + kvh];
+      vsc[1] = vsm[t1 * p.n_kv + kvh];
     } else if constexpr (CACHE == TC_FP8) {
       sc0 *= head_k_scale;
       sc1 *= head_k_scale;
     }
     const bool ok0 = t0 < valid, ok1 = t1 < valid;
-    const float s00 = ok0 ? (sa[0] + sb[0]) * sc0 : -INFINITY;  // token g,   head 2c
-    const float s01 = ok0 ? (sa[1] + sb[1]) * sc0 : -INFINITY;  // token g,   head 2c+1
-    const float s10 = ok1 ? (sa[2] + sb[2]) * sc1 : -INFINITY;  // token g+8, head 2c
-    const float s11 = ok1 ? (sa[3] + sb[3]) * sc1 : -INFINITY;  // token g+8, head 2c+1
-    // The reference max m of each head moves only when some score exceeds it by
-    // more than kLazyLog2, so probabilities stay <= 2^kLazyLog2 and most blocks
-    // skip the cross-lane max and the rescale of the accumulators; the final
-    // o / l and lse = m + log2(l) do not depend on which m was used.
-    float mx0 = fmaxf(s00, s10), mx1 = fmaxf(s01, s11);
-    if (__any_sync(0xffffffffu, mx0 > m0 + kLazyLog2 || mx1 > m1 + kLazyLog2)) {
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-      }
-      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      l0 *= al0;
-      l1 *= al1;
-#pragma unroll
-      for (int mt = 0; mt < KS; ++mt) {
-        acc[mt][0] *= al0;
-        acc[mt][1] *= al1;
-        acc[mt][2] *= al0;
-        acc[mt][3] *= al1;
-      }
-    }
-    const float p00 = ex2(s00 - m0), p01 = ex2(s01 - m1);
-    const float p10 = ex2(s10 - m0), p11 = ex2(s11 - m1);
-    l0 += p00 + p10;
-    l1 += p01 + p11;
+    sv[0] = ok0 ? (sa[0] + sb[0]) * sc0 : -INFINITY;
+    sv[1] = ok0 ? (sa[1] + sb[1]) * sc0 : -INFINITY;
+    sv[2] = ok1 ? (sa[2] + sb[2]) * sc1 : -INFINITY;
+    sv[3] = ok1 ? (sa[3] + sb[3]) * sc1 : -INFINITY;
+  };
 
-    // ---- O^T += V^T P^T
+  // O^T += V^T P^T for one block with probabilities pr (layout of the scores).
+  auto block_pv = [&](const uint8_t* st, int valid, const float (&pr)[4], const float (&vsc)[2]) {
+    const uint32_t vt = smem_addr(st + (p.HPC + head_local) * Tr::kTile);
+    const bool ok0 = g < valid, ok1 = g + 8 < valid;
     uint32_t pb0, pb1;
     if constexpr (CACHE == TC_BF16) {
-      pb0 = movmatrix_trans(pack_bf16(p00, p01));
-      pb1 = movmatrix_trans(pack_bf16(p10, p11));
+      pb0 = movmatrix_trans(pack_bf16(pr[0], pr[1]));
+      pb1 = movmatrix_trans(pack_bf16(pr[2], pr[3]));
     } else if constexpr (CACHE == TC_INT8) {
-      pb0 = movmatrix_trans(pack_f16(ok0 ? p00 * vs0 : 0.f, ok0 ? p01 * vs0 : 0.f));
-      pb1 = movmatrix_trans(pack_f16(ok1 ? p10 * vs1 : 0.f, ok1 ? p11 * vs1 : 0.f));
+      pb0 = movmatrix_trans(pack_f16(ok0 ? pr[0] * vsc[0] : 0.f, ok0 ? pr[1] * vsc[0] : 0.f));
+      pb1 = movmatrix_trans(pack_f16(ok1 ? pr[2] * vsc[1] : 0.f, ok1 ? pr[3] * vsc[1] : 0.f));
     } else {
-      pb0 = movmatrix_trans(pack_f16(p00, p01));
-      pb1 = movmatrix_trans(pack_f16(p10, p11));
+      pb0 = movmatrix_trans(pack_f16(pr[0], pr[1]));
+      pb1 = movmatrix_trans(pack_f16(pr[2], pr[3]));
     }
     // token pairs of the A fragments: (2c, 2c+1) and (2c+8, 2c+9)
     uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
@@ -613,12 +535,139 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         mma_f16(acc[mt], af, pb0, pb1);
       }
     }
+  };
+
+  // One step over NB (1 or 2) consecutive blocks of the current unit: their
+  // scores, one online-softmax update, then their P.V.  Two blocks give each
+  // warp two independent MMA chains.  Returns false if a wait timed out.
+  int it = 0;
+  auto step = [&](auto nb_const) -> bool {
+    constexpr int NB = decltype(nb_const)::value;
+    const uint8_t* st[NB];
+    int stage[NB], valid[NB];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      stage[k] = (it + k) % p.stages;
+      if (!mbar_wait(&full[stage[k]], ((it + k) / p.stages) & 1)) return false;
+      st[k] = smem + (size_t)stage[k] * p.stage_bytes;
+      valid[k] = min(kBlockSize, L - (j + k) * kBlockSize);
+    }
+    float sv[NB][4], vsc[NB][2];
+#pragma unroll
+    for (int k = 0; k < NB; ++k) block_scores(st[k], valid[k], sv[k], vsc[k]);
+
+    // The reference max m of each head moves only when some score exceeds it by
+    // more than kLazyLog2, so probabilities stay <= 2^kLazyLog2 and most steps
+    // skip the cross-lane max and the rescale of the accumulators; the final
+    // o / l and lse = m + log2(l) do not depend on which m was used.
+    float mx0 = fmaxf(sv[0][0], sv[0][2]), mx1 = fmaxf(sv[0][1], sv[0][3]);
+#pragma unroll
+    for (int k = 1; k < NB; ++k) {
+      mx0 = fmaxf(mx0, fmaxf(sv[k][0], sv[k][2]));
+      mx1 = fmaxf(mx1, fmaxf(sv[k][1], sv[k][3]));
+    }
+    if (__any_sync(0xffffffffu, mx0 > m0 + kLazyLog2 || mx1 > m1 + kLazyLog2)) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= al0;
+      l1 *= al1;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        acc[mt][0] *= al0;
+        acc[mt][1] *= al1;
+        acc[mt][2] *= al0;
+        acc[mt][3] *= al1;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < NB; ++k) {
+      float pr[4];
+      pr[0] = ex2(sv[k][0] - m0);
+      pr[1] = ex2(sv[k][1] - m1);
+      pr[2] = ex2(sv[k][2] - m0);
+      pr[3] = ex2(sv[k][3] - m1);
+      l0 += pr[0] + pr[2];
+      l1 += pr[1] + pr[3];
+      block_pv(st[k], valid[k], pr, vsc[k]);
+    }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[stage]);
+    if (lane == 0) {
+#pragma unroll
+      for (int k = 0; k < NB; ++k) mbar_arrive(&empty[stage[k]]);
+    }
+    return true;
+  };
+
+  int i = a;
+  while (i < b) {
+    if (i == a || j == 0) {
+      // ---- unit start: this warp's 8 query rows as MMA B fragments
+      s = u / p.HG;
+      hg = u - s * p.HG;
+      L = seq_len(p, s, false);
+      if constexpr (CACHE == TC_BF16) {
+        fetch_query(u);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qf[ks][0] = qraw[ks][0];
+          qf[ks][1] = qraw[ks][1];
+        }
+      } else {
+        if (p.act_bf16) {
+          fetch_query(u);
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = pack_f16(__uint_as_float(qraw[ks][0] << 16), __uint_as_float(qraw[ks][0] & 0xFFFF0000u));
+            qf[ks][1] = pack_f16(__uint_as_float(qraw[ks][1] << 16), __uint_as_float(qraw[ks][1] & 0xFFFF0000u));
+          }
+        } else {
+          // float32 queries: loaded and rounded to f16 here (not prefetched)
+          const int kv = hg * p.HPC + head_local;
+          const bool q_ok = qc * 8 + g < p.G;
+          const size_t qoff = ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q_ok) w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
+            qf[ks][0] = pack_f16(w.x, w.y);
+            qf[ks][1] = pack_f16(w.z, w.w);
+          }
+          if constexpr (CACHE == TC_FP8) {
+            raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
+            raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
+          }
+        }
+      }
+      head_k_scale = raw_k_scale;
+      head_v_scale = raw_v_scale;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+
+    const int uend = P[u + 1];
+    const int nb = (i + 1 < b && i + 1 < uend) ? 2 : 1;
+    const bool ok = nb == 2 ? step(std::integral_constant<int, 2>{}) : step(std::integral_constant<int, 1>{});
+    if (!ok) {
+      flag_error(p.err, DEVERR_TIMEOUT);
+      break;
+    }
+    i += nb;
+    it += nb;
+    j += nb;
 
     // ---- unit end: finish here, or hand a piece to the merge
-    const bool unit_end = (i + 1 == P[u + 1]);
-    if (unit_end || i + 1 == b) {
+    const bool unit_end = (i == uend);
+    if (unit_end || i == b) {
       float lt0 = l0, lt1 = l1;
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) {
@@ -689,7 +738,6 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         }
       }
     }
-    ++j;
     if (unit_end) {
       ++u;
       while (u < units && P[u + 1] == P[u]) ++u;
@@ -842,13 +890,14 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   const int want_stages = tuning ? tuning->stages : 0;
   int stages = want_stages;
   if (stages <= 0) {
-    // Deepest ring (up to 4 stages) that still lets 4 CTAs share an SM; fewer
-    // CTAs per SM only when even 2 stages do not fit.
+    // Deepest ring that still lets 4 CTAs share an SM, so the SM keeps its
+    // whole shared memory (~190 KB) of K/V in flight; fewer CTAs per SM only
+    // when even 2 stages do not fit.
     stages = 2;
     for (int per = kTargetCtasPerSm; per >= 1; --per) {
       const size_t budget = (size_t)kSmemPerSm / per - 1024;
       if (budget < fixed) continue;
-      const int fit = (int)std::min<size_t>(4, (budget - fixed) / pl.stage_bytes);
+      const int fit = (int)std::min<size_t>(kMaxStages, (budget - fixed) / pl.stage_bytes);
       if (fit >= 2) {
         stages = fit;
         break;
