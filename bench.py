@@ -2,9 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference] [--config NAME]
 
-A step appends one token per sequence (pkv_kv_cache_write) and runs decode
-attention over every sequence's paged cache (pkv_paged_attention_decode), for
-one layer of the workload.  Default workload: the Llama-3-8B-shaped decode
+A step appends one token per sequence and runs decode attention over every
+sequence's paged cache, for one layer of the workload: one fused launch
+(pkv_paged_decode_step), or with --unfused the two calls pkv_kv_cache_write and
+pkv_paged_attention_decode.  Default workload: the Llama-3-8B-shaped decode
 step (batch 64, 32 query / 8 KV heads, head_dim 128, BF16 cache, block 16,
 context lengths uniform in [512, 4096], shuffled pool sized to fit exactly).
 
@@ -41,6 +42,7 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--config", default="llama3_8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--unfused", action="store_true", help="append and decode as two launches")
     return ap.parse_args()
 
 
@@ -333,10 +335,14 @@ def run_b200(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
 
-    def step():
-        ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
-        ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                   device_error=err)
+    def step(q=q, k_new=k_new, v_new=v_new, bt=bt, cl=cl, slots=slots):
+        if args.unfused:
+            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+            ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                       device_error=err)
+        else:
+            ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
+                                  workspace=ws, device_error=err)
 
     def barrier():
         if world > 1:
@@ -359,10 +365,15 @@ def run_b200(args, rank, world, local):
     att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     ev_start.record(stream)
     for k in range(args.steps):
-        ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
-        att[k][0].record(stream)
-        ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                   device_error=err)
+        if args.unfused:
+            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+            att[k][0].record(stream)
+            ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                       device_error=err)
+        else:
+            att[k][0].record(stream)
+            ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
+                                  workspace=ws, device_error=err)
         att[k][1].record(stream)
     ev_end.record(stream)
     torch.cuda.synchronize()
@@ -374,25 +385,30 @@ def run_b200(args, rank, world, local):
     assert int(err.item()) == 0, f"device error flag {int(err.item())}"
 
     # ---------------- end to end through the public API with host buffers
-    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-    h_q, h_k, h_v, h_slots, h_bt, h_cl = pin(q), pin(k_new), pin(v_new), pin(slots), pin(bt), pin(cl)
+    # The step's inputs (query, new K/V rows, block tables, lengths, slots) live
+    # in one pinned host buffer and cross to the device in one copy per step;
+    # the output comes back in one copy, and the host waits for it.
+    parts = [q, k_new, v_new, bt, cl, slots]
+    offs, total = [], 0
+    for t in parts:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
+    views = []
+    for t, o in zip(parts, offs):
+        nbytes = t.numel() * t.element_size()
+        h_in[o : o + nbytes].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
+        views.append(d_in[o : o + nbytes].view(t.dtype).view(t.shape))
+    d_q, d_k, d_v, d_bt, d_cl, d_slots = views
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
-    d_slots, d_bt, d_cl = torch.empty_like(slots), torch.empty_like(bt), torch.empty_like(cl)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_cl))
+    h2d = total
     d2h = h_out.numel() * h_out.element_size()
     e2e_steps = min(args.steps, 500)
 
     def e2e_step():
-        d_q.copy_(h_q, non_blocking=True)
-        d_k.copy_(h_k, non_blocking=True)
-        d_v.copy_(h_v, non_blocking=True)
-        d_slots.copy_(h_slots, non_blocking=True)
-        d_bt.copy_(h_bt, non_blocking=True)
-        d_cl.copy_(h_cl, non_blocking=True)
-        ops.kv_cache_write(d_k, d_v, kc, vc, d_slots, ks, vs, err)
-        ops.paged_attention_decode(out, d_q, kc, vc, d_bt, d_cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                   device_error=err)
+        d_in.copy_(h_in, non_blocking=True)
+        step(q=d_q, k_new=d_k, v_new=d_v, bt=d_bt, cl=d_cl, slots=d_slots)
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()  # the host reads the step's result
 
@@ -435,14 +451,16 @@ def run_b200(args, rank, world, local):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": traffic,
-                "kernel": "decode_tc_kernel (pkv_paged_attention_decode)",
+                "kernel": "decode_tc_kernel (pkv_paged_attention_decode)" if args.unfused
+                else "decode_tc_kernel with fused append (pkv_paged_decode_step)",
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "bytes_per_launch": kv_bytes,
                 "launch_ms": att_ms,
             },
             "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (2 if args.unfused else 1) * args.steps,
+            "step": "append + decode, two launches" if args.unfused else "append + decode fused in one launch",
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -137,6 +137,31 @@ pkv_status pkv_paged_attention_decode(void* out, const void* query, const void* 
                                       void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream);
 
 /*
+ * One decode step in one launch: append each sequence's new token, then attend.
+ *
+ * Same result as pkv_kv_cache_write(key, value, ...) with slot_mapping[s] =
+ * the slot of position context_lens[s] - 1 (block_tables[s][(L-1) / 16] * 16 +
+ * (L-1) % 16), followed by pkv_paged_attention_decode(...).  New tokens fill
+ * the current block ("Chapter 18 - KV-Cache Optimization Strategies", How
+ * PagedAttention Works), and the decode then reads them through the block
+ * table like every other row.
+ *
+ *   key, value   device, [num_seqs, n_kv, head_dim], act_dtype: the new
+ *                token's rows; sequences with context_lens[s] == 0 append nothing
+ *   key_cache, value_cache, k_scale, v_scale   as for pkv_kv_cache_write
+ *                (INT8 scales are written, FP8 per-head scales are read)
+ * Other arguments, shapes and errors as for pkv_paged_attention_decode.  In the
+ * tensor-core path the CTA that reads a sequence's last block writes its new
+ * rows first, so no second launch is needed.
+ */
+pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, const void* value, void* key_cache,
+                                 void* value_cache, float* k_scale, float* v_scale, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                 int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                 float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                 void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream);
+
+/*
  * Launch shape overrides for pkv_paged_attention_decode_ex (0 = automatic).
  * num_ctas: persistent CTAs sharing the blocks of all (sequence, KV-head group)
  * pairs; stages: depth of the shared-memory ring of K/V blocks; heads_per_cta:

@@ -84,7 +84,7 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
                               int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks, float sm_scale,
                               pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out, void* workspace,
                               size_t workspace_bytes, int32_t* device_error, const pkv_decode_tuning* tuning,
-                              void* stream) {
+                              void* stream, const void* new_key = nullptr, const void* new_value = nullptr) {
   const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, act_dtype, cache_dtype};
   pkv_status st = check_decode_shape(s);
   if (st != PKV_OK) return st;
@@ -99,7 +99,7 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
 
   TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
-           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error};
+           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error, new_key, new_value};
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (cache_dtype == PKV_F32) return launch_decode_f32(s, a, strm);
   TcPlan plan;
@@ -170,6 +170,20 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
   return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
                      context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream);
+}
+
+pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, const void* value, void* key_cache,
+                                 void* value_cache, float* k_scale, float* v_scale, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                 int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                 float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                 void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream) {
+  if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
+  if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream, key,
+                     value);
 }
 
 const char* pkv_status_string(pkv_status status) {

@@ -19,6 +19,9 @@ struct F32Params {
   const int32_t* context_lens;
   float* lse_out;
   int* err;
+  // fused decode step: token L-1 comes from these rows and is stored to the cache
+  const float* new_key;
+  const float* new_value;
   long long num_blocks;
   int max_blocks_per_seq, cap_len, num_seqs, n_q, n_kv, G;
   float sm_scale;
@@ -53,16 +56,34 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const F32Params p) {
       continue;
     }
     const size_t row = (((size_t)blk * kBlockSize + pos % kBlockSize) * p.n_kv + kv) * D + lane * EPL;
+    const float* krow = p.key_cache + row;
+    const float* vrow = p.value_cache + row;
+    if (p.new_key && pos == L - 1) {
+      // the appended token: read from the new rows; the group's first query
+      // head's warp stores them into the cache (no warp reads them back there)
+      const size_t nrow = ((size_t)s * p.n_kv + kv) * D + lane * EPL;
+      krow = p.new_key + nrow;
+      vrow = p.new_value + nrow;
+      if (h % p.G == 0) {
+        float* kc = const_cast<float*>(p.key_cache) + row;
+        float* vc = const_cast<float*>(p.value_cache) + row;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) {
+          kc[e] = __ldg(krow + e);
+          vc[e] = __ldg(vrow + e);
+        }
+      }
+    }
     float dot = 0.f;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) dot = fmaf(q[e], __ldg(p.key_cache + row + e), dot);
+    for (int e = 0; e < EPL; ++e) dot = fmaf(q[e], __ldg(krow + e), dot);
     dot = warp_sum(dot) * p.sm_scale;
     const float mn = fmaxf(m, dot);
     const float alpha = expf(m - mn);
     const float w = expf(dot - mn);
     l = l * alpha + w;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, __ldg(p.value_cache + row + e), acc[e] * alpha);
+    for (int e = 0; e < EPL; ++e) acc[e] = fmaf(w, __ldg(vrow + e), acc[e] * alpha);
     m = mn;
   }
   float* orow = p.out + ((size_t)s * p.n_q + h) * D + lane * EPL;
@@ -82,6 +103,8 @@ pkv_status launch_decode_f32(const DecodeShape& sh, const TcArgs& a, cudaStream_
   p.context_lens = a.context_lens;
   p.lse_out = a.lse_out;
   p.err = a.device_error;
+  p.new_key = static_cast<const float*>(a.new_key);
+  p.new_value = static_cast<const float*>(a.new_value);
   p.num_blocks = a.num_blocks;
   p.max_blocks_per_seq = a.max_blocks_per_seq;
   const int64_t cap = (int64_t)a.max_blocks_per_seq * kBlockSize;

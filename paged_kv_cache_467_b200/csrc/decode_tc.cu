@@ -32,6 +32,7 @@
 #include <mutex>
 #include <type_traits>
 
+#include "cache_row.cuh"
 #include "internal.h"
 #include "pkv_device.cuh"
 
@@ -40,8 +41,14 @@ namespace pkv {
 struct TcParams {
   void* out;
   const void* query;
-  const float* k_scale;
-  const float* v_scale;
+  float* k_scale;  // written by the fused step's int8 append, read otherwise
+  float* v_scale;
+  // fused decode step: the new token's rows [num_seqs, n_kv, D] (act dtype),
+  // appended as token L-1 of each sequence before it is attended; null = none
+  const void* new_key;
+  const void* new_value;
+  void* key_cache;
+  void* value_cache;
   const int32_t* block_tables;
   const int32_t* context_lens;
   float* lse_out;
@@ -225,7 +232,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)p.stages * p.stage_bytes);
   uint64_t* empty = full + p.stages;
-  int* wsum = reinterpret_cast<int*>(empty + p.stages);
+  uint64_t* append_done = empty + p.stages;  // fused step: the new rows are in the cache
+  int* wsum = reinterpret_cast<int*>(append_done + 1);
   int* P = wsum + 32;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -236,6 +244,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       mbar_init(&full[k], 1);
       mbar_init(&empty[k], p.NCW);
     }
+    mbar_init(append_done, p.HPC);  // one arrival per KV head of the CTA
     fence_barrier_init();
   }
   if (warp == p.NCW && lane == 0) {
@@ -253,14 +262,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   if (warp == p.NCW) {
     if (a >= b) return;
     int it = 0;
-    bool abort = false;
+    bool abort = false, appended = false;
     for (int base = a; base < b && !abort; base += 32) {
       const int i = base + lane;
-      int phys = -1, hg = 0;
+      int phys = -1, hg = 0, unit_last = 0;
       if (i < b) {
         const int u = upper_bound_smem(P, units + 1, i) - 1;
         const int s = u / p.HG;
         hg = u - s * p.HG;
+        unit_last = (i + 1 == P[u + 1]);
         phys = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + (i - P[u]));
         if (phys < 0 || (long long)phys >= p.num_blocks) {
           flag_error(p.err, DEVERR_BLOCK_RANGE);
@@ -271,10 +281,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       for (int k = 0; k < n; ++k) {
         const int ph = __shfl_sync(0xffffffffu, phys, k);
         const int hgk = __shfl_sync(0xffffffffu, hg, k);
+        const int lastk = __shfl_sync(0xffffffffu, unit_last, k);
         int ok = 1;
         if (lane == 0) {
           const int stage = it % p.stages;
           if (it >= p.stages && !mbar_wait(&empty[stage], ((it / p.stages) & 1) ^ 1)) {
+            flag_error(p.err, DEVERR_TIMEOUT);
+            ok = 0;
+          } else if (p.new_key && lastk && !appended && !(appended = mbar_wait(append_done, 0))) {
+            // the block holding a new token is read only after the consumers wrote it
             flag_error(p.err, DEVERR_TIMEOUT);
             ok = 0;
           } else {
@@ -336,6 +351,41 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     }
   }
   if (a >= b) return;
+
+  // Fused step: this CTA reads the last block of every unit that ends inside
+  // its range, so it writes those units' new rows (token L-1) into the cache
+  // first, one warp per KV head, while the producer starts the ring.  The
+  // proxy fence orders these generic stores before the TMA reads of the block.
+  if (p.new_key && qc == 0) {
+    for (int uu = upper_bound_smem(P, units + 1, a) - 1; uu < units && P[uu] < b; ++uu) {
+      if (P[uu + 1] > b) break;  // ends past this range: another CTA appends it
+      if (P[uu] == P[uu + 1]) continue;
+      const int ss = uu / p.HG, kv = (uu - ss * p.HG) * p.HPC + head_local;
+      const int pos = seq_len(p, ss, false) - 1;
+      const int phys = __ldg(p.block_tables + (size_t)ss * p.max_blocks_per_seq + pos / kBlockSize);
+      if (phys < 0 || (long long)phys >= p.num_blocks) {
+        if (lane == 0) flag_error(p.err, DEVERR_BLOCK_RANGE);
+        continue;
+      }
+      const size_t dst_row = ((size_t)phys * kBlockSize + pos % kBlockSize) * p.n_kv + kv;
+      const size_t src_row = (size_t)ss * p.n_kv + kv;
+      constexpr int kind = CACHE == TC_BF16 ? WK_COPY : (CACHE == TC_INT8 ? WK_INT8 : WK_FP8);
+      if (p.act_bf16) {
+        write_row<true, kind, D / 32>(static_cast<const uint8_t*>(p.new_key) + src_row * D * 2, p.key_cache, p.k_scale,
+                                      dst_row, kv, p.n_kv, lane);
+        write_row<true, kind, D / 32>(static_cast<const uint8_t*>(p.new_value) + src_row * D * 2, p.value_cache,
+                                      p.v_scale, dst_row, kv, p.n_kv, lane);
+      } else if constexpr (CACHE != TC_BF16) {
+        write_row<false, kind, D / 32>(static_cast<const uint8_t*>(p.new_key) + src_row * D * 4, p.key_cache, p.k_scale,
+                                       dst_row, kv, p.n_kv, lane);
+        write_row<false, kind, D / 32>(static_cast<const uint8_t*>(p.new_value) + src_row * D * 4, p.value_cache,
+                                       p.v_scale, dst_row, kv, p.n_kv, lane);
+      }
+    }
+    fence_proxy_async_global();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(append_done);
+  }
 
   // Per-lane ldmatrix offsets inside a head tile (128-byte swizzle: the 16-byte
   // chunk j of row r lives at chunk j ^ (r & 7)).
@@ -814,8 +864,12 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   TcParams prm;
   prm.out = a.out;
   prm.query = a.query;
-  prm.k_scale = a.k_scale;
-  prm.v_scale = a.v_scale;
+  prm.k_scale = const_cast<float*>(a.k_scale);
+  prm.v_scale = const_cast<float*>(a.v_scale);
+  prm.new_key = a.new_key;
+  prm.new_value = a.new_value;
+  prm.key_cache = const_cast<void*>(a.key_cache);
+  prm.value_cache = const_cast<void*>(a.value_cache);
   prm.block_tables = a.block_tables;
   prm.context_lens = a.context_lens;
   prm.lse_out = a.lse_out;
@@ -886,7 +940,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   const int sms = device_sm_count();
   const int optin = device_smem_optin();
   if (sms <= 0 || optin <= 0) return PKV_ERR_CUDA;
-  const size_t fixed = align_up(2 * 8 * kMaxStages + 32 * 4 + ((size_t)pl.units + 1) * 4, 16) + 1024;
+  const size_t fixed = align_up(2 * 8 * kMaxStages + 16 + 32 * 4 + ((size_t)pl.units + 1) * 4, 16) + 1024;
   const int want_stages = tuning ? tuning->stages : 0;
   int stages = want_stages;
   if (stages <= 0) {

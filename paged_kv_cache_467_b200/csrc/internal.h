@@ -56,6 +56,10 @@ struct TcArgs {
   float* lse_out;
   void* workspace;
   int32_t* device_error;
+  // fused decode step only: new rows [num_seqs, n_kv, head_dim] appended as token
+  // L-1 of each sequence before the attention (the caches are then written)
+  const void* new_key = nullptr;
+  const void* new_value = nullptr;
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);

@@ -59,8 +59,13 @@ def _rows(x, w, device):
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(device=device, dtype=_TORCH_ACT[w.act_dtype])
 
 
-def fill_gpu(w: workloads.DecodeWorkload, device="cuda", fp8_scales=None, chunk_tokens=1 << 20) -> GpuState:
-    """Allocate a poisoned pool and append every row through pkv_kv_cache_write."""
+def fill_gpu(w: workloads.DecodeWorkload, device="cuda", fp8_scales=None, chunk_tokens=1 << 20,
+             append_new: bool = True) -> GpuState:
+    """Allocate a poisoned pool and append rows through pkv_kv_cache_write.
+
+    With ``append_new=False`` the new token (position L-1) is left out, for
+    the fused decode step to append.
+    """
     from paged_kv_cache_467_b200 import ops
 
     kc, vc = _poisoned_cache(w, device)
@@ -92,8 +97,9 @@ def fill_gpu(w: workloads.DecodeWorkload, device="cuda", fp8_scales=None, chunk_
         if n >= chunk_tokens or s == w.num_seqs - 1:
             write(np.concatenate(bk), np.concatenate(bv), np.concatenate(bslots))
             bk, bv, bslots, n = [], [], [], 0
-    nk, nv = w.new_kv()
-    write(nk, nv, w.new_token_slots())
+    if append_new:
+        nk, nv = w.new_kv()
+        write(nk, nv, w.new_token_slots())
     torch.cuda.synchronize()
     return GpuState(
         key_cache=kc,
@@ -198,3 +204,21 @@ def assert_close(got, want, cache_dtype, what=""):
     mx, mean = errors(got, want)
     assert mx <= mx_tol and mean <= mean_tol, f"{what}: max abs {mx:.3e} (tol {mx_tol}), mean abs {mean:.3e} (tol {mean_tol})"
     return mx, mean
+
+
+def new_rows(w, device="cuda"):
+    nk, nv = w.new_kv()
+    return _rows(nk, w, device), _rows(nv, w, device)
+
+
+def run_decode_step(w, st: GpuState, workspace=None):
+    """The fused step (append token L-1, then attend) through pkv_paged_decode_step."""
+    from paged_kv_cache_467_b200 import ops
+
+    k, v = new_rows(w, st.query.device)
+    out = torch.full((w.num_seqs, w.n_q, w.head_dim), float("nan"), dtype=_TORCH_ACT[w.act_dtype], device=st.query.device)
+    lse = torch.full((w.num_seqs, w.n_q), float("nan"), dtype=torch.float32, device=st.query.device)
+    ops.paged_decode_step(out, st.query, k, v, st.key_cache, st.value_cache, st.block_tables, st.context_lens,
+                          w.max_context_len, w.sm_scale, st.k_scale, st.v_scale, lse, workspace, st.device_error)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
