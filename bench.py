@@ -43,6 +43,7 @@ def parse_args():
     ap.add_argument("--config", default="llama3_8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true", help="append and decode as two launches")
+    ap.add_argument("--no-overlap", action="store_true", help="launch each step without overlapping its prologue")
     return ap.parse_args()
 
 
@@ -330,19 +331,23 @@ def run_b200(args, rank, world, local):
     cl = torch.from_numpy(w.context_lens).to(dev)
     out = torch.empty_like(q)
     err = torch.zeros(1, dtype=torch.int32, device=dev)
+    # Block tables and lengths are set up before the loop and never written by
+    # the kernel launched right before a step, so each step may overlap its
+    # prologue with the previous step's tail (programmatic dependent launch).
+    tuning = None if args.no_overlap else ops.DecodeTuning(0, 0, 0, ops.TUNE_OVERLAP_PROLOGUE)
     nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc))
     ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
 
-    def step(q=q, k_new=k_new, v_new=v_new, bt=bt, cl=cl, slots=slots):
+    def step(q=q, k_new=k_new, v_new=v_new, bt=bt, cl=cl, slots=slots, overlap=True):
         if args.unfused:
             ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
             ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
                                        device_error=err)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err)
+                                  workspace=ws, device_error=err, tuning=tuning if overlap else None)
 
     def barrier():
         if world > 1:
@@ -362,7 +367,13 @@ def run_b200(args, rank, world, local):
     barrier()
     torch.cuda.synchronize()
     ev_start, ev_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # Two-launch step: events around each decode launch give the decode
+    # kernel's own time.  One-launch step: the kernel is the whole step, and
+    # nothing is recorded between launches (an event between two kernels would
+    # keep a step's prologue from overlapping the previous step), so its
+    # per-launch time is the timed region / K, gaps included.
+    att = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps if args.unfused else 0)]
     ev_start.record(stream)
     for k in range(args.steps):
         if args.unfused:
@@ -370,17 +381,16 @@ def run_b200(args, rank, world, local):
             att[k][0].record(stream)
             ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
                                        device_error=err)
+            att[k][1].record(stream)
         else:
-            att[k][0].record(stream)
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err)
-        att[k][1].record(stream)
+                                  workspace=ws, device_error=err, tuning=tuning)
     ev_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     ms = ev_start.elapsed_time(ev_end) / args.steps
-    att_ms = sum(a.elapsed_time(b) for a, b in att) / args.steps
+    att_ms = sum(a.elapsed_time(b) for a, b in att) / args.steps if args.unfused else ms
     ms, att_ms = max_over_ranks([ms, att_ms], world, dev)
     assert int(err.item()) == 0, f"device error flag {int(err.item())}"
 
@@ -408,7 +418,8 @@ def run_b200(args, rank, world, local):
 
     def e2e_step():
         d_in.copy_(h_in, non_blocking=True)
-        step(q=d_q, k_new=d_k, v_new=d_v, bt=d_bt, cl=d_cl, slots=d_slots)
+        # lengths and tables arrive with this copy, so no prologue overlap here
+        step(q=d_q, k_new=d_k, v_new=d_v, bt=d_bt, cl=d_cl, slots=d_slots, overlap=False)
         h_out.copy_(out, non_blocking=True)
         stream.synchronize()  # the host reads the step's result
 
@@ -460,7 +471,8 @@ def run_b200(args, rank, world, local):
             "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
             "gpu_launches": (2 if args.unfused else 1) * args.steps,
-            "step": "append + decode, two launches" if args.unfused else "append + decode fused in one launch",
+            "step": ("append + decode, two launches" if args.unfused else "append + decode fused in one launch")
+            + ("" if args.no_overlap or args.unfused else "; prologue overlaps the previous step (programmatic launch)"),
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

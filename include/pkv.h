@@ -171,11 +171,30 @@ typedef struct {
   int num_ctas;
   int stages;
   int heads_per_cta;
+  int flags; /* PKV_TUNE_* bits */
 } pkv_decode_tuning;
+
+/* Launch the decode kernel so that it may start while the kernel launched just
+ * before it on the same stream is still finishing (programmatic dependent
+ * launch).  Its CTAs then build their schedule from context_lens and
+ * block_tables and wait for the earlier kernel before reading anything else
+ * (queries, new rows, the cache, the workspace) or writing anything.  Only
+ * valid when context_lens and block_tables were not written by the kernel
+ * launched immediately before this call. */
+#define PKV_TUNE_OVERLAP_PROLOGUE 0x1
 
 /* Workspace bytes for pkv_paged_attention_decode_ex with the given tuning. */
 size_t pkv_paged_attention_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
                                              pkv_dtype cache_dtype, const pkv_decode_tuning* tuning);
+
+/* pkv_paged_decode_step with launch overrides (tuning may be NULL). */
+pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* key, const void* value, void* key_cache,
+                                    void* value_cache, float* k_scale, float* v_scale, const int32_t* block_tables,
+                                    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                    int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                    void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                    const pkv_decode_tuning* tuning, void* stream);
 
 /* pkv_paged_attention_decode with explicit launch shape (tuning may be NULL). */
 pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const void* key_cache, const void* value_cache,

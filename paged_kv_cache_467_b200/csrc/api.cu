@@ -172,18 +172,31 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream);
 }
 
+pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* key, const void* value, void* key_cache,
+                                    void* value_cache, float* k_scale, float* v_scale, const int32_t* block_tables,
+                                    int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
+                                    int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                    void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                    const pkv_decode_tuning* tuning, void* stream) {
+  if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
+  if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream, key,
+                     value);
+}
+
 pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, const void* value, void* key_cache,
                                  void* value_cache, float* k_scale, float* v_scale, const int32_t* block_tables,
                                  int max_blocks_per_seq, const int32_t* context_lens, int max_context_len,
                                  int num_seqs, int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
                                  float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
                                  void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream) {
-  if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
-  if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
-  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
-                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
-                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream, key,
-                     value);
+  return pkv_paged_decode_step_ex(out, query, key, value, key_cache, value_cache, k_scale, v_scale, block_tables,
+                                  max_blocks_per_seq, context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim,
+                                  block_size, num_blocks, sm_scale, act_dtype, cache_dtype, lse_out, workspace,
+                                  workspace_bytes, device_error, nullptr, stream);
 }
 
 const char* pkv_status_string(pkv_status status) {

@@ -239,6 +239,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int units = p.units;
 
+  grid_launch_dependents();
   if (threadIdx.x == 0) {
     for (int k = 0; k < p.stages; ++k) {
       mbar_init(&full[k], 1);
@@ -257,6 +258,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const int per = max(1, (total + (int)gridDim.x - 1) / (int)gridDim.x);
   const int a = min((int)blockIdx.x * per, total);
   const int b = min(a + per, total);
+  // Everything above read only context_lens and block_tables.  Under a
+  // programmatic launch the previous kernel may still be running: wait for it
+  // before touching queries, new rows, the cache, the workspace or outputs.
+  grid_wait_prerequisites();
 
   // ------------------------------------------------------------ producer
   if (warp == p.NCW) {
@@ -837,8 +842,18 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
     configured_bytes = (int)plan.smem_bytes;
   }
-  kern<<<plan.num_ctas, (plan.NCW + 1) * 32, plan.smem_bytes, stream>>>(km, vm, prm);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(plan.num_ctas);
+  cfg.blockDim = dim3((plan.NCW + 1) * 32);
+  cfg.dynamicSmemBytes = plan.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = plan.overlap_prologue ? 1 : 0;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, prm);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_tc_kernel launch");
   return PKV_OK;
 }
@@ -965,6 +980,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   // CTAs resident per SM from shared memory alone (1 KB reserved per CTA).
   const int per_sm = std::max(1, std::min(kTargetCtasPerSm, (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
   const int want_ctas = tuning ? tuning->num_ctas : 0;
+  pl.overlap_prologue = tuning && (tuning->flags & PKV_TUNE_OVERLAP_PROLOGUE);
   pl.num_ctas = want_ctas > 0 ? want_ctas : sms * per_sm;
   if (pl.num_ctas > kMaxCtas) return want_ctas > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   const size_t QH = (size_t)pl.HPC * pl.G;

@@ -32,6 +32,7 @@ struct TcPlan {
   int chunks;       // 128-byte row chunks per KV head row (head_dim * elem / 128)
   int stages;
   int num_ctas;
+  bool overlap_prologue;  // programmatic dependent launch (PKV_TUNE_OVERLAP_PROLOGUE)
   int units;        // num_seqs * HG
   uint32_t stage_bytes, tx_bytes;
   size_t smem_bytes;

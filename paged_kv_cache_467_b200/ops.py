@@ -39,7 +39,11 @@ class PkvError(RuntimeError):
 
 
 class DecodeTuning(ctypes.Structure):
-    _fields_ = [("num_ctas", ctypes.c_int), ("stages", ctypes.c_int), ("heads_per_cta", ctypes.c_int)]
+    _fields_ = [("num_ctas", ctypes.c_int), ("stages", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
+                ("flags", ctypes.c_int)]
+
+
+TUNE_OVERLAP_PROLOGUE = 0x1
 
 
 def _load() -> ctypes.CDLL:
@@ -61,6 +65,8 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i64,
                                           f32, i32, i32, vp, vp, sz, vp, vp]
     lib.pkv_paged_decode_step.restype = i32
+    lib.pkv_paged_decode_step_ex.argtypes = lib.pkv_paged_decode_step.argtypes[:-1] + [ctypes.POINTER(DecodeTuning), vp]
+    lib.pkv_paged_decode_step_ex.restype = i32
     lib.pkv_paged_attention_decode_static.argtypes = decode_args[:20] + [vp, vp]
     lib.pkv_paged_attention_decode_static.restype = i32
     lib.pkv_status_string.argtypes = [i32]
@@ -192,7 +198,7 @@ def paged_attention_decode(
 
 def paged_decode_step(out, query, key, value, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
                       sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None, workspace=None,
-                      device_error=None):
+                      device_error=None, tuning: DecodeTuning | None = None):
     """One fused decode step: append ``key``/``value`` [S, n_kv, d] as token L-1 of each sequence, then attend."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
@@ -200,15 +206,19 @@ def paged_decode_step(out, query, key, value, key_cache, value_cache, block_tabl
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:
-        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode)
+        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, tuning)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib.pkv_paged_decode_step(
+    args = [
         _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
         _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q,
         n_kv, d, block_size, num_blocks, float(sm_scale), act_code(query), ccode, _ptr(lse_out), _ptr(workspace),
-        ws_bytes, _ptr(device_error), _stream(query.device),
-    )
+        ws_bytes, _ptr(device_error),
+    ]
+    if tuning is None:
+        st = lib.pkv_paged_decode_step(*args, _stream(query.device))
+    else:
+        st = lib.pkv_paged_decode_step_ex(*args, ctypes.byref(tuning), _stream(query.device))
     _check(st, "pkv_paged_decode_step")
     return out
 

@@ -54,3 +54,34 @@ def test_decode_step_full_llama_config():
     out, lse = run_decode_step(w, st)
     assert int(st.device_error.item()) == 0
     check_all(w, st, out, lse, seqs=range(0, 64, 7))
+
+
+def test_overlapped_prologue_in_a_step_loop():
+    """PKV_TUNE_OVERLAP_PROLOGUE: each step's query and new rows come from a
+    torch kernel launched just before the decode, so a decode that read them
+    before its wait would see the previous step's values."""
+    from paged_kv_cache_467_b200 import ops
+
+    w = workloads.make_workload("o", seed=43, context_lens=[900 + 61 * i for i in range(24)], n_q=32, n_kv=8,
+                                head_dim=128)
+    a = fill_gpu(w, append_new=False)
+    b = fill_gpu(w, append_new=False)
+    over = ops.DecodeTuning(0, 0, 0, ops.TUNE_OVERLAP_PROLOGUE)
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    S, nq, nkv, d = w.num_seqs, w.n_q, w.n_kv, w.head_dim
+    q = torch.empty((S, nq, d), dtype=torch.bfloat16, device="cuda")
+    k = torch.empty((S, nkv, d), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    out_a, out_b = torch.empty_like(q), torch.empty_like(q)
+    for step in range(6):
+        k.copy_(torch.randn((S, nkv, d), device="cuda", generator=gen))
+        v.copy_(torch.randn((S, nkv, d), device="cuda", generator=gen))
+        q.copy_(torch.randn((S, nq, d), device="cuda", generator=gen))  # the kernel right before the decode
+        ops.paged_decode_step(out_a, q, k, v, a.key_cache, a.value_cache, a.block_tables, a.context_lens,
+                              w.max_context_len, w.sm_scale, tuning=over, device_error=a.device_error)
+        ops.paged_decode_step(out_b, q, k, v, b.key_cache, b.value_cache, b.block_tables, b.context_lens,
+                              w.max_context_len, w.sm_scale, device_error=b.device_error)
+        torch.cuda.synchronize()
+        assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16)), f"step {step}"
+    assert torch.equal(a.key_cache.view(torch.int16), b.key_cache.view(torch.int16))
+    assert int(a.device_error.item()) == 0 and int(b.device_error.item()) == 0
