@@ -22,3 +22,4 @@ from .paged_attention import (  # noqa: F401
     kv_head_of,
     paged_attention_decode,
 )
+from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402

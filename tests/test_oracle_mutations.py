@@ -89,3 +89,26 @@ def test_int8_scale_of_wrong_head_is_caught(monkeypatch):
 
     monkeypatch.setattr(pa, "dequantize_rows", head0_scale)
     _fails(lambda: pins.test_quantized_decode_is_attention_over_dequantized_rows("int8"))
+
+
+def test_copy_direction_swapped_is_caught(monkeypatch):
+    import numpy as np
+
+    import oracle.block_ops as bo
+    import test_oracle_block_ops as bpins
+
+    real = bo.copy_blocks
+    monkeypatch.setattr(bpins, "copy_blocks", lambda pools, pairs: real(pools, np.asarray(pairs)[:, ::-1]))
+    _fails(bpins.test_copy_on_write_divergence)
+
+
+def test_swap_ignoring_destination_slot_is_caught(monkeypatch):
+    import numpy as np
+
+    import oracle.block_ops as bo
+    import test_oracle_block_ops as bpins
+
+    real = bo.swap_blocks
+    monkeypatch.setattr(bpins, "swap_blocks",
+                        lambda s, d, pairs: real(s, d, np.stack([np.asarray(pairs)[:, 0]] * 2, axis=1)))
+    _fails(lambda: bpins.test_offload_example(read_golden))
