@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true", help="append and decode as two launches")
     ap.add_argument("--no-overlap", action="store_true", help="launch each step without overlapping its prologue")
+    ap.add_argument("--op", default="decode_step", choices=["decode_step", "copy_blocks", "swap_blocks"],
+                    help="what a step runs (the default is the decode step)")
     return ap.parse_args()
 
 
@@ -490,11 +492,74 @@ def run_b200(args, rank, world, local):
         dist.destroy_process_group()
 
 
+def run_block_ops(args):
+    """--op copy_blocks / swap_blocks: throughput of the block movers on the
+    default workload's pool (bf16, 8 KV heads, head_dim 128, 64 KiB of K+V per
+    block).  A step moves 1024 random blocks: inside the pool (copy-on-write
+    copies), or to page-locked host memory and back (offload, restore)."""
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_467_b200 import ops, workloads
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workloads.CONFIGS[args.config]()
+    shape = (w.num_blocks, w.block_size, w.n_kv, w.head_dim)
+    gen = torch.Generator(device=dev).manual_seed(7)
+    kc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+    vc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+    n = 1024
+    perm = np.random.default_rng(3).permutation(w.num_blocks)
+    block_bytes = 2 * kc[0].numel() * kc.element_size()
+    stream = torch.cuda.current_stream(dev)
+    if args.op == "copy_blocks":
+        pairs = torch.from_numpy(np.stack([perm[:n], perm[n : 2 * n]], 1).astype(np.int64)).to(dev)
+        steps = [lambda: ops.copy_blocks(kc, vc, pairs)]
+        moved = 2 * n * block_bytes  # read + write, like the copy peak
+        peak, peak_src, bound, what = measured_peaks()[0], "measured hbm_gbs (copy: read + write)", "hbm", "copy"
+    else:
+        hk = torch.empty((n,) + shape[1:], dtype=torch.bfloat16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        out_pairs = torch.from_numpy(np.stack([perm[:n], np.arange(n)], 1).astype(np.int64)).to(dev)
+        in_pairs = torch.from_numpy(np.stack([np.arange(n), perm[n : 2 * n]], 1).astype(np.int64)).to(dev)
+        steps = [lambda: ops.swap_blocks(kc, vc, hk, hv, out_pairs),
+                 lambda: ops.swap_blocks(hk, hv, kc, vc, in_pairs, device=dev)]
+        moved = 2 * n * block_bytes  # n blocks out + n blocks back in
+        peak, peak_src, bound, what = 64.0, "nominal PCIe Gen5 x16, per direction (no measured host-link peak)", \
+            "host link", "offload + restore"
+    for _ in range(max(args.warmup, 3)):
+        for f in steps:
+            f()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for f in steps:
+            f()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    gbs = moved / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "metric": f"paged block {what} GB/s", "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "blocks_per_step": n, "bytes_per_block_kv": block_bytes,
+                   "bytes_moved_per_step": moved},
+        "roofline": {"bound": bound, "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                     "traffic": None, "peak_source": peak_src},
+        "gpu_launches": len(steps) * args.steps,
+    }), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.op != "decode_step":
+        run_block_ops(args)
         return
     run_b200(args, rank, world, local)
 

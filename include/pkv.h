@@ -239,6 +239,46 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const
                                              float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype,
                                              float* lse_out, int32_t* device_error, void* stream);
 
+/*
+ * Copy whole physical blocks inside one pool: copy-on-write of shared blocks.
+ *
+ * Several block tables may point at one physical block; when a sequence
+ * diverges, only the affected block is duplicated ("Chapter 18 - KV-Cache
+ * Optimization Strategies", Prefix Caching; KV-cache overview page t13_4,
+ * copy-on-write paragraph).  For each pair p: block block_mapping[2p+1] of the
+ * K and V pools (and, for INT8, of k_scale / v_scale) <- block block_mapping[2p].
+ *
+ *   key_cache, value_cache  device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
+ *   k_scale, v_scale        INT8 only: device [num_blocks, block_size, n_kv]; NULL otherwise
+ *                           (FP8 per-head scales belong to no block)
+ *   block_mapping           device (or mapped host) int64 [num_pairs, 2] = (src, dst)
+ * Destinations must be distinct and no block may be both a source and a
+ * destination in one call (all pairs run in parallel).  Out-of-range block ids
+ * set PKV_DEVERR_BLOCK_RANGE and the pair is skipped.  n_kv * head_dim * bytes
+ * must be a multiple of 16.
+ */
+pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                           const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
+                           int64_t num_blocks, pkv_dtype cache_dtype, int32_t* device_error, void* stream);
+
+/*
+ * Move whole blocks between two pools: offload to host memory and restore.
+ *
+ * Blocks not needed now move to a larger, slower tier and come back when they
+ * are needed again ("KV Cache Engineering for LLM Serving", section 12, Cache
+ * Offloading from GPU).  For each pair p: block block_mapping[2p+1] of the dst
+ * pools <- block block_mapping[2p] of the src pools (K, V and INT8 scales).
+ * Either side may be page-locked host memory mapped into the device address
+ * space (cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped): the
+ * kernel reads or writes it directly over the host link.  Same layouts,
+ * dtype rules and error handling as pkv_copy_blocks; destinations distinct.
+ */
+pkv_status pkv_swap_blocks(const void* src_key, const void* src_value, const float* src_k_scale,
+                           const float* src_v_scale, int64_t src_num_blocks, void* dst_key, void* dst_value,
+                           float* dst_k_scale, float* dst_v_scale, int64_t dst_num_blocks,
+                           const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
+                           pkv_dtype cache_dtype, int32_t* device_error, void* stream);
+
 /* Static text for a status code. */
 const char* pkv_status_string(pkv_status status);
 

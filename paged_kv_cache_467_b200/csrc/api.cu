@@ -109,6 +109,84 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   return launch_tc(s, plan, a, strm);
 }
 
+// Address a kernel on the current device may use for p: device (or managed)
+// memory of this device as is, page-locked host memory through its mapped
+// device address.  Anything else (pageable host memory, another device's
+// memory) is rejected, so the kernel never dereferences an unmapped pointer.
+static pkv_status device_address(const void* p, const void** out) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of the query
+    return PKV_ERR_INVALID_ARG;
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PKV_ERR_CUDA;
+  switch (a.type) {
+    case cudaMemoryTypeDevice:
+      if (a.device != dev) return PKV_ERR_INVALID_ARG;
+      *out = p;
+      return PKV_OK;
+    case cudaMemoryTypeManaged:
+      *out = p;
+      return PKV_OK;
+    case cudaMemoryTypeHost:
+      if (!a.devicePointer) return PKV_ERR_INVALID_ARG;
+      *out = a.devicePointer;
+      return PKV_OK;
+    default:
+      return PKV_ERR_INVALID_ARG;
+  }
+}
+
+static pkv_status device_addresses(const void* src[4], void* dst[4], int npools, const int64_t** pairs) {
+  for (int i = 0; i < npools; ++i) {
+    const void* d = nullptr;
+    pkv_status st = device_address(src[i], &src[i]);
+    if (st != PKV_OK) return st;
+    st = device_address(dst[i], &d);
+    if (st != PKV_OK) return st;
+    dst[i] = const_cast<void*>(d);
+  }
+  const void* m = nullptr;
+  pkv_status st = device_address(*pairs, &m);
+  if (st != PKV_OK) return st;
+  *pairs = static_cast<const int64_t*>(m);
+  return PKV_OK;
+}
+
+// Shared checks of the block movers; fills the pool descriptors.
+static pkv_status move_plan(const void* src_k, const void* src_v, const float* src_ks, const float* src_vs,
+                            void* dst_k, void* dst_v, float* dst_ks, float* dst_vs, const int64_t* pairs,
+                            int64_t num_pairs, int n_kv, int head_dim, int block_size, pkv_dtype cache_dtype,
+                            const void* src[4], void* dst[4], size_t bpb[4], int* npools) {
+  if (num_pairs < 0 || n_kv <= 0 || head_dim <= 0 || block_size <= 0) return PKV_ERR_INVALID_ARG;
+  if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
+  if (num_pairs > 0 && (!pairs || !src_k || !src_v || !dst_k || !dst_v)) return PKV_ERR_INVALID_ARG;
+  const size_t elem = cache_dtype == PKV_F32 ? 4 : (cache_dtype == PKV_BF16 ? 2 : 1);
+  const size_t row = (size_t)n_kv * head_dim * elem;
+  if (row % 16 != 0) return PKV_ERR_UNSUPPORTED;
+  if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v)) return PKV_ERR_INVALID_ARG;
+  src[0] = src_k;
+  src[1] = src_v;
+  dst[0] = dst_k;
+  dst[1] = dst_v;
+  bpb[0] = bpb[1] = row * block_size;
+  *npools = 2;
+  const bool int8 = cache_dtype == PKV_INT8;
+  if (int8 != (src_ks && src_vs && dst_ks && dst_vs)) return PKV_ERR_INVALID_ARG;
+  if (int8) {
+    if (!aligned16(src_ks) || !aligned16(src_vs) || !aligned16(dst_ks) || !aligned16(dst_vs)) return PKV_ERR_INVALID_ARG;
+    if (((size_t)block_size * n_kv * 4) % 16 != 0) return PKV_ERR_UNSUPPORTED;
+    src[2] = src_ks;
+    src[3] = src_vs;
+    dst[2] = dst_ks;
+    dst[3] = dst_vs;
+    bpb[2] = bpb[3] = (size_t)block_size * n_kv * 4;
+    *npools = 4;
+  }
+  return PKV_OK;
+}
+
 }  // namespace pkv
 
 using namespace pkv;
@@ -197,6 +275,45 @@ pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, 
                                   max_blocks_per_seq, context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim,
                                   block_size, num_blocks, sm_scale, act_dtype, cache_dtype, lse_out, workspace,
                                   workspace_bytes, device_error, nullptr, stream);
+}
+
+pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                           const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
+                           int64_t num_blocks, pkv_dtype cache_dtype, int32_t* device_error, void* stream) {
+  const void* src[4];
+  void* dst[4];
+  size_t bpb[4];
+  int npools = 0;
+  pkv_status st = move_plan(key_cache, value_cache, k_scale, v_scale, key_cache, value_cache, k_scale, v_scale,
+                            block_mapping, num_pairs, n_kv, head_dim, block_size, cache_dtype, src, dst, bpb, &npools);
+  if (st != PKV_OK) return st;
+  if (num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PKV_OK;
+  st = device_addresses(src, dst, npools, &block_mapping);
+  if (st != PKV_OK) return st;
+  return launch_move_blocks(src, dst, bpb, npools, block_mapping, num_pairs, num_blocks, num_blocks, device_error,
+                            static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_swap_blocks(const void* src_key, const void* src_value, const float* src_k_scale,
+                           const float* src_v_scale, int64_t src_num_blocks, void* dst_key, void* dst_value,
+                           float* dst_k_scale, float* dst_v_scale, int64_t dst_num_blocks,
+                           const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
+                           pkv_dtype cache_dtype, int32_t* device_error, void* stream) {
+  const void* src[4];
+  void* dst[4];
+  size_t bpb[4];
+  int npools = 0;
+  pkv_status st = move_plan(src_key, src_value, src_k_scale, src_v_scale, dst_key, dst_value, dst_k_scale,
+                            dst_v_scale, block_mapping, num_pairs, n_kv, head_dim, block_size, cache_dtype, src, dst,
+                            bpb, &npools);
+  if (st != PKV_OK) return st;
+  if (src_num_blocks < 0 || dst_num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PKV_OK;
+  st = device_addresses(src, dst, npools, &block_mapping);
+  if (st != PKV_OK) return st;
+  return launch_move_blocks(src, dst, bpb, npools, block_mapping, num_pairs, src_num_blocks, dst_num_blocks,
+                            device_error, static_cast<cudaStream_t>(stream));
 }
 
 const char* pkv_status_string(pkv_status status) {

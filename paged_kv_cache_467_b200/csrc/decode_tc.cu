@@ -936,10 +936,12 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     pl.HPC = want_hpc;
   } else {
     // Two consumer warps per CTA (2 KV heads when the group fits one warp) and
-    // several CTAs per SM measured best: each SM then streams several units.
+    // four CTAs per SM measured best for bf16 and int8; FP8, whose dequant is
+    // heavier on the ALUs, does best with four warps per CTA and two CTAs.
+    const int warps = pl.cache_kind == TC_FP8 ? 4 : 2;
     pl.HPC = 1;
-    for (int h = std::min(s.n_kv, 2); h >= 1; --h) {
-      if (s.n_kv % h == 0 && h * pl.QC <= 2) {
+    for (int h = std::min(s.n_kv, warps); h >= 1; --h) {
+      if (s.n_kv % h == 0 && h * pl.QC <= warps) {
         pl.HPC = h;
         break;
       }
@@ -963,7 +965,8 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     // whole shared memory (~190 KB) of K/V in flight; fewer CTAs per SM only
     // when even 2 stages do not fit.
     stages = 2;
-    for (int per = kTargetCtasPerSm; per >= 1; --per) {
+    const int target_per_sm = pl.cache_kind == TC_FP8 ? 2 : kTargetCtasPerSm;
+    for (int per = target_per_sm; per >= 1; --per) {
       const size_t budget = (size_t)kSmemPerSm / per - 1024;
       if (budget < fixed) continue;
       const int fit = (int)std::min<size_t>(kMaxStages, (budget - fixed) / pl.stage_bytes);
@@ -978,7 +981,8 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.smem_bytes = (size_t)stages * pl.stage_bytes + fixed;
   if (pl.smem_bytes > (size_t)optin) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   // CTAs resident per SM from shared memory alone (1 KB reserved per CTA).
-  const int per_sm = std::max(1, std::min(kTargetCtasPerSm, (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
+  const int per_sm = std::max(1, std::min(pl.cache_kind == TC_FP8 ? 2 : kTargetCtasPerSm,
+                                          (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
   const int want_ctas = tuning ? tuning->num_ctas : 0;
   pl.overlap_prologue = tuning && (tuning->flags & PKV_TUNE_OVERLAP_PROLOGUE);
   pl.num_ctas = want_ctas > 0 ? want_ctas : sms * per_sm;

@@ -72,6 +72,10 @@ pkv_status launch_cache_write(const void* key, const void* value, void* key_cach
                               int block_size, int64_t num_blocks, pkv_dtype act, pkv_dtype cache, int32_t* device_error,
                               cudaStream_t stream);
 
+pkv_status launch_move_blocks(const void* const src[4], void* const dst[4], const size_t bytes_per_block[4], int npools,
+                              const int64_t* pairs, int64_t num_pairs, int64_t src_blocks, int64_t dst_blocks,
+                              int32_t* device_error, cudaStream_t stream);
+
 // Records the CUDA error text for pkv_last_cuda_error() and returns PKV_ERR_CUDA.
 pkv_status cuda_fail(cudaError_t e, const char* where);
 pkv_status driver_fail(int code, const char* where);

@@ -69,6 +69,10 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_decode_step_ex.restype = i32
     lib.pkv_paged_attention_decode_static.argtypes = decode_args[:20] + [vp, vp]
     lib.pkv_paged_attention_decode_static.restype = i32
+    lib.pkv_copy_blocks.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i32, vp, vp]
+    lib.pkv_copy_blocks.restype = i32
+    lib.pkv_swap_blocks.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, i64, vp, i64, i32, i32, i32, i32, vp, vp]
+    lib.pkv_swap_blocks.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_cuda_error.argtypes = []
@@ -240,3 +244,24 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     if st != 0:
         raise PkvError(st, "pkv_paged_attention_decode_static", lib.pkv_last_cuda_error().decode())
     return out
+
+
+def copy_blocks(key_cache, value_cache, block_mapping, k_scale=None, v_scale=None, device_error=None, stream=None):
+    """Copy-on-write block copies inside one pool; ``block_mapping`` int64 [P, 2] = (src, dst)."""
+    nb, bs, n_kv, d = key_cache.shape
+    st = lib.pkv_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_mapping),
+                             block_mapping.shape[0], n_kv, d, bs, nb, cache_code(key_cache), _ptr(device_error),
+                             stream if stream is not None else _stream(key_cache.device))
+    _check(st, "pkv_copy_blocks")
+
+
+def swap_blocks(src_key, src_value, dst_key, dst_value, block_mapping, src_k_scale=None, src_v_scale=None,
+                dst_k_scale=None, dst_v_scale=None, device_error=None, device=None):
+    """Move blocks between two pools (either may be pinned host memory); (src, dst) pairs."""
+    snb, bs, n_kv, d = src_key.shape
+    dev = device if device is not None else (src_key.device if src_key.is_cuda else dst_key.device)
+    st = lib.pkv_swap_blocks(_ptr(src_key), _ptr(src_value), _ptr(src_k_scale), _ptr(src_v_scale), snb,
+                             _ptr(dst_key), _ptr(dst_value), _ptr(dst_k_scale), _ptr(dst_v_scale), dst_key.shape[0],
+                             _ptr(block_mapping), block_mapping.shape[0], n_kv, d, bs, cache_code(src_key),
+                             _ptr(device_error), _stream(dev))
+    _check(st, "pkv_swap_blocks")
