@@ -117,6 +117,23 @@ def attention_one_sequence(q, K, V, sm_scale: float, return_weights: bool = Fals
     return out, lse
 
 
+def attended_positions(length: int, window: int = 0, sinks: int = 0) -> np.ndarray:
+    """Positions a new token attends to under a sliding window with sinks.
+
+    Sliding window ("KV Cache Engineering for LLM Serving", section 3): only the
+    latest ``window`` positions are kept; each new entry removes the oldest
+    once the window is full.  Attention sinks ("Chapter 18 - KV-Cache
+    Optimization Strategies", Token Eviction and Pruning, StreamingLLM): the
+    first ``sinks`` positions are always kept as well.  window == 0 keeps
+    every position.
+    """
+    pos = np.arange(length)
+    if window <= 0:
+        return pos
+    keep = (pos >= length - window) | (pos < sinks)
+    return pos[keep]
+
+
 def paged_attention_decode(
     q,
     key_cache,
@@ -127,11 +144,14 @@ def paged_attention_decode(
     cache_dtype: str = "f32",
     k_scale=None,
     v_scale=None,
+    window: int = 0,
+    sinks: int = 0,
 ):
     """Decode attention of S sequences over a paged cache.
 
     For each sequence: gather its K and V rows through its block table
-    (dequantising where the cache is quantised), then attend.  Returns
+    (dequantising where the cache is quantised), keep the attended positions
+    (all of them, or a sliding window plus sinks), then attend.  Returns
     (out [S, n_q, d], lse [S, n_q]) in float64.
     """
     q = np.asarray(q)
@@ -143,6 +163,9 @@ def paged_attention_decode(
         L = int(context_lens[s])
         K = gather_dequantized(key_cache, k_scale, block_tables[s], L, block_size, cache_dtype)
         V = gather_dequantized(value_cache, v_scale, block_tables[s], L, block_size, cache_dtype)
+        if window > 0:
+            keep = attended_positions(L, window, sinks)
+            K, V = K[keep], V[keep]
         out[s], lse[s] = attention_one_sequence(q[s], K, V, sm_scale)
     return out, lse
 

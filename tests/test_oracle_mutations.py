@@ -112,3 +112,18 @@ def test_swap_ignoring_destination_slot_is_caught(monkeypatch):
     monkeypatch.setattr(bpins, "swap_blocks",
                         lambda s, d, pairs: real(s, d, np.stack([np.asarray(pairs)[:, 0]] * 2, axis=1)))
     _fails(lambda: bpins.test_offload_example(read_golden))
+
+
+def test_window_off_by_one_is_caught(monkeypatch):
+    import numpy as np
+
+    def shifted(length, window=0, sinks=0):
+        pos = np.arange(length)
+        if window <= 0:
+            return pos
+        return pos[(pos > length - window) | (pos < sinks)]
+
+    import test_oracle_window as wpins
+
+    monkeypatch.setattr(pa, "attended_positions", shifted)
+    _fails(lambda: wpins.test_sliding_window_example(read_golden))
