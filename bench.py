@@ -248,7 +248,7 @@ def replica_workload(base, rank):
     return workloads.make_workload(
         base.name, seed=base.seed + 1000 * rank, context_lens=base.context_lens, n_q=base.n_q, n_kv=base.n_kv,
         head_dim=base.head_dim, cache_dtype=base.cache_dtype, shared_prefix_tokens=base.shared_prefix_tokens,
-        outlier_fraction=0.01 if base.k_outlier_channels is not None else 0.0)
+        outlier_fraction=0.01 if base.k_outlier_channels is not None else 0.0, window=base.window, sinks=base.sinks)
 
 
 def max_over_ranks(values, world, device=None):
@@ -342,11 +342,21 @@ def run_b200(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
 
+    if w.window:
+        args.unfused = True  # the windowed decode has no fused-append entry point
+
+    def decode(out, q, bt, cl):
+        if w.window:
+            ops.paged_attention_decode_window(out, q, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
+                                              w.sm_scale, ks, vs, workspace=ws, device_error=err)
+        else:
+            ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
+                                       device_error=err)
+
     def step(q=q, k_new=k_new, v_new=v_new, bt=bt, cl=cl, slots=slots, overlap=True):
         if args.unfused:
             ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
-            ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                       device_error=err)
+            decode(out, q, bt, cl)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
                                   workspace=ws, device_error=err, tuning=tuning if overlap else None)
@@ -381,8 +391,7 @@ def run_b200(args, rank, world, local):
         if args.unfused:
             ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
             att[k][0].record(stream)
-            ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                       device_error=err)
+            decode(out, q, bt, cl)
             att[k][1].record(stream)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,

@@ -162,6 +162,27 @@ pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, 
                                  void* workspace, size_t workspace_bytes, int32_t* device_error, void* stream);
 
 /*
+ * Decode attention over a sliding window with attention sinks.
+ *
+ * Like pkv_paged_attention_decode, but sequence s attends only to positions
+ * p < min(sinks, L) and p >= L - window (L = context_lens[s]); window == 0
+ * attends to every position.  A local layer keeps only its latest `window`
+ * positions ("KV Cache Engineering for LLM Serving", section 3, Sliding
+ * windows); StreamingLLM keeps the first tokens as attention sinks plus a recent
+ * window ("Chapter 18 - KV-Cache Optimization Strategies", Token Eviction and
+ * Pruning).  Blocks holding no attended position are never read, so their
+ * block-table entries may be -1 once the engine has freed them.
+ */
+pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const void* key_cache,
+                                             const void* value_cache, const float* k_scale, const float* v_scale,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                             int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                             float sm_scale, int window, int sinks, pkv_dtype act_dtype,
+                                             pkv_dtype cache_dtype, float* lse_out, void* workspace,
+                                             size_t workspace_bytes, int32_t* device_error, void* stream);
+
+/*
  * Launch shape overrides for pkv_paged_attention_decode_ex (0 = automatic).
  * num_ctas: persistent CTAs sharing the blocks of all (sequence, KV-head group)
  * pairs; stages: depth of the shared-memory ring of K/V blocks; heads_per_cta:

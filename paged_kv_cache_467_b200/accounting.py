@@ -45,7 +45,11 @@ def decode_kv_bytes(w, unique: bool = True) -> int:
     """
     per_token = cache_bytes(1, w.n_kv, w.head_dim, 1, BYTES_PER_VALUE[w.cache_dtype])
     per_token += scale_bytes_per_token(w.cache_dtype, w.n_kv)
-    tokens = int(w.context_lens.astype("int64").sum())
+    lens = w.context_lens.astype("int64")
+    if getattr(w, "window", 0) > 0:
+        # attended positions only: [0, sinks) and [L - window, L)
+        lens = lens.clip(max=w.window + w.sinks)
+    tokens = int(lens.sum())
     if unique and w.shared_prefix_tokens:
         tokens -= (w.num_seqs - 1) * w.shared_prefix_tokens
     return int(tokens * per_token)

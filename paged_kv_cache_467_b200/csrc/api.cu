@@ -84,7 +84,8 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
                               int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks, float sm_scale,
                               pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out, void* workspace,
                               size_t workspace_bytes, int32_t* device_error, const pkv_decode_tuning* tuning,
-                              void* stream, const void* new_key = nullptr, const void* new_value = nullptr) {
+                              void* stream, const void* new_key = nullptr, const void* new_value = nullptr,
+                              int window = 0, int sinks = 0) {
   const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, act_dtype, cache_dtype};
   pkv_status st = check_decode_shape(s);
   if (st != PKV_OK) return st;
@@ -97,9 +98,11 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   if (quant && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale))) return PKV_ERR_INVALID_ARG;
   if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
   if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
+  if (window < 0 || sinks < 0) return PKV_ERR_INVALID_ARG;
 
   TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
-           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error, new_key, new_value};
+           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error, new_key, new_value, window,
+           sinks};
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (cache_dtype == PKV_F32) return launch_decode_f32(s, a, strm);
   TcPlan plan;
@@ -248,6 +251,20 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
   return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
                      context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream);
+}
+
+pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const void* key_cache,
+                                             const void* value_cache, const float* k_scale, const float* v_scale,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                             int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                             float sm_scale, int window, int sinks, pkv_dtype act_dtype,
+                                             pkv_dtype cache_dtype, float* lse_out, void* workspace,
+                                             size_t workspace_bytes, int32_t* device_error, void* stream) {
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream,
+                     nullptr, nullptr, window, sinks);
 }
 
 pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* key, const void* value, void* key_cache,

@@ -24,6 +24,7 @@ struct F32Params {
   const float* new_value;
   long long num_blocks;
   int max_blocks_per_seq, cap_len, num_seqs, n_q, n_kv, G;
+  int window, sinks;  // attend to [0, sinks) and [L - window, L) only; window 0 = every position
   float sm_scale;
 };
 
@@ -49,7 +50,15 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const F32Params p) {
   }
   float m = -INFINITY, l = 0.f;
   const int32_t* table = p.block_tables + (size_t)s * p.max_blocks_per_seq;
+  // attended positions: [0, s_eff) then [lo_w, L) (one run when they touch)
+  int s_eff = L, lo_w = L;
+  if (p.window > 0 && L > p.window) {
+    s_eff = min(p.sinks, L);
+    lo_w = max(L - p.window, s_eff);
+  }
   for (int pos = 0; pos < L; ++pos) {
+    if (pos == s_eff) pos = lo_w;
+    if (pos >= L) break;
     const int blk = __ldg(table + pos / kBlockSize);
     if (blk < 0 || (long long)blk >= p.num_blocks) {
       flag_error(p.err, DEVERR_BLOCK_RANGE);
@@ -114,6 +123,8 @@ pkv_status launch_decode_f32(const DecodeShape& sh, const TcArgs& a, cudaStream_
   p.n_kv = sh.n_kv;
   p.G = sh.n_q / sh.n_kv;
   p.sm_scale = a.sm_scale;
+  p.window = a.window;
+  p.sinks = a.sinks;
   const long long warps = (long long)sh.num_seqs * sh.n_q;
   const int threads = 128;
   const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);

@@ -61,6 +61,7 @@ struct TcParams {
   int cap_len;  // min(max_context_len, max_blocks_per_seq * 16)
   int max_context_len;
   int num_seqs, n_q, n_kv;
+  int window, sinks;  // attend to [0, sinks) and [L - window, L) only; window 0 = every position
   int G, QC, HPC, HG, NCW, stages, units;
   float scale_log2;
   int act_bf16;
@@ -87,6 +88,51 @@ __device__ __forceinline__ int seq_len(const TcParams& p, int s, bool report) {
   return L;
 }
 
+// The blocks a sequence of length L attends to, in order: all of them, or the
+// blocks holding the sink positions [0, s_eff) followed by those holding the
+// window [lo_w, L) (one contiguous run when the two touch).
+struct AttendSet {
+  int nb;           // blocks in the set
+  int sink_blocks;  // set index j < sink_blocks is logical block j
+  int win_first;    // set index j >= sink_blocks is logical block win_first + j - sink_blocks
+  int s_eff, lo_w;  // attended positions: p < s_eff or lo_w <= p < L
+};
+
+__device__ __forceinline__ AttendSet attend_set(const TcParams& p, int L) {
+  AttendSet a;
+  const int nbl = (L + kBlockSize - 1) / kBlockSize;
+  a.nb = a.sink_blocks = a.win_first = nbl;
+  a.s_eff = L;
+  a.lo_w = 0;
+  if (p.window > 0 && L > p.window) {
+    a.lo_w = L - p.window;
+    a.s_eff = min(p.sinks, L);
+    if (a.lo_w <= a.s_eff) {
+      a.s_eff = L;  // sinks reach the window: every position
+      a.lo_w = 0;
+    } else {
+      const int sb = (a.s_eff + kBlockSize - 1) / kBlockSize, wb0 = a.lo_w / kBlockSize;
+      if (wb0 >= sb) {
+        a.sink_blocks = sb;
+        a.win_first = wb0;
+        a.nb = sb + (nbl - wb0);
+      }
+    }
+  }
+  return a;
+}
+
+__device__ __forceinline__ int logical_block(const AttendSet& a, int j) {
+  return j < a.sink_blocks ? j : a.win_first + (j - a.sink_blocks);
+}
+
+// Rows of logical block lb that are attended: bit r <=> position lb*16 + r.
+__device__ __forceinline__ uint32_t token_mask(const AttendSet& a, int L, int lb) {
+  const int base = lb * kBlockSize;
+  auto below = [](int n) -> uint32_t { return n <= 0 ? 0u : (n >= kBlockSize ? 0xFFFFu : (1u << n) - 1u); };
+  return below(L - base) & (below(a.s_eff - base) | (0xFFFFu & ~below(a.lo_w - base)));
+}
+
 // First index i in [0, n) with P[i] > x (n if none).
 __device__ __forceinline__ int upper_bound_smem(const int* P, int n, int x) {
   int lo = 0, hi = n;
@@ -107,7 +153,7 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
   int local = 0;
   for (int u = u0; u < u1; ++u) {
     const int s = u / p.HG;
-    local += (seq_len(p, s, (u % p.HG) == 0) + kBlockSize - 1) / kBlockSize;
+    local += attend_set(p, seq_len(p, s, (u % p.HG) == 0)).nb;
   }
   int x = local;
 #pragma unroll
@@ -131,7 +177,7 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
   int run = wsum[warp] + x - local;
   for (int u = u0; u < u1; ++u) {
     P[u] = run;
-    run += (seq_len(p, u / p.HG, false) + kBlockSize - 1) / kBlockSize;
+    run += attend_set(p, seq_len(p, u / p.HG, false)).nb;
   }
   if (u1 == units && u0 < u1) P[units] = run;
   if (units == 0 && t == 0) P[0] = 0;
@@ -276,7 +322,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const int s = u / p.HG;
         hg = u - s * p.HG;
         unit_last = (i + 1 == P[u + 1]);
-        phys = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + (i - P[u]));
+        const int lb = logical_block(attend_set(p, seq_len(p, s, false)), i - P[u]);
+        phys = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + lb);
         if (phys < 0 || (long long)phys >= p.num_blocks) {
           flag_error(p.err, DEVERR_BLOCK_RANGE);
           phys = -1;
@@ -417,6 +464,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   int u = u_first;
   int j = a - P[u];
   int s = 0, hg = 0, L = 0;
+  AttendSet aset{};
   float head_k_scale = 1.f, head_v_scale = 1.f;
 
   uint32_t qf[KS][2];
@@ -457,7 +505,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   // [16 tokens x 8 heads] in log2 units, -inf past the sequence end.
   // sv = (token g, head 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); vsc = int8 V
   // scales of tokens g and g+8 (1 otherwise).
-  auto block_scores = [&](const uint8_t* st, int valid, float (&sv)[4], float (&vsc)[2]) {
+  auto block_scores = [&](const uint8_t* st, uint32_t vm, float (&sv)[4], float (&vsc)[2]) {
     const uint32_t kt = smem_addr(st + head_local * Tr::kTile);
     const int t0 = g, t1 = g + 8;
     // ---- S^T = K Q^T : [16 tokens x 8 heads]
@@ -515,7 +563,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       sc0 *= head_k_scale;
       sc1 *= head_k_scale;
     }
-    const bool ok0 = t0 < valid, ok1 = t1 < valid;
+    const bool ok0 = (vm >> t0) & 1u, ok1 = (vm >> t1) & 1u;
     sv[0] = ok0 ? (sa[0] + sb[0]) * sc0 : -INFINITY;
     sv[1] = ok0 ? (sa[1] + sb[1]) * sc0 : -INFINITY;
     sv[2] = ok1 ? (sa[2] + sb[2]) * sc1 : -INFINITY;
@@ -523,9 +571,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   };
 
   // O^T += V^T P^T for one block with probabilities pr (layout of the scores).
-  auto block_pv = [&](const uint8_t* st, int valid, const float (&pr)[4], const float (&vsc)[2]) {
+  auto block_pv = [&](const uint8_t* st, uint32_t vm, const float (&pr)[4], const float (&vsc)[2]) {
     const uint32_t vt = smem_addr(st + (p.HPC + head_local) * Tr::kTile);
-    const bool ok0 = g < valid, ok1 = g + 8 < valid;
+    const bool ok0 = (vm >> g) & 1u, ok1 = (vm >> (g + 8)) & 1u;
     uint32_t pb0, pb1;
     if constexpr (CACHE == TC_BF16) {
       pb0 = movmatrix_trans(pack_bf16(pr[0], pr[1]));
@@ -539,10 +587,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     }
     // token pairs of the A fragments: (2c, 2c+1) and (2c+8, 2c+9)
     uint32_t mlo = 0xFFFFFFFFu, mhi = 0xFFFFFFFFu;
-    const bool partial = valid < kBlockSize;
+    const bool partial = vm != 0xFFFFu;
     if (partial) {
-      mlo = (2 * c < valid ? 0x0000FFFFu : 0u) | (2 * c + 1 < valid ? 0xFFFF0000u : 0u);
-      mhi = (2 * c + 8 < valid ? 0x0000FFFFu : 0u) | (2 * c + 9 < valid ? 0xFFFF0000u : 0u);
+      mlo = ((vm >> (2 * c)) & 1u ? 0x0000FFFFu : 0u) | ((vm >> (2 * c + 1)) & 1u ? 0xFFFF0000u : 0u);
+      mhi = ((vm >> (2 * c + 8)) & 1u ? 0x0000FFFFu : 0u) | ((vm >> (2 * c + 9)) & 1u ? 0xFFFF0000u : 0u);
     }
     if constexpr (CACHE == TC_BF16) {
 #pragma unroll
@@ -599,13 +647,14 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   auto step = [&](auto nb_const) -> bool {
     constexpr int NB = decltype(nb_const)::value;
     const uint8_t* st[NB];
-    int stage[NB], valid[NB];
+    int stage[NB];
+    uint32_t valid[NB];  // attended-row masks
 #pragma unroll
     for (int k = 0; k < NB; ++k) {
       stage[k] = (it + k) % p.stages;
       if (!mbar_wait(&full[stage[k]], ((it + k) / p.stages) & 1)) return false;
       st[k] = smem + (size_t)stage[k] * p.stage_bytes;
-      valid[k] = min(kBlockSize, L - (j + k) * kBlockSize);
+      valid[k] = token_mask(aset, L, logical_block(aset, j + k));
     }
     float sv[NB][4], vsc[NB][2];
 #pragma unroll
@@ -667,6 +716,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       s = u / p.HG;
       hg = u - s * p.HG;
       L = seq_len(p, s, false);
+      aset = attend_set(p, L);
       if constexpr (CACHE == TC_BF16) {
         fetch_query(u);
 #pragma unroll
@@ -900,6 +950,8 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.num_seqs = s.num_seqs;
   prm.n_q = s.n_q;
   prm.n_kv = s.n_kv;
+  prm.window = a.window;
+  prm.sinks = a.sinks;
   prm.G = plan.G;
   prm.QC = plan.QC;
   prm.HPC = plan.HPC;

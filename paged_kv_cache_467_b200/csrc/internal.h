@@ -61,6 +61,9 @@ struct TcArgs {
   // L-1 of each sequence before the attention (the caches are then written)
   const void* new_key = nullptr;
   const void* new_value = nullptr;
+  // sliding window with sinks: attend to [0, sinks) and [L - window, L); 0 = all
+  int window = 0;
+  int sinks = 0;
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);

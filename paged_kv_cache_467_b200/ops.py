@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_decode_step_ex.restype = i32
     lib.pkv_paged_attention_decode_static.argtypes = decode_args[:20] + [vp, vp]
     lib.pkv_paged_attention_decode_static.restype = i32
+    lib.pkv_paged_attention_decode_window.argtypes = decode_args[:17] + [i32, i32] + decode_args[17:] + [vp]
+    lib.pkv_paged_attention_decode_window.restype = i32
     lib.pkv_copy_blocks.argtypes = [vp, vp, vp, vp, vp, i64, i32, i32, i32, i64, i32, vp, vp]
     lib.pkv_copy_blocks.restype = i32
     lib.pkv_swap_blocks.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, i64, vp, i64, i32, i32, i32, i32, vp, vp]
@@ -265,3 +267,26 @@ def swap_blocks(src_key, src_value, dst_key, dst_value, block_mapping, src_k_sca
                              _ptr(block_mapping), block_mapping.shape[0], n_kv, d, bs, cache_code(src_key),
                              _ptr(device_error), _stream(dev))
     _check(st, "pkv_swap_blocks")
+
+
+def paged_attention_decode_window(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
+                                  window: int, sinks: int = 0, sm_scale: float | None = None, k_scale=None,
+                                  v_scale=None, lse_out=None, workspace=None, device_error=None):
+    """Decode attention over positions [0, sinks) and [L - window, L) of each sequence."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ccode = cache_code(key_cache)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.pkv_paged_attention_decode_window(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
+        float(sm_scale), int(window), int(sinks), act_code(query), ccode, _ptr(lse_out), _ptr(workspace), ws_bytes,
+        _ptr(device_error), _stream(query.device),
+    )
+    _check(st, "pkv_paged_attention_decode_window")
+    return out

@@ -96,6 +96,8 @@ class DecodeWorkload:
     shared_prefix_blocks: np.ndarray | None = None
     k_outlier_channels: np.ndarray | None = None  # flat (head * d + dim) indices
     outlier_factor: float = 10.0
+    window: int = 0  # sliding window (0 = attend to every position)
+    sinks: int = 0  # attention sinks kept with the window
     _prefix_cache: tuple | None = field(default=None, repr=False)
 
     # ----------------------------------------------------------------- sizes
@@ -272,6 +274,8 @@ def make_workload(
     extra_blocks: int = 0,
     shared_prefix_tokens: int = 0,
     outlier_fraction: float = 0.0,
+    window: int = 0,
+    sinks: int = 0,
 ) -> DecodeWorkload:
     """Generic workload from explicit lengths (used by the parity tests)."""
     assert act_dtype in DTYPES[:2] and cache_dtype in DTYPES
@@ -303,6 +307,8 @@ def make_workload(
         shared_prefix_tokens=shared_prefix_tokens,
         shared_prefix_blocks=shared if pblocks else None,
         k_outlier_channels=outliers,
+        window=window,
+        sinks=sinks,
     )
 
 
@@ -378,6 +384,14 @@ def quantized(cache_dtype: str = "int8", seed: int = 4) -> DecodeWorkload:
     )
 
 
+def sliding_window(seed: int = 1) -> DecodeWorkload:
+    """The Llama-3-8B-shaped step on a local layer: 1024-token window plus 4 sinks."""
+    w = llama3_8b(seed)
+    w.name = "window1024_sinks4_b64_32q8kv_d128_bf16"
+    w.window, w.sinks = 1024, 4
+    return w
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama3_8b": llama3_8b,
@@ -385,4 +399,5 @@ CONFIGS = {
     "prefix": prefix_sharing,
     "int8": lambda: quantized("int8"),
     "fp8": lambda: quantized("fp8_e4m3", seed=5),
+    "window": sliding_window,
 }

@@ -128,7 +128,7 @@ def run_decode(w, st: GpuState, tuning=None, workspace=None, block_tables=None):
 
 
 # ------------------------------------------------------------------ oracle side
-def oracle_sequence(w, s, fp8_scales=None):
+def oracle_sequence(w, s, fp8_scales=None, window=0, sinks=0):
     """Oracle (out [n_q, d], lse [n_q], written rows) for sequence s.
 
     The sequence's rows are appended by ``oracle.kv_cache_write`` into a compact
@@ -151,7 +151,7 @@ def oracle_sequence(w, s, fp8_scales=None):
     oracle.kv_cache_write(K, V, kc, vc, np.arange(L, dtype=np.int64), w.cache_dtype, ks, vs)
     table = np.arange(nb, dtype=np.int32)[None]
     out, lse = oracle.paged_attention_decode(w.query()[s : s + 1], kc, vc, table, np.array([L]), w.sm_scale,
-                                             w.cache_dtype, ks, vs)
+                                             w.cache_dtype, ks, vs, window=window, sinks=sinks)
     return out[0], lse[0], (kc, vc, ks, vs)
 
 
