@@ -23,3 +23,4 @@ from .paged_attention import (  # noqa: F401
     paged_attention_decode,
 )
 from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402
+from .quest import page_scores, page_summaries, quest_decode, select_pages  # noqa: F401,E402

@@ -127,3 +127,28 @@ def test_window_off_by_one_is_caught(monkeypatch):
 
     monkeypatch.setattr(pa, "attended_positions", shifted)
     _fails(lambda: wpins.test_sliding_window_example(read_golden))
+
+
+def test_quest_score_without_min_is_caught(monkeypatch):
+    import numpy as np
+
+    import oracle.quest as oq
+    import test_oracle_quest as qpins
+
+    def max_only(q, mins, maxs):
+        q = np.asarray(q, dtype=np.float64)
+        n_q, n_kv = q.shape[0], mins.shape[1]
+        return np.stack([(q[h] * maxs[:, h // (n_q // n_kv), :]).sum(axis=1) for h in range(n_q)])
+
+    monkeypatch.setattr(oq, "page_scores", max_only)
+    _fails(qpins.check_upper_bound)
+
+
+def test_quest_selecting_lowest_scores_is_caught(monkeypatch):
+    import numpy as np
+
+    import oracle.quest as oq
+    import test_oracle_quest as qpins
+
+    monkeypatch.setattr(oq, "select_pages", lambda s, k: np.sort(np.argsort(np.asarray(s))[: min(k, len(s))]))
+    _fails(lambda: qpins.test_quest_worked_example(read_golden))
