@@ -23,4 +23,5 @@ from .paged_attention import (  # noqa: F401
     paged_attention_decode,
 )
 from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402
-from .quest import page_scores, page_summaries, quest_decode, select_pages  # noqa: F401,E402
+from .quest import (decode_over_pages, group_scores, page_scores, page_summaries, quest_decode,  # noqa: F401,E402
+                    select_pages)

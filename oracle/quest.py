@@ -28,6 +28,8 @@ def page_summaries(keys, page_size: int):
     keys = np.asarray(keys, dtype=np.float64)
     L = keys.shape[0]
     pages = -(-L // page_size)
+    if pages == 0:  # an empty sequence has no pages
+        return np.zeros((0,) + keys.shape[1:]), np.zeros((0,) + keys.shape[1:])
     mins = np.stack([keys[j * page_size : min((j + 1) * page_size, L)].min(axis=0) for j in range(pages)])
     maxs = np.stack([keys[j * page_size : min((j + 1) * page_size, L)].max(axis=0) for j in range(pages)])
     return mins, maxs
@@ -59,6 +61,39 @@ def select_pages(scores, k: int):
     return np.array(sorted(order[: min(k, len(scores))]), dtype=np.int64)
 
 
+def decode_over_pages(q, key_cache, value_cache, block_row, length: int, sm_scale: float, pages,
+                      cache_dtype: str = "f32", k_scale=None, v_scale=None):
+    """Decode one sequence, KV head kv attending only to the rows of logical pages ``pages[kv]``.
+
+    ``pages`` [n_kv, k]: page indices below ceil(length / block_size); a -1 entry
+    and all after it are ignored.  Returns (out [n_q, d], lse [n_q]); a head with
+    no page gets a zero output and lse -inf.
+    """
+    block_size = key_cache.shape[1]
+    K = gather_dequantized(key_cache, k_scale, block_row, length, block_size, cache_dtype)
+    V = gather_dequantized(value_cache, v_scale, block_row, length, block_size, cache_dtype)
+    q = np.asarray(q, dtype=np.float64)
+    n_q, d = q.shape
+    n_kv = K.shape[1]
+    g = n_q // n_kv
+    out = np.zeros((n_q, d))
+    lse = np.full(n_q, -np.inf)
+    for kv in range(n_kv):
+        listed = []
+        for j in pages[kv]:
+            if j < 0:
+                break
+            assert j * block_size < length, "page past the sequence"
+            listed.append(int(j))
+        if not listed:
+            continue
+        rows = np.concatenate([np.arange(j * block_size, min((j + 1) * block_size, length)) for j in listed])
+        o, l = attention_one_sequence(q[kv * g : (kv + 1) * g], K[rows][:, kv : kv + 1], V[rows][:, kv : kv + 1],
+                                      sm_scale)
+        out[kv * g : (kv + 1) * g], lse[kv * g : (kv + 1) * g] = o, l
+    return out, lse
+
+
 def quest_decode(q, key_cache, value_cache, block_row, length: int, sm_scale: float, k_pages: int,
                  cache_dtype: str = "f32", k_scale=None, v_scale=None):
     """Decode one sequence reading only each KV head's k best pages.
@@ -67,19 +102,10 @@ def quest_decode(q, key_cache, value_cache, block_row, length: int, sm_scale: fl
     """
     block_size = key_cache.shape[1]
     K = gather_dequantized(key_cache, k_scale, block_row, length, block_size, cache_dtype)
-    V = gather_dequantized(value_cache, v_scale, block_row, length, block_size, cache_dtype)
-    q = np.asarray(q, dtype=np.float64)
-    n_q, d = q.shape
     n_kv = K.shape[1]
     mins, maxs = page_summaries(K, block_size)
     chosen = group_scores(page_scores(q, mins, maxs), n_kv)
-    selected = np.stack([select_pages(chosen[kv], k_pages) for kv in range(n_kv)])
-    out = np.zeros((n_q, d))
-    lse = np.zeros(n_q)
-    g = n_q // n_kv
-    for kv in range(n_kv):
-        rows = np.concatenate([np.arange(j * block_size, min((j + 1) * block_size, length)) for j in selected[kv]])
-        o, l = attention_one_sequence(q[kv * g : (kv + 1) * g], K[rows][:, kv : kv + 1], V[rows][:, kv : kv + 1],
-                                      sm_scale)
-        out[kv * g : (kv + 1) * g], lse[kv * g : (kv + 1) * g] = o, l
+    selected = np.stack([select_pages(chosen[kv], k_pages) for kv in range(n_kv)]).reshape(n_kv, -1)
+    out, lse = decode_over_pages(q, key_cache, value_cache, block_row, length, sm_scale, selected, cache_dtype,
+                                 k_scale, v_scale)
     return out, lse, selected

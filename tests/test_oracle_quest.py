@@ -96,3 +96,27 @@ def test_quest_decode_attends_over_selected_rows():
         worst_chosen = grp[kv, sel[kv]].min()
         rest = np.delete(grp[kv], sel[kv])
         assert (rest <= worst_chosen).all()
+
+
+def test_decode_over_listed_pages():
+    """Listing every page is full attention; -1 ends a list; an empty list is
+    the empty sum (zero output, lse -inf); each head sees only its own list."""
+    kc, vc, table, K, V, q = _pool(3, 90)  # 6 pages, the last one partial
+    full, lse_full = paged_attention_decode(q[None], kc, vc, table[None], [90], 0.25)
+    out, lse = oq.decode_over_pages(q, kc, vc, table, 90, 0.25, np.array([[0, 1, 2, 3, 4, 5], [0, 1, 2, 3, 4, 5]]))
+    np.testing.assert_allclose(out, full[0], atol=1e-12)
+    np.testing.assert_allclose(lse, lse_full[0], atol=1e-12)
+    out, lse = oq.decode_over_pages(q, kc, vc, table, 90, 0.25, np.array([[1, 5, -1, 3], [-1, -1, -1, -1]]))
+    rows = np.r_[16:32, 80:90]
+    np.testing.assert_allclose(out[:4], sdpa_reference(q[:4], K[rows][:, :1], V[rows][:, :1], 0.25), atol=1e-12)
+    assert (out[4:] == 0).all() and np.isneginf(lse[4:]).all()
+
+
+def test_empty_sequence_has_no_pages():
+    """Length 0: no page, nothing selected, zero output and lse -inf (the
+    empty-sum reading of the decode)."""
+    kc, vc, table, K, V, q = _pool(4, 40)
+    mins, maxs = oq.page_summaries(K[:0], 16)
+    assert mins.shape == (0, 2, 16) and maxs.shape == (0, 2, 16)
+    out, lse, sel = oq.quest_decode(q, kc, vc, table, 0, 0.25, k_pages=3)
+    assert sel.shape == (2, 0) and (out == 0).all() and np.isneginf(lse).all()
