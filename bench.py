@@ -42,10 +42,12 @@ def parse_args():
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--config", default="llama3_8b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--unfused", action="store_true", help="append and decode as two launches")
+    ap.add_argument("--unfused", action="store_true", help="append in its own launch before the decode")
     ap.add_argument("--no-overlap", action="store_true", help="launch each step without overlapping its prologue")
-    ap.add_argument("--op", default="decode_step", choices=["decode_step", "copy_blocks", "swap_blocks"],
+    ap.add_argument("--op", default="decode_step", choices=["decode_step", "copy_blocks", "swap_blocks", "quest"],
                     help="what a step runs (the default is the decode step)")
+    ap.add_argument("--quest-budget", type=int, default=4096,
+                    help="--op quest: tokens each KV head reads (a multiple of the 16-token page)")
     return ap.parse_args()
 
 
@@ -473,16 +475,18 @@ def run_b200(args, rank, world, local):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": traffic,
-                "kernel": "decode_tc_kernel (pkv_paged_attention_decode)" if args.unfused
-                else "decode_tc_kernel with fused append (pkv_paged_decode_step)",
+                "kernel": "decode_tc_kernel + decode_merge_kernel (pkv_paged_attention_decode)" if args.unfused
+                else "decode_tc_kernel with fused append + decode_merge_kernel (pkv_paged_decode_step)",
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "bytes_per_launch": kv_bytes,
                 "launch_ms": att_ms,
             },
             "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
-            "gpu_launches": (2 if args.unfused else 1) * args.steps,
-            "step": ("append + decode, two launches" if args.unfused else "append + decode fused in one launch")
+            # decode kernel + merge of split sequences (+ the cache write when unfused)
+            "gpu_launches": ((1 if w.cache_dtype == "f32" else 2) + (1 if args.unfused else 0)) * args.steps,
+            "step": ("append, then decode + merge of split sequences" if args.unfused
+                     else "append fused into the decode kernel, then the merge of split sequences")
             + ("" if args.no_overlap or args.unfused else "; prologue overlaps the previous step (programmatic launch)"),
             "clocks": clocks,
         }
@@ -561,11 +565,143 @@ def run_block_ops(args):
     }), flush=True)
 
 
+def run_quest(args):
+    """--op quest: one decode step with query-aware page selection.  A step
+    appends the new token, refreshes the summary of each sequence's last page,
+    scores every page and keeps each KV head's best budget / 16 pages, then
+    attends over those pages only.  The full fused decode step on the same
+    cache is timed beside it."""
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_467_b200 import ops, workloads
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workloads.CONFIGS[args.config]()
+    if w.cache_dtype != "bf16" or w.window:
+        raise SystemExit("--op quest runs on a bf16 cache without a window")
+    S, nq, nkv, d, bs = w.num_seqs, w.n_q, w.n_kv, w.head_dim, w.block_size
+    gen = torch.Generator(device=dev).manual_seed(99)
+    shape = (w.num_blocks, bs, nkv, d)
+    kc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+    vc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+    q = torch.randn((S, nq, d), device=dev, generator=gen).to(torch.bfloat16)
+    k_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    v_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    slots = torch.from_numpy(w.new_token_slots()).to(dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    out = torch.empty_like(q)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    k_pages = max(1, args.quest_budget // bs)
+    pmin = torch.empty((w.num_blocks, nkv, d), dtype=torch.bfloat16, device=dev)
+    pmax = torch.empty_like(pmin)
+    sel = torch.empty((S, nkv, k_pages), dtype=torch.int32, device=dev)
+    scores = torch.empty((S, nkv, -(-min(w.max_context_len, w.max_blocks_per_seq * bs) // bs)), device=dev)
+    ops.quest_page_summaries(kc, pmin, pmax, bt, cl, err)
+    nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc))
+    ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    def quest_step(record=False):
+        if record:
+            ev[0].record(stream)
+        ops.kv_cache_write(k_new, v_new, kc, vc, slots, None, None, err)
+        ops.quest_page_summaries(kc, pmin, pmax, bt, cl, err, last_page_only=True)
+        if record:
+            ev[1].record(stream)
+        ops.quest_select(q, pmin, pmax, bt, cl, w.max_context_len, k_pages, sel, scores, err)
+        if record:
+            ev[2].record(stream)
+        ops.paged_attention_decode_pages(out, q, kc, vc, bt, cl, w.max_context_len, sel, w.sm_scale, workspace=ws,
+                                         device_error=err)
+        if record:
+            ev[3].record(stream)
+
+    def full_step():
+        ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, workspace=ws,
+                              device_error=err)
+
+    for _ in range(max(args.warmup, 3)):
+        quest_step()
+        full_step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0")
+    sampler.start()
+    t_spin = time.perf_counter()
+    while time.perf_counter() - t_spin < 0.4:
+        quest_step()
+        torch.cuda.synchronize()
+    parts = np.zeros(3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        quest_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    n_split = min(args.steps, 200)
+    for _ in range(n_split):  # per-launch split (events between launches)
+        quest_step(record=True)
+        torch.cuda.synchronize()
+        parts += [ev[0].elapsed_time(ev[1]), ev[1].elapsed_time(ev[2]), ev[2].elapsed_time(ev[3])]
+    parts /= n_split
+    e0.record(stream)
+    for _ in range(args.steps):
+        full_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    full_ms = e0.elapsed_time(e1) / args.steps
+    clocks = sampler.stop()
+    assert int(err.item()) == 0, f"device error flag {int(err.item())}"
+
+    # algorithmic bytes: every page summary of every KV head (min and max), the
+    # K and V rows of the selected pages, the refreshed last pages
+    lens = w.context_lens.astype(np.int64)
+    pages = -(-lens // bs)
+    summ_bytes = int(pages.sum()) * nkv * 2 * d * 2
+    sel_h = sel.cpu().numpy()
+    rows = 0
+    for s_ in range(S):
+        for kv in range(nkv):
+            for j in sel_h[s_, kv]:
+                if j >= 0:
+                    rows += min(bs, int(lens[s_]) - int(j) * bs)
+    kv_bytes = rows * d * 2 * 2
+    refresh_bytes = S * (bs * nkv * d * 2 + 2 * nkv * d * 2)
+    total = summ_bytes + kv_bytes + refresh_bytes
+    full_bytes = int(lens.sum()) * nkv * d * 2 * 2
+    peak, peak_kind = measured_peaks()
+    print(json.dumps({
+        "metric": "Quest decode step: tokens/s", "value": S / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic", "config": {"workload": w.name, "budget_tokens": k_pages * bs, "pages_per_head": k_pages,
+                                        "context_tokens": int(lens.sum())},
+        "full_decode_ms_per_step": full_ms, "speedup_vs_full_decode": full_ms / ms,
+        "split_ms": {"append + last-page refresh": parts[0], "quest_select": parts[1], "decode_pages": parts[2]},
+        "bytes_per_step": {"summaries": summ_bytes, "selected_kv": kv_bytes, "refresh": refresh_bytes,
+                           "full_decode_kv": full_bytes},
+        "roofline": {"bound": "hbm", "achieved": total / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": total / (ms * 1e-3) / 1e9 / peak, "traffic": None, "peak_source": f"{peak_kind} hbm_gbs",
+                     "select_gbs": summ_bytes / (parts[1] * 1e-3) / 1e9,
+                     "decode_pages_gbs": kv_bytes / (parts[2] * 1e-3) / 1e9},
+        # append, last-page refresh, page scoring, top-k, decode over pages, merge
+        "gpu_launches": 6 * args.steps, "clocks": clocks,
+    }), flush=True)
+
+
 def main():
     args = parse_args()
     rank, world, local = dist_env()
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.op == "quest":
+        run_quest(args)
         return
     if args.op != "decode_step":
         run_block_ops(args)

@@ -116,13 +116,14 @@ size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int h
  *   max_context_len    host upper bound of context_lens (sizes the launch; no
  *                      device->host read happens)
  *   lse_out            optional device float [num_seqs, n_q]
- *   workspace          device scratch of workspace_bytes; zero-filled once by
- *                      the caller before its first use.  Its first 256 KiB hold
- *                      merge counters at a fixed place for every shape, and each
- *                      call leaves them zeroed, so one workspace serves calls of
- *                      any shape in stream order.  Calls that may run
- *                      concurrently need separate workspaces; after a call
- *                      reports PKV_DEVERR_TIMEOUT, zero the workspace again.
+ *   workspace          device scratch of workspace_bytes (any contents: every
+ *                      byte is written before it is read), 16-byte aligned.
+ *                      One workspace serves calls of any shape in stream order;
+ *                      calls that may run concurrently need separate ones.
+ *
+ * A BF16/INT8/FP8 call makes two launches on `stream`: the decode kernel and,
+ * queued behind it with programmatic stream serialisation, the merge of
+ * sequences whose blocks were split over several CTAs.
  *
  * Supported: block_size 16; act F32 with an F32 cache (head_dim 32..256, a
  * multiple of 32); act BF16 with a BF16 cache (head_dim 64 or 128); act BF16
@@ -183,6 +184,63 @@ pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const
                                              size_t workspace_bytes, int32_t* device_error, void* stream);
 
 /*
+ * Quest, query-aware sparse reads ("KV Cache Engineering for LLM Serving",
+ * section 7).  A page is one cache block.  Each page keeps the element-wise
+ * minimum and maximum of its keys; a query scores a page by
+ * sum_i max(q_i * min_i, q_i * max_i) (an upper bound of q . k for every key of
+ * the page), and only the best pages are read.  Pages are chosen per
+ * (sequence, KV head) by the largest score of that head's query heads; the
+ * k best are kept, ties toward the lower page index.  BF16 and F32 caches,
+ * head_dim 64 or 128, block_size 16.
+ */
+
+/* Page summaries: page_min / page_max [num_blocks, n_kv, head_dim] (device, in
+ * the cache dtype) receive, for each listed block of each sequence, the
+ * element-wise min / max of its keys (the last page over rows < L only).
+ * Blocks shared by several sequences are written with identical values.  With
+ * last_page_only nonzero only the page holding token L-1 of each sequence is
+ * refreshed: the per-step update after appending one token.  A block table
+ * entry outside [0, num_blocks) sets the block-range bit and is skipped; a
+ * length outside [0, max_blocks_per_seq * block_size] sets the context bit. */
+pkv_status pkv_quest_page_summaries(const void* key_cache, void* page_min, void* page_max,
+                                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                                    int num_seqs, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    pkv_dtype cache_dtype, int last_page_only, int32_t* device_error, void* stream);
+
+/* Page selection: selected [num_seqs, n_kv, k_pages] (int32, device) receives
+ * each KV head's min(k_pages, ceil(L / block_size)) best logical pages in
+ * increasing order, -1 after them.  scores (required, device float
+ * [num_seqs, n_kv, ceil(min(max_context_len, max_blocks_per_seq * 16) / 16)])
+ * receives every page's score (entries past a sequence's pages are left as
+ * they are); the selection reads it back.  query [num_seqs, n_q, head_dim] in
+ * act_dtype; page_min / page_max as written by pkv_quest_page_summaries.  Two
+ * launches (scoring, then top-k) on `stream`.  A block table entry outside
+ * [0, num_blocks) sets the block-range bit and gives its page the score -inf. */
+pkv_status pkv_quest_select(const void* query, const void* page_min, const void* page_max,
+                            const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                            int max_context_len, int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                            int64_t num_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype, int k_pages,
+                            int32_t* selected, float* scores, int32_t* device_error, void* stream);
+
+/* Decode attention over listed pages only: KV head kv of sequence s attends
+ * to the tokens of the logical pages pages[s][kv][0 .. k_pages) (int32,
+ * device, strictly increasing; the list ends at its first -1 and every later
+ * entry must be -1 too).  At most min(k_pages, ceil(L / block_size)) entries
+ * are read.  A listed page at or past the sequence's page count sets the
+ * block-range bit of device_error and the outputs are then undefined.
+ * An empty list gives a zero output and lse -inf.  BF16/INT8/FP8/F32 caches as
+ * pkv_paged_attention_decode, whose arguments and results this shares; a
+ * workspace sized by pkv_paged_attention_workspace_size suffices. */
+pkv_status pkv_paged_attention_decode_pages(void* out, const void* query, const void* key_cache,
+                                            const void* value_cache, const float* k_scale, const float* v_scale,
+                                            const int32_t* block_tables, int max_blocks_per_seq,
+                                            const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                            int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                            float sm_scale, const int32_t* pages, int k_pages, pkv_dtype act_dtype,
+                                            pkv_dtype cache_dtype, float* lse_out, void* workspace,
+                                            size_t workspace_bytes, int32_t* device_error, void* stream);
+
+/*
  * Launch shape overrides for pkv_paged_attention_decode_ex (0 = automatic).
  * num_ctas: persistent CTAs sharing the blocks of all (sequence, KV-head group)
  * pairs; stages: depth of the shared-memory ring of K/V blocks; heads_per_cta:
@@ -226,6 +284,20 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
                                          float* lse_out, void* workspace, size_t workspace_bytes, int32_t* device_error,
                                          const pkv_decode_tuning* tuning, void* stream);
 
+/* pkv_paged_attention_decode_pages with explicit launch shape (tuning may be
+ * NULL; heads_per_cta must be 0 or 1: a page list belongs to one KV head).
+ * Size the workspace with pkv_paged_attention_workspace_size_ex and the same
+ * tuning with heads_per_cta 1. */
+pkv_status pkv_paged_attention_decode_pages_ex(void* out, const void* query, const void* key_cache,
+                                               const void* value_cache, const float* k_scale, const float* v_scale,
+                                               const int32_t* block_tables, int max_blocks_per_seq,
+                                               const int32_t* context_lens, int max_context_len, int num_seqs,
+                                               int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                               float sm_scale, const int32_t* pages, int k_pages,
+                                               pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                               void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                               const pkv_decode_tuning* tuning, void* stream);
+
 /*
  * pkv_paged_attention_decode for callers that cannot allocate device memory.
  * This entry point has no counterpart in the paper; it exists for the callers
@@ -247,10 +319,9 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress).  Make that first call before any stream capture
  *     on that device.
- *   - Every call on a device shares the one array.  Each call clears the array's
- *     merge counters (cudaMemsetAsync on `stream`) before launching.  Calls whose
- *     work can overlap on the GPU (different streams, no ordering between them)
- *     race on the array and give wrong results; keep such calls in one stream.
+ *   - Every call on a device shares the one array.  Calls whose work can
+ *     overlap on the GPU (different streams, no ordering between them) race on
+ *     the array and give wrong results; keep such calls in one stream.
  */
 pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const void* key_cache,
                                              const void* value_cache, const float* k_scale, const float* v_scale,

@@ -85,7 +85,7 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
                               pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out, void* workspace,
                               size_t workspace_bytes, int32_t* device_error, const pkv_decode_tuning* tuning,
                               void* stream, const void* new_key = nullptr, const void* new_value = nullptr,
-                              int window = 0, int sinks = 0) {
+                              int window = 0, int sinks = 0, const int32_t* pages = nullptr, int k_pages = 0) {
   const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, act_dtype, cache_dtype};
   pkv_status st = check_decode_shape(s);
   if (st != PKV_OK) return st;
@@ -99,12 +99,19 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
   if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
   if (window < 0 || sinks < 0) return PKV_ERR_INVALID_ARG;
+  if (pages && (k_pages < 1 || window > 0 || new_key)) return PKV_ERR_INVALID_ARG;
 
   TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
            max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error, new_key, new_value, window,
-           sinks};
+           sinks, pages, k_pages};
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (cache_dtype == PKV_F32) return launch_decode_f32(s, a, strm);
+  // a page list is per KV head: one KV head per CTA
+  pkv_decode_tuning one_head = tuning ? *tuning : pkv_decode_tuning{0, 0, 0, 0};
+  if (pages) {
+    one_head.heads_per_cta = 1;
+    tuning = &one_head;
+  }
   TcPlan plan;
   st = plan_tc(s, tuning, &plan);
   if (st != PKV_OK) return st;
@@ -265,6 +272,72 @@ pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const
                      context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream,
                      nullptr, nullptr, window, sinks);
+}
+
+pkv_status pkv_quest_page_summaries(const void* key_cache, void* page_min, void* page_max,
+                                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                                    int num_seqs, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    pkv_dtype cache_dtype, int last_page_only, int32_t* device_error, void* stream) {
+  if (num_seqs < 0 || n_kv <= 0 || head_dim <= 0 || max_blocks_per_seq < 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (block_size != kBlockSize) return PKV_ERR_UNSUPPORTED;
+  if (cache_dtype != PKV_BF16 && cache_dtype != PKV_F32) return PKV_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  if (num_seqs == 0 || max_blocks_per_seq == 0) return PKV_OK;
+  if (!key_cache || !page_min || !page_max || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
+  return launch_quest_summaries(key_cache, page_min, page_max, block_tables, max_blocks_per_seq, context_lens,
+                                num_seqs, n_kv, head_dim, num_blocks, cache_dtype, last_page_only, device_error,
+                                static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_quest_select(const void* query, const void* page_min, const void* page_max,
+                            const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                            int max_context_len, int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                            int64_t num_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype, int k_pages,
+                            int32_t* selected, float* scores, int32_t* device_error, void* stream) {
+  if (num_seqs < 0 || n_q <= 0 || n_kv <= 0 || n_q % n_kv || k_pages < 1 || max_context_len < 0 || num_blocks < 0)
+    return PKV_ERR_INVALID_ARG;
+  if (act_dtype != PKV_BF16 && act_dtype != PKV_F32) return PKV_ERR_INVALID_ARG;
+  if (block_size != kBlockSize) return PKV_ERR_UNSUPPORTED;
+  if (cache_dtype != PKV_BF16 && cache_dtype != PKV_F32) return PKV_ERR_UNSUPPORTED;
+  if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PKV_OK;
+  if (!query || !page_min || !page_max || !block_tables || !context_lens || !selected || !scores)
+    return PKV_ERR_INVALID_ARG;
+  return launch_quest_select(query, page_min, page_max, block_tables, max_blocks_per_seq, context_lens,
+                             max_context_len, num_seqs, n_q, n_kv, head_dim, num_blocks, act_dtype, cache_dtype,
+                             k_pages, selected, scores, device_error, static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_paged_attention_decode_pages(void* out, const void* query, const void* key_cache,
+                                            const void* value_cache, const float* k_scale, const float* v_scale,
+                                            const int32_t* block_tables, int max_blocks_per_seq,
+                                            const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                            int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                            float sm_scale, const int32_t* pages, int k_pages, pkv_dtype act_dtype,
+                                            pkv_dtype cache_dtype, float* lse_out, void* workspace,
+                                            size_t workspace_bytes, int32_t* device_error, void* stream) {
+  return pkv_paged_attention_decode_pages_ex(out, query, key_cache, value_cache, k_scale, v_scale, block_tables,
+                                             max_blocks_per_seq, context_lens, max_context_len, num_seqs, n_q, n_kv,
+                                             head_dim, block_size, num_blocks, sm_scale, pages, k_pages, act_dtype,
+                                             cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr,
+                                             stream);
+}
+
+pkv_status pkv_paged_attention_decode_pages_ex(void* out, const void* query, const void* key_cache,
+                                               const void* value_cache, const float* k_scale, const float* v_scale,
+                                               const int32_t* block_tables, int max_blocks_per_seq,
+                                               const int32_t* context_lens, int max_context_len, int num_seqs,
+                                               int n_q, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                               float sm_scale, const int32_t* pages, int k_pages,
+                                               pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                               void* workspace, size_t workspace_bytes, int32_t* device_error,
+                                               const pkv_decode_tuning* tuning, void* stream) {
+  if (num_seqs > 0 && (!pages || k_pages < 1)) return PKV_ERR_INVALID_ARG;
+  if (tuning && tuning->heads_per_cta > 1) return PKV_ERR_INVALID_ARG;  // a page list is per KV head
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream,
+                     nullptr, nullptr, 0, 0, pages, k_pages);
 }
 
 pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* key, const void* value, void* key_cache,

@@ -25,6 +25,8 @@ struct F32Params {
   long long num_blocks;
   int max_blocks_per_seq, cap_len, num_seqs, n_q, n_kv, G;
   int window, sinks;  // attend to [0, sinks) and [L - window, L) only; window 0 = every position
+  const int32_t* pages;  // Quest: [num_seqs, n_kv, k_pages] logical pages to read (ascending, -1 past the count)
+  int k_pages;
   float sm_scale;
 };
 
@@ -56,8 +58,28 @@ __global__ void __launch_bounds__(128) decode_f32_kernel(const F32Params p) {
     s_eff = min(p.sinks, L);
     lo_w = max(L - p.window, s_eff);
   }
+  const int32_t* plist = p.pages ? p.pages + ((size_t)s * p.n_kv + kv) * p.k_pages : nullptr;
+  const int plen = min(p.k_pages, (L + kBlockSize - 1) / kBlockSize);  // entries read at most
+  int pi = 0;  // next listed page
   for (int pos = 0; pos < L; ++pos) {
-    if (pos == s_eff) pos = lo_w;
+    if (plist) {
+      if (pos % kBlockSize == 0) {
+        // next listed page; the list ends at k_pages entries or its first -1;
+        // a page past the sequence (or out of order) is a range error
+        int pg = -1;
+        while (pi < plen) {
+          pg = __ldg(plist + pi++);
+          if (pg < 0) break;
+          if ((long long)pg * kBlockSize >= pos && (long long)pg * kBlockSize < L) break;
+          if (h % p.G == 0) flag_error(p.err, DEVERR_BLOCK_RANGE);
+          pg = -1;
+        }
+        if (pg < 0) break;
+        pos = pg * kBlockSize;
+      }
+    } else {
+      if (pos == s_eff) pos = lo_w;
+    }
     if (pos >= L) break;
     const int blk = __ldg(table + pos / kBlockSize);
     if (blk < 0 || (long long)blk >= p.num_blocks) {
@@ -125,6 +147,8 @@ pkv_status launch_decode_f32(const DecodeShape& sh, const TcArgs& a, cudaStream_
   p.sm_scale = a.sm_scale;
   p.window = a.window;
   p.sinks = a.sinks;
+  p.pages = a.pages;
+  p.k_pages = a.k_pages;
   const long long warps = (long long)sh.num_seqs * sh.n_q;
   const int threads = 128;
   const unsigned blocks = (unsigned)((warps * 32 + threads - 1) / threads);

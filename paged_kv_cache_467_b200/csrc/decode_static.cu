@@ -6,8 +6,9 @@
 // allocator to plug-ins, or a serving loop that must never call cudaMalloc
 // because cudaMalloc can synchronise the device.  For them,
 // pkv_paged_attention_decode_static runs the same decode kernel as
-// pkv_paged_attention_decode, with its scratch (merge counters and partial
-// results) in one fixed array that is part of the loaded library.
+// pkv_paged_attention_decode, with its scratch (partial results of split
+// sequences and their merge descriptors) in one fixed array that is part of
+// the loaded library.
 //
 // The array below is kStaticScratchBytes (16 MiB) of device memory that every
 // GPU which loads libpkv holds until the process exits.
@@ -75,10 +76,7 @@ extern "C" pkv_status pkv_paged_attention_decode_static(
     if (dev < 0 || dev >= kMaxDevices) return PKV_ERR_UNSUPPORTED;
     scratch = static_scratch_address(dev, &e);
     if (!scratch) return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
-    // The array keeps whatever the previous call left; the merge counters must
-    // start at zero, so clear them (the partial results are written before read).
-    e = cudaMemsetAsync(scratch, 0, (size_t)kMaxCtas * kMaxConsumerWarps * sizeof(int), static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(static scratch counters)");
+    // Whatever the previous call left there is overwritten before it is read.
   }
   return pkv_paged_attention_decode(out, query, key_cache, value_cache, k_scale, v_scale, block_tables,
                                     max_blocks_per_seq, context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim,

@@ -52,7 +52,7 @@ struct TcParams {
   const int32_t* block_tables;
   const int32_t* context_lens;
   float* lse_out;
-  int* counters;
+  int2* desc;  // per unit: (first CTA | second-slot flag << 30, pieces) for the merge launch
   float* part_o;
   float* part_lse;
   int* err;
@@ -62,6 +62,10 @@ struct TcParams {
   int max_context_len;
   int num_seqs, n_q, n_kv;
   int window, sinks;  // attend to [0, sinks) and [L - window, L) only; window 0 = every position
+  // Quest: per (sequence, KV head) list of k_pages logical pages (ascending, -1
+  // past the count) to read instead of every block; one KV head per unit
+  const int32_t* pages;
+  int k_pages;
   int G, QC, HPC, HG, NCW, stages, units;
   float scale_log2;
   int act_bf16;
@@ -133,6 +137,23 @@ __device__ __forceinline__ uint32_t token_mask(const AttendSet& a, int L, int lb
   return below(L - base) & (below(a.s_eff - base) | (0xFFFFu & ~below(a.lo_w - base)));
 }
 
+// Blocks of unit u (sequence length L): its attended set or, with a page list,
+// the list's entries before its first -1, at most min(k_pages, pages of the
+// sequence).  A full list (the usual case) costs one load.
+__device__ __forceinline__ int unit_blocks(const TcParams& p, int u, int L) {
+  const int nb = attend_set(p, L).nb;
+  if (!p.pages) return nb;
+  const int32_t* list = p.pages + (size_t)u * p.k_pages;  // one KV head per unit: u = s * n_kv + kv
+  const int n = min(p.k_pages, nb);
+  if (n == 0 || __ldg(list + n - 1) >= 0) return n;
+  int lo = 0, hi = n - 1;  // listed pages (>= 0) come first, then -1
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(list + mid) >= 0) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
 // First index i in [0, n) with P[i] > x (n if none).
 __device__ __forceinline__ int upper_bound_smem(const int* P, int n, int x) {
   int lo = 0, hi = n;
@@ -150,10 +171,20 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
   const int units = p.units;
   const int per_t = (units + nthreads - 1) / nthreads;
   const int u0 = min(t * per_t, units), u1 = min(u0 + per_t, units);
+  // counts into P[u]: four units at a time, so their loads are in flight together
   int local = 0;
-  for (int u = u0; u < u1; ++u) {
-    const int s = u / p.HG;
-    local += attend_set(p, seq_len(p, s, (u % p.HG) == 0)).nb;
+  for (int u = u0; u < u1; u += 4) {
+    int L[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) L[k] = u + k < u1 ? seq_len(p, (u + k) / p.HG, ((u + k) % p.HG) == 0) : 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (u + k < u1) {
+        const int n = unit_blocks(p, u + k, L[k]);
+        P[u + k] = n;
+        local += n;
+      }
+    }
   }
   int x = local;
 #pragma unroll
@@ -175,9 +206,10 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
   }
   __syncthreads();
   int run = wsum[warp] + x - local;
-  for (int u = u0; u < u1; ++u) {
+  for (int u = u0; u < u1; ++u) {  // this thread's own counts become offsets
+    const int n = P[u];
     P[u] = run;
-    run += attend_set(p, seq_len(p, u / p.HG, false)).nb;
+    run += n;
   }
   if (u1 == units && u0 < u1) P[units] = run;
   if (units == 0 && t == 0) P[0] = 0;
@@ -199,72 +231,68 @@ __device__ __forceinline__ int d_of(int mt, int hi, int g) {
   else return g * 16 + 2 * mt + hi;
 }
 
-// Merge the pieces of one unit for this warp's query heads (up to 8).  Lane
-// owns dims [lane * D/32, (lane + 1) * D/32) of every head, so all loads of one
-// piece are independent and each piece costs about one L2 round trip.  Pieces
-// are combined in CTA order: M = max lse_k, w_k = 2^(lse_k - M),
-// o = sum w_k o_k / sum w_k, lse = M + log2(sum w_k) (base-2 log-sum-exp).
+// ---------------------------------------------------------------- merge
+// A unit split over several CTAs leaves one normalised partial output and its
+// base-2 log-sum-exp per CTA ("piece").  A second launch, queued behind the
+// decode kernel with programmatic serialisation, combines them: one CTA per
+// unit, a thread per (query head, 4 dims), so every piece's loads of a thread
+// are independent and the whole merge costs about two L2 round trips instead
+// of a serial tail in the decode kernel.  Pieces are combined in CTA order:
+// M = max lse_k, w_k = 2^(lse_k - M), o = sum w_k o_k / sum w_k,
+// lse = M + log2(sum w_k).
+struct MergeParams {
+  void* out;
+  float* lse_out;
+  const float* part_o;
+  const float* part_lse;
+  const int2* desc;
+  int HG, QH, n_q, num_ctas, act_bf16;
+};
+
 template <int D>
-__device__ void merge_pieces(const TcParams& p, int qbase_local, int nh, int c0, int npieces, bool c0_slot1,
-                             long long out_row0, int lane) {
-  const int QH = p.HPC * p.G;
-  constexpr int kPer = D / 32;
-  float M[8], wsum[8], acc[8][kPer];
-#pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    M[n] = -INFINITY;
-    wsum[n] = 0.f;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[n][e] = 0.f;
-  }
-#pragma unroll 1
-  for (int k = 0; k < npieces; ++k) {
-    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-    const float* lse = p.part_lse + ((size_t)(c0 + k) * 2 + slot) * QH + qbase_local;
-#pragma unroll
-    for (int n = 0; n < 8; ++n)
-      if (n < nh) M[n] = fmaxf(M[n], __ldcg(lse + n));
-  }
-#pragma unroll 1
-  for (int k = 0; k < npieces; ++k) {
-    const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-    const size_t piece = ((size_t)(c0 + k) * 2 + slot) * QH + qbase_local;
-    const float* lse = p.part_lse + piece;
-    const float* src = p.part_o + piece * D + lane * kPer;
-#pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      if (n < nh) {
-        const float w = ex2(__ldcg(lse + n) - M[n]);
-        wsum[n] += w;
-        if constexpr (kPer == 4) {
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)n * D));
-          acc[n][0] += w * v.x;
-          acc[n][1] += w * v.y;
-          acc[n][2] += w * v.z;
-          acc[n][3] += w * v.w;
-        } else {
-          const float2 v = __ldcg(reinterpret_cast<const float2*>(src + (size_t)n * D));
-          acc[n][0] += w * v.x;
-          acc[n][1] += w * v.y;
-        }
-      }
+__global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) {
+  grid_launch_dependents();
+  grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
+  const int u = blockIdx.x;
+  const int2 d = p.desc[u];
+  const int c0 = d.x & 0x3FFFFFFF, n = d.y;
+  const bool c0_slot1 = (d.x >> 30) & 1;
+  if (n < 2 || c0 + n > p.num_ctas) return;  // whole unit in one CTA (written there), or no pieces
+  const int s = u / p.HG, hg = u - s * p.HG;
+  constexpr int V = D / 4;
+  for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
+    const int h = idx / V, v = idx - h * V;
+    float M = -INFINITY;
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const int slot = (k == 0 && c0_slot1) ? 1 : 0;
+      M = fmaxf(M, __ldcg(p.part_lse + ((size_t)(c0 + k) * 2 + slot) * p.QH + h));
     }
-  }
-#pragma unroll
-  for (int n = 0; n < 8; ++n) {
-    if (n >= nh) break;
-    const long long row = out_row0 + n;
-    const float inv = 1.f / wsum[n];
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const int slot = (k == 0 && c0_slot1) ? 1 : 0;
+      const size_t piece = ((size_t)(c0 + k) * 2 + slot) * p.QH + h;
+      const float w = ex2(__ldcg(p.part_lse + piece) - M);
+      const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + piece * D) + v);
+      wsum += w;
+      acc.x += w * o.x;
+      acc.y += w * o.y;
+      acc.z += w * o.z;
+      acc.w += w * o.w;
+    }
+    const float inv = 1.f / wsum;
+    const long long row = (long long)s * p.n_q + hg * p.QH + h;
     if (p.act_bf16) {
-      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(p.out) + row * D + lane * kPer;
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) o[e] = __float2bfloat16_rn(acc[n][e] * inv);
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + row * D + 4 * v);
+      o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     } else {
-      float* o = reinterpret_cast<float*>(p.out) + row * D + lane * kPer;
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) o[e] = acc[n][e] * inv;
+      reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * D)[v] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
-    if (p.lse_out && lane == 0) p.lse_out[row] = (M[n] + log2f(wsum[n])) * kLn2;
+    if (p.lse_out && v == 0) p.lse_out[row] = (M + log2f(wsum)) * kLn2;
   }
 }
 
@@ -322,8 +350,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const int s = u / p.HG;
         hg = u - s * p.HG;
         unit_last = (i + 1 == P[u + 1]);
-        const int lb = logical_block(attend_set(p, seq_len(p, s, false)), i - P[u]);
-        phys = __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + lb);
+        const int Ls = seq_len(p, s, false);
+        int lb;
+        if (p.pages) {
+          lb = __ldg(p.pages + ((size_t)s * p.n_kv + hg) * p.k_pages + (i - P[u]));
+          if (lb < 0 || (long long)lb * kBlockSize >= Ls) lb = -1;  // not a page of this sequence
+        } else {
+          lb = logical_block(attend_set(p, Ls), i - P[u]);
+        }
+        phys = lb < 0 ? -1 : __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + lb);
         if (phys < 0 || (long long)phys >= p.num_blocks) {
           flag_error(p.err, DEVERR_BLOCK_RANGE);
           phys = -1;
@@ -386,10 +421,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const int qbase_local = head_local * p.G + qc * 8;  // q head index inside the unit
   const bool head0_ok = qc * 8 + 2 * c < p.G, head1_ok = qc * 8 + 2 * c + 1 < p.G;
 
-  // CTA 0 writes the sequences with no tokens: out = 0, lse = -inf.
-  if (blockIdx.x == 0) {
-    for (int u = 0; u < units; ++u) {
-      if (P[u] != P[u + 1]) continue;
+  // Units with no blocks (empty sequences, empty page lists): out = 0,
+  // lse = -inf.  CTAs share the scan, 32 units per warp step.
+  for (int u0 = blockIdx.x * 32; u0 < units; u0 += gridDim.x * 32) {
+    const int uu = u0 + lane;
+    unsigned empty_units = __ballot_sync(0xffffffffu, uu < units && P[uu] == P[uu + 1]);
+    while (empty_units) {
+      const int u = u0 + __ffs(empty_units) - 1;
+      empty_units &= empty_units - 1;
+      if (warp == 0 && lane == 0) p.desc[u] = make_int2(0, 0);
       const int s = u / p.HG, hg = u - s * p.HG;
       for (int n = 0; n < 8; ++n) {
         if (qc * 8 + n >= p.G) break;
@@ -465,6 +505,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   int j = a - P[u];
   int s = 0, hg = 0, L = 0;
   AttendSet aset{};
+  int last_page = 0;
   float head_k_scale = 1.f, head_v_scale = 1.f;
 
   uint32_t qf[KS][2];
@@ -654,7 +695,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       stage[k] = (it + k) % p.stages;
       if (!mbar_wait(&full[stage[k]], ((it + k) / p.stages) & 1)) return false;
       st[k] = smem + (size_t)stage[k] * p.stage_bytes;
-      valid[k] = token_mask(aset, L, logical_block(aset, j + k));
+      if (p.pages)
+        valid[k] = (j + k + 1 == P[u + 1] - P[u]) ? token_mask(aset, L, last_page) : 0xFFFFu;
+      else
+        valid[k] = token_mask(aset, L, logical_block(aset, j + k));
     }
     float sv[NB][4], vsc[NB][2];
 #pragma unroll
@@ -713,10 +757,17 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   while (i < b) {
     if (i == a || j == 0) {
       // ---- unit start: this warp's 8 query rows as MMA B fragments
+      if (j == 0 && warp == 0 && lane == 0) {
+        // this CTA holds the unit's first block: record its pieces for the merge
+        const int c1 = (P[u + 1] - 1) / per;
+        p.desc[u] = make_int2((int)blockIdx.x | ((P[u] % per) != 0 ? (1 << 30) : 0), c1 - (int)blockIdx.x + 1);
+      }
       s = u / p.HG;
       hg = u - s * p.HG;
       L = seq_len(p, s, false);
       aset = attend_set(p, L);
+      if (p.pages)  // only the list's last entry can be the sequence's partial last page
+        last_page = __ldg(p.pages + ((size_t)s * p.n_kv + hg) * p.k_pages + (P[u + 1] - P[u] - 1));
       if constexpr (CACHE == TC_BF16) {
         fetch_query(u);
 #pragma unroll
@@ -822,25 +873,6 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           if (head0_ok) __stcg(p.part_lse + pbase, lse0);
           if (head1_ok) __stcg(p.part_lse + pbase + 1, lse1);
         }
-        __threadfence();
-        __syncwarp();
-        const int c0 = P[u] / per, c1 = (P[u + 1] - 1) / per;
-        const int npieces = c1 - c0 + 1;
-        int last = 0;
-        if (lane == 0) {
-          // A split unit's last CTA (c1) is unique to it: the unit holds c1's first block.
-          int* ctr = p.counters + (size_t)c1 * kMaxConsumerWarps + warp;
-          const int old = atomicAdd(ctr, 1);
-          last = (old == npieces - 1);
-          if (last) *ctr = 0;  // leave the counter zeroed for the next call
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          const bool c0_slot1 = (P[u] % per) != 0;
-          const int nh = min(8, p.G - qc * 8);
-          merge_pieces<D>(p, qbase_local, nh, c0, npieces, c0_slot1, (long long)s * p.n_q + hg * QH + qbase_local, lane);
-        }
       }
     }
     if (unit_end) {
@@ -905,6 +937,33 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, prm);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_tc_kernel launch");
+
+  // The merge of split units, allowed to become resident while the decode
+  // kernel runs; it waits for the decode kernel's completion on the device.
+  MergeParams mp;
+  mp.out = prm.out;
+  mp.lse_out = prm.lse_out;
+  mp.part_o = prm.part_o;
+  mp.part_lse = prm.part_lse;
+  mp.desc = prm.desc;
+  mp.HG = plan.HG;
+  mp.QH = plan.HPC * plan.G;
+  mp.n_q = prm.n_q;
+  mp.num_ctas = plan.num_ctas;
+  mp.act_bf16 = prm.act_bf16;
+  cudaLaunchConfig_t mcfg = {};
+  mcfg.gridDim = dim3(plan.units);
+  mcfg.blockDim = dim3((unsigned)std::min(256, (mp.QH * (D / 4) + 31) / 32 * 32));
+  mcfg.dynamicSmemBytes = 0;
+  mcfg.stream = stream;
+  cudaLaunchAttribute mattr[1];
+  mattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  mattr[0].val.programmaticStreamSerializationAllowed = 1;
+  mcfg.attrs = mattr;
+  mcfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&mcfg, decode_merge_kernel<D>, mp);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode_merge_kernel launch");
   return PKV_OK;
 }
 
@@ -939,7 +998,7 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.context_lens = a.context_lens;
   prm.lse_out = a.lse_out;
   uint8_t* ws = static_cast<uint8_t*>(a.workspace);
-  prm.counters = reinterpret_cast<int*>(ws + plan.ws_counters);
+  prm.desc = reinterpret_cast<int2*>(ws + plan.ws_desc);
   prm.part_o = reinterpret_cast<float*>(ws + plan.ws_part_o);
   prm.part_lse = reinterpret_cast<float*>(ws + plan.ws_part_lse);
   prm.err = a.device_error;
@@ -952,6 +1011,8 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.n_kv = s.n_kv;
   prm.window = a.window;
   prm.sinks = a.sinks;
+  prm.pages = a.pages;
+  prm.k_pages = a.k_pages;
   prm.G = plan.G;
   prm.QC = plan.QC;
   prm.HPC = plan.HPC;
@@ -1040,12 +1101,12 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.num_ctas = want_ctas > 0 ? want_ctas : sms * per_sm;
   if (pl.num_ctas > kMaxCtas) return want_ctas > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   const size_t QH = (size_t)pl.HPC * pl.G;
-  // Counters sit in a fixed region whatever the shape, so one zero-filled
-  // workspace can serve calls of different shapes.
-  pl.ws_counters = 0;
-  pl.ws_part_o = (size_t)kMaxCtas * kMaxConsumerWarps * 4;
+  // Pieces (two slots per CTA), their lse, one merge descriptor per unit.
+  // Every byte read is written earlier in the same call: no zeroing needed.
+  pl.ws_part_o = 0;
   pl.ws_part_lse = align_up(pl.ws_part_o + (size_t)pl.num_ctas * 2 * QH * s.head_dim * 4, 256);
-  pl.ws_total = align_up(pl.ws_part_lse + (size_t)pl.num_ctas * 2 * QH * 4, 256);
+  pl.ws_desc = align_up(pl.ws_part_lse + (size_t)pl.num_ctas * 2 * QH * 4, 256);
+  pl.ws_total = align_up(pl.ws_desc + (size_t)pl.units * 8, 256);
   *plan = pl;
   return PKV_OK;
 }

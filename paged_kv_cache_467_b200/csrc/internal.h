@@ -36,7 +36,7 @@ struct TcPlan {
   int units;        // num_seqs * HG
   uint32_t stage_bytes, tx_bytes;
   size_t smem_bytes;
-  size_t ws_counters, ws_part_o, ws_part_lse, ws_total;  // byte offsets / total
+  size_t ws_part_o, ws_part_lse, ws_desc, ws_total;  // byte offsets / total
 };
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
@@ -64,6 +64,9 @@ struct TcArgs {
   // sliding window with sinks: attend to [0, sinks) and [L - window, L); 0 = all
   int window = 0;
   int sinks = 0;
+  // Quest decode only: [num_seqs, n_kv, k_pages] logical pages to read
+  const int32_t* pages = nullptr;
+  int k_pages = 0;
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);
@@ -78,6 +81,16 @@ pkv_status launch_cache_write(const void* key, const void* value, void* key_cach
 pkv_status launch_move_blocks(const void* const src[4], void* const dst[4], const size_t bytes_per_block[4], int npools,
                               const int64_t* pairs, int64_t num_pairs, int64_t src_blocks, int64_t dst_blocks,
                               int32_t* device_error, cudaStream_t stream);
+
+pkv_status launch_quest_summaries(const void* key_cache, void* page_min, void* page_max, const int32_t* block_tables,
+                                  int max_blocks_per_seq, const int32_t* context_lens, int num_seqs, int n_kv,
+                                  int head_dim, int64_t num_blocks, pkv_dtype cache, int last_page_only,
+                                  int32_t* device_error, cudaStream_t stream);
+pkv_status launch_quest_select(const void* query, const void* page_min, const void* page_max,
+                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                               int max_context_len, int num_seqs, int n_q, int n_kv, int head_dim, int64_t num_blocks,
+                               pkv_dtype act, pkv_dtype cache, int k_pages, int32_t* selected, float* scores,
+                               int32_t* device_error, cudaStream_t stream);
 
 // Records the CUDA error text for pkv_last_cuda_error() and returns PKV_ERR_CUDA.
 pkv_status cuda_fail(cudaError_t e, const char* where);

@@ -75,6 +75,16 @@ def _load() -> ctypes.CDLL:
     lib.pkv_copy_blocks.restype = i32
     lib.pkv_swap_blocks.argtypes = [vp, vp, vp, vp, i64, vp, vp, vp, vp, i64, vp, i64, i32, i32, i32, i32, vp, vp]
     lib.pkv_swap_blocks.restype = i32
+    lib.pkv_quest_page_summaries.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i64, i32, i32, vp, vp]
+    lib.pkv_quest_page_summaries.restype = i32
+    lib.pkv_quest_select.argtypes = [vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32, i64, i32, i32, i32, vp, vp,
+                                     vp, vp]
+    lib.pkv_quest_select.restype = i32
+    lib.pkv_paged_attention_decode_pages.argtypes = decode_args[:17] + [vp, i32] + decode_args[17:] + [vp]
+    lib.pkv_paged_attention_decode_pages.restype = i32
+    lib.pkv_paged_attention_decode_pages_ex.argtypes = (lib.pkv_paged_attention_decode_pages.argtypes[:-1]
+                                                        + [ctypes.POINTER(DecodeTuning), vp])
+    lib.pkv_paged_attention_decode_pages_ex.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_cuda_error.argtypes = []
@@ -289,4 +299,59 @@ def paged_attention_decode_window(out, query, key_cache, value_cache, block_tabl
         _ptr(device_error), _stream(query.device),
     )
     _check(st, "pkv_paged_attention_decode_window")
+    return out
+
+
+def quest_page_summaries(key_cache, page_min, page_max, block_tables, context_lens, device_error=None,
+                         last_page_only: bool = False):
+    """Element-wise min / max of each page's keys into ``page_min`` / ``page_max`` [num_blocks, n_kv, d]."""
+    nb, bs, n_kv, d = key_cache.shape
+    st = lib.pkv_quest_page_summaries(_ptr(key_cache), _ptr(page_min), _ptr(page_max), _ptr(block_tables),
+                                      block_tables.shape[1], _ptr(context_lens), block_tables.shape[0], n_kv, d, bs,
+                                      nb, cache_code(key_cache), int(bool(last_page_only)), _ptr(device_error),
+                                      _stream(key_cache.device))
+    _check(st, "pkv_quest_page_summaries")
+
+
+def quest_select(query, page_min, page_max, block_tables, context_lens, max_context_len: int, k_pages: int,
+                 selected, scores=None, device_error=None):
+    """Each (sequence, KV head)'s ``k_pages`` best pages into ``selected`` [S, n_kv, k_pages] (ascending, -1 after)."""
+    S, n_q, d = query.shape
+    nb, n_kv = page_min.shape[0], page_min.shape[1]
+    if scores is None:
+        cap = min(int(max_context_len), block_tables.shape[1] * 16)
+        scores = torch.empty((S, n_kv, max(1, -(-cap // 16))), dtype=torch.float32, device=query.device)
+    st = lib.pkv_quest_select(_ptr(query), _ptr(page_min), _ptr(page_max), _ptr(block_tables), block_tables.shape[1],
+                              _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, 16, nb, act_code(query),
+                              cache_code(page_min), int(k_pages), _ptr(selected), _ptr(scores), _ptr(device_error),
+                              _stream(query.device))
+    _check(st, "pkv_quest_select")
+    return selected
+
+
+def paged_attention_decode_pages(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
+                                 pages, sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None,
+                                 workspace=None, device_error=None, tuning: DecodeTuning | None = None):
+    """Decode attention over the logical pages listed in ``pages`` [S, n_kv, k] for each KV head."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ccode = cache_code(key_cache)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        t1 = None if tuning is None else DecodeTuning(tuning.num_ctas, tuning.stages, 1, tuning.flags)
+        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, t1)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    args = [
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
+        float(sm_scale), _ptr(pages), pages.shape[-1], act_code(query), ccode, _ptr(lse_out), _ptr(workspace),
+        ws_bytes, _ptr(device_error),
+    ]
+    if tuning is None:
+        st = lib.pkv_paged_attention_decode_pages(*args, _stream(query.device))
+    else:
+        st = lib.pkv_paged_attention_decode_pages_ex(*args, ctypes.byref(tuning), _stream(query.device))
+    _check(st, "pkv_paged_attention_decode_pages")
     return out
