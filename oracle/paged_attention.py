@@ -9,7 +9,9 @@ arrays and then applies the textbook attention definition.
 Cache layout (reading of the Physical KV Block figure in Chapter 18): separate
 key and value pools, each ``[num_blocks, block_size, n_kv, d]``.
 Dtype names: "f32", "bf16" (values held as float), "int8" (codes with a float32
-scale per (block, row, head)), "fp8_e4m3" (bytes with a float32 scale per head).
+scale per (block, row, head)), "int4" (two codes per byte, pools
+``[num_blocks, block_size, n_kv, d/2]``, a float32 scale per (block, row,
+head)), "fp8_e4m3" and "fp8_e5m2" (bytes with a float32 scale per head).
 """
 from __future__ import annotations
 
@@ -17,7 +19,10 @@ import math
 
 import numpy as np
 
-from .quant import absmax_quantize, e4m3_decode, e4m3_encode
+from .quant import absmax_quantize, e4m3_decode, e4m3_encode, e5m2_decode, e5m2_encode, pack_int4, unpack_int4
+
+FP8_CODECS = {"fp8_e4m3": (e4m3_encode, e4m3_decode), "fp8_e5m2": (e5m2_encode, e5m2_decode)}
+ROW_SCALED = ("int8", "int4")
 
 
 def kv_head_of(h: int, n_q: int, n_kv: int) -> int:
@@ -57,23 +62,26 @@ def gather_sequence(cache, block_row, length: int, block_size: int):
 def dequantize_rows(rows, cache_dtype: str, row_scales=None, head_scales=None):
     """Stored rows -> float64 values.
 
-    int8: code * scale of that (token, head) ("KV Cache Engineering", section 8:
-    multiplying the codes by the scale restores the values).  fp8_e4m3: E4M3
+    int8 / int4: code * scale of that (token, head) ("KV Cache Engineering",
+    section 8: multiplying the codes by the scale restores the values); int4
+    codes are unpacked from their nibbles first.  fp8_e4m3 / fp8_e5m2: FP8
     value * per-head scale.  f32 / bf16: the stored values.
     """
     if cache_dtype == "int8":
         return rows.astype(np.float64) * np.asarray(row_scales, dtype=np.float64)[..., None]
-    if cache_dtype == "fp8_e4m3":
-        return e4m3_decode(rows) * np.asarray(head_scales, dtype=np.float64)[None, :, None]
+    if cache_dtype == "int4":
+        return unpack_int4(rows).astype(np.float64) * np.asarray(row_scales, dtype=np.float64)[..., None]
+    if cache_dtype in FP8_CODECS:
+        return FP8_CODECS[cache_dtype][1](rows) * np.asarray(head_scales, dtype=np.float64)[None, :, None]
     return rows.astype(np.float64)
 
 
 def gather_dequantized(cache, scales, block_row, length, block_size, cache_dtype):
     rows = gather_sequence(cache, block_row, length, block_size)
-    if cache_dtype == "int8":
+    if cache_dtype in ROW_SCALED:
         row_scales = gather_sequence(scales, block_row, length, block_size)
         return dequantize_rows(rows, cache_dtype, row_scales=row_scales)
-    if cache_dtype == "fp8_e4m3":
+    if cache_dtype in FP8_CODECS:
         return dequantize_rows(rows, cache_dtype, head_scales=scales)
     return dequantize_rows(rows, cache_dtype)
 
@@ -181,8 +189,19 @@ def quantize_row_int8(x):
     return codes.astype(np.int8), np.float32(scale)
 
 
-def quantize_rows_fp8(x, head_scales):
-    """[..., n_kv, d] rows -> E4M3 bytes of x / scale_h (division in float32).
+def quantize_row_int4(x):
+    """One (token, head) row -> (packed int4 bytes, float32 scale).
+
+    The section-8 absmax quantiser of "KV Cache Engineering" at 4 bits (codes
+    -7..7, the page's own example), one scale per (token, head), arithmetic in
+    IEEE float32, codes packed two per byte.
+    """
+    codes, scale, _ = absmax_quantize(np.asarray(x, dtype=np.float32), 4, np.float32)
+    return pack_int4(codes), np.float32(scale)
+
+
+def quantize_rows_fp8(x, head_scales, cache_dtype: str = "fp8_e4m3"):
+    """[..., n_kv, d] rows -> FP8 bytes of x / scale_h (division in float32).
 
     Reading for scale_h == 0: codes 0 (no division).
     """
@@ -190,7 +209,7 @@ def quantize_rows_fp8(x, head_scales):
     sc = np.asarray(head_scales, dtype=np.float32)[:, None]
     safe = np.where(sc == 0, np.float32(1), sc).astype(np.float32)
     y = (x / safe).astype(np.float32)
-    codes = e4m3_encode(y)
+    codes = FP8_CODECS[cache_dtype][0](y)
     return np.where(sc == 0, np.uint8(0), codes).astype(np.uint8)
 
 
@@ -199,9 +218,9 @@ def kv_cache_write(key, value, key_cache, value_cache, slot_mapping, cache_dtype
 
     Chapter 18, How PagedAttention Works: new tokens fill the current block.
     Slot sigma addresses row sigma % block_size of block sigma // block_size;
-    slot -1 means "no write".  int8 also writes the per-(token, head) scales
-    into ``k_scale``/``v_scale`` [num_blocks, block_size, n_kv]; fp8_e4m3 reads
-    per-head scales from them.
+    slot -1 means "no write".  int8 / int4 also write the per-(token, head)
+    scales into ``k_scale``/``v_scale`` [num_blocks, block_size, n_kv]; the FP8
+    formats read per-head scales from them.
     """
     block_size = key_cache.shape[1]
     key = np.asarray(key)
@@ -210,13 +229,14 @@ def kv_cache_write(key, value, key_cache, value_cache, slot_mapping, cache_dtype
         if slot < 0:
             continue
         b, r = int(slot) // block_size, int(slot) % block_size
-        if cache_dtype == "int8":
+        if cache_dtype in ROW_SCALED:
+            quantize = quantize_row_int8 if cache_dtype == "int8" else quantize_row_int4
             for h in range(key.shape[1]):
-                key_cache[b, r, h], k_scale[b, r, h] = quantize_row_int8(key[t, h])
-                value_cache[b, r, h], v_scale[b, r, h] = quantize_row_int8(value[t, h])
-        elif cache_dtype == "fp8_e4m3":
-            key_cache[b, r] = quantize_rows_fp8(key[t], k_scale)
-            value_cache[b, r] = quantize_rows_fp8(value[t], v_scale)
+                key_cache[b, r, h], k_scale[b, r, h] = quantize(key[t, h])
+                value_cache[b, r, h], v_scale[b, r, h] = quantize(value[t, h])
+        elif cache_dtype in FP8_CODECS:
+            key_cache[b, r] = quantize_rows_fp8(key[t], k_scale, cache_dtype)
+            value_cache[b, r] = quantize_rows_fp8(value[t], v_scale, cache_dtype)
         else:
             key_cache[b, r] = key[t]
             value_cache[b, r] = value[t]

@@ -86,3 +86,80 @@ def e4m3_encode(y) -> np.ndarray:
     mag = np.where(a >= E4M3_MAX, 0x7E, mag)
     code = mag.astype(np.uint8) | np.where(np.signbit(y), 0x80, 0).astype(np.uint8)
     return np.where(np.isnan(y), np.uint8(0x7F), code).astype(np.uint8)
+
+
+# --------------------------------------------------------------- FP8 E5M2
+def _e5m2_value(byte: int) -> float:
+    """Value of one E5M2 byte from the OCP 8-bit floating point definition.
+
+    Layout S.EEEEE.MM, exponent bias 15, IEEE-like: exponent field 31 with
+    mantissa 0 is infinity, with mantissa != 0 NaN; exponent field 0 encodes
+    subnormals 2**-14 * M/4.
+    """
+    s = -1.0 if byte & 0x80 else 1.0
+    e = (byte >> 2) & 0x1F
+    m = byte & 0x3
+    if e == 0x1F:
+        return s * float("inf") if m == 0 else float("nan")
+    if e == 0:
+        return s * (2.0 ** -14) * (m / 4.0)
+    return s * (2.0 ** (e - 15)) * (1.0 + m / 4.0)
+
+
+def e5m2_value_table() -> np.ndarray:
+    """float64 [256]: value of every E5M2 byte."""
+    return np.array([_e5m2_value(b) for b in range(256)], dtype=np.float64)
+
+
+_TABLE52 = e5m2_value_table()
+_POS52 = _TABLE52[:0x7C]  # magnitudes of the finite codes 0x00..0x7B, increasing
+E5M2_MAX = float(_POS52[-1])  # 57344
+
+
+def e5m2_decode(codes) -> np.ndarray:
+    return _TABLE52[np.asarray(codes, dtype=np.uint8)]
+
+
+def e5m2_encode(y) -> np.ndarray:
+    """Round float values to E5M2: nearest finite value, ties to the even code.
+
+    As for E4M3, a scaled cache saturates: magnitudes above 57344 (infinities
+    included) become +-57344; the sign bit follows the input; NaN encodes as
+    0x7F.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    idx = np.searchsorted(_POS52, np.minimum(a, E5M2_MAX))
+    idx = np.clip(idx, 0, len(_POS52) - 1)
+    lo = np.clip(idx - 1, 0, len(_POS52) - 1)
+    d_lo = np.abs(a - _POS52[lo])
+    d_hi = np.abs(_POS52[idx] - a)
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (idx % 2 == 0))
+    mag = np.where(pick_hi, idx, lo)
+    mag = np.where(a >= E5M2_MAX, 0x7B, mag)
+    code = mag.astype(np.uint8) | np.where(np.signbit(y), 0x80, 0).astype(np.uint8)
+    return np.where(np.isnan(y), np.uint8(0x7F), code).astype(np.uint8)
+
+
+# --------------------------------------------------------------- INT4
+def pack_int4(codes) -> np.ndarray:
+    """Signed 4-bit codes [..., d] (d even, values in [-8, 7]) -> bytes [..., d/2].
+
+    Storage reading for the 4-bit cache ("KV Cache Engineering", section 8:
+    a 4-bit format cuts the payload to a quarter of BF16): two's-complement
+    nibbles, the code of element 2j in the low nibble of byte j and that of
+    element 2j+1 in the high nibble.
+    """
+    c = np.asarray(codes, dtype=np.int64)
+    nib = (c & 0xF).astype(np.uint8)
+    return (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed) -> np.ndarray:
+    """Bytes [..., d/2] -> signed codes [..., d] (inverse of pack_int4)."""
+    b = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    lo, hi = b & 0xF, b >> 4
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int64)
+    out[..., 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[..., 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out

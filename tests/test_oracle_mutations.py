@@ -152,3 +152,26 @@ def test_quest_selecting_lowest_scores_is_caught(monkeypatch):
 
     monkeypatch.setattr(oq, "select_pages", lambda s, k: np.sort(np.argsort(np.asarray(s))[: min(k, len(s))]))
     _fails(lambda: qpins.test_quest_worked_example(read_golden))
+
+
+def test_swapped_int4_nibbles_are_caught(monkeypatch):
+    import test_oracle_formats as fpins
+
+    def swapped(codes):
+        c = np.asarray(codes, dtype=np.int64)
+        nib = (c & 0xF).astype(np.uint8)
+        return (nib[..., 1::2] | (nib[..., 0::2] << 4)).astype(np.uint8)
+
+    monkeypatch.setattr(oq, "pack_int4", swapped)
+    monkeypatch.setattr(pa, "pack_int4", swapped)
+    _fails(fpins.test_int4_nibble_order)
+    _fails(fpins.test_int4_cache_decode_is_attention_over_restored_values)
+
+
+def test_e5m2_wrong_bias_is_caught(monkeypatch):
+    import test_oracle_formats as fpins
+
+    t = oq.e5m2_value_table() * 2.0  # bias 14 instead of 15
+    monkeypatch.setattr(oq, "e5m2_value_table", lambda: t)
+    _fails(fpins.test_e5m2_table_closed_forms)
+    _fails(fpins.test_e5m2_table_matches_torch_float8)
