@@ -143,18 +143,25 @@ def oracle_step_sample(w, seqs, host_rows):
 
     import oracle
 
+    from paged_kv_cache_467_b200 import accounting
+
+    per_token = accounting.cache_bytes(1, w.n_kv, w.head_dim, 1, accounting.BYTES_PER_VALUE[w.cache_dtype])
+    per_token += accounting.scale_bytes_per_token(w.cache_dtype, w.n_kv)
     kv_bytes = 0
     for s in seqs:
-        kc, vc, K, V, q = host_rows[s]
+        kc, vc, ks, vs, K, V, q = host_rows[s]
         L = int(w.context_lens[s])
-        oracle.kv_cache_write(K[L - 1 : L], V[L - 1 : L], kc, vc, np.array([L - 1], dtype=np.int64))
+        oracle.kv_cache_write(K[L - 1 : L], V[L - 1 : L], kc, vc, np.array([L - 1], dtype=np.int64), w.cache_dtype,
+                              ks, vs)
         nb = kc.shape[0]
-        oracle.paged_attention_decode(q, kc, vc, np.arange(nb, dtype=np.int32)[None], np.array([L]), w.sm_scale)
-        kv_bytes += L * w.n_kv * w.head_dim * 2 * 2
+        oracle.paged_attention_decode(q, kc, vc, np.arange(nb, dtype=np.int32)[None], np.array([L]), w.sm_scale,
+                                      w.cache_dtype, ks, vs, window=w.window, sinks=w.sinks)
+        att = min(L, w.window + w.sinks) if w.window else L
+        kv_bytes += int(att * per_token)
     return kv_bytes
 
 
-def prepare_oracle_rows(w, seqs):
+def prepare_oracle_rows(w, seqs, scales=None):
     import numpy as np
 
     import oracle
@@ -165,10 +172,19 @@ def prepare_oracle_rows(w, seqs):
         L = int(w.context_lens[s])
         nb = -(-L // w.block_size)
         K, V = w.sequence_kv(s)
-        kc = np.zeros((nb, w.block_size, w.n_kv, w.head_dim))
+        width = w.head_dim // 2 if w.cache_dtype == "int4" else w.head_dim
+        kc = np.zeros((nb, w.block_size, w.n_kv, width),
+                      {"int8": np.int8, "int4": np.uint8}.get(w.cache_dtype, np.uint8 if "fp8" in w.cache_dtype
+                                                              else np.float64))
         vc = np.zeros_like(kc)
-        oracle.kv_cache_write(K[: L - 1], V[: L - 1], kc, vc, np.arange(L - 1, dtype=np.int64))
-        rows[s] = (kc, vc, K, V, q[s : s + 1])
+        ks = vs = None
+        if w.cache_dtype in ("int8", "int4"):
+            ks = np.zeros((nb, w.block_size, w.n_kv), np.float32)
+            vs = np.zeros_like(ks)
+        elif w.cache_dtype.startswith("fp8"):
+            ks, vs = scales
+        oracle.kv_cache_write(K[: L - 1], V[: L - 1], kc, vc, np.arange(L - 1, dtype=np.int64), w.cache_dtype, ks, vs)
+        rows[s] = (kc, vc, ks, vs, K, V, q[s : s + 1])
     return rows
 
 
@@ -187,10 +203,11 @@ def time_oracle(w, budget_s: float, max_seqs: int | None = None):
     order = list(range(w.num_seqs))
     seqs, t_total, b_total = [], 0.0, 0
     host = {}
+    scales = w.fp8_head_scales() if w.cache_dtype.startswith("fp8") else None
     for s in order:
         if max_seqs is not None and len(seqs) >= max_seqs:
             break
-        host.update(prepare_oracle_rows(w, [s]))
+        host.update(prepare_oracle_rows(w, [s], scales))
         t0 = time.perf_counter()
         b = oracle_step_sample(w, [s], host)
         t_total += time.perf_counter() - t0
@@ -305,6 +322,7 @@ def run_b200(args, rank, world, local):
 
     w = replica_workload(workloads.CONFIGS[args.config](), rank)
     S, nq, nkv, d, bs = w.num_seqs, w.n_q, w.n_kv, w.head_dim, w.block_size
+    named = "int4" if w.cache_dtype == "int4" else None  # an int4 pool's torch dtype (uint8) does not name it
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
     shape = (w.num_blocks, bs, nkv, d)
     # q/K/V ~ N(0,1) synthetic cache, filled on the device (the writer is exercised by the step's append)
@@ -313,20 +331,24 @@ def run_b200(args, rank, world, local):
         vc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
         ks = vs = None
     else:
-        kc = torch.empty(shape, device=dev, dtype=torch.int8 if w.cache_dtype == "int8" else torch.uint8)
+        pool_dtype = {"int8": torch.int8, "fp8_e4m3": torch.uint8, "fp8_e5m2": torch.float8_e5m2,
+                      "int4": torch.uint8}[w.cache_dtype]
+        pool_shape = shape[:3] + (d // 2,) if w.cache_dtype == "int4" else shape
+        kc = torch.empty(pool_shape, device=dev, dtype=pool_dtype)
         vc = torch.empty_like(kc)
-        if w.cache_dtype == "int8":
+        if w.cache_dtype in ("int8", "int4"):
             ks = torch.empty(shape[:3], device=dev)
             vs = torch.empty(shape[:3], device=dev)
         else:
-            ks = torch.full((nkv,), 5.0 / 448, device=dev)
-            vs = torch.full((nkv,), 5.0 / 448, device=dev)
+            top = 448.0 if w.cache_dtype == "fp8_e4m3" else 57344.0
+            ks = torch.full((nkv,), 5.0 / top, device=dev)
+            vs = torch.full((nkv,), 5.0 / top, device=dev)
         slots_all = torch.arange(w.num_blocks * bs, device=dev, dtype=torch.int64)
         for c0 in range(0, slots_all.numel(), 1 << 20):
             sl = slots_all[c0 : c0 + (1 << 20)]
             kk = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
             vv = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
-            ops.kv_cache_write(kk, vv, kc, vc, sl, ks, vs)
+            ops.kv_cache_write(kk, vv, kc, vc, sl, ks, vs, cache_dtype=named)
     q = torch.randn((S, nq, d), device=dev, generator=gen).to(torch.bfloat16)
     k_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
     v_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
@@ -339,7 +361,7 @@ def run_b200(args, rank, world, local):
     # the kernel launched right before a step, so each step may overlap its
     # prologue with the previous step's tail (programmatic dependent launch).
     tuning = None if args.no_overlap else ops.DecodeTuning(0, 0, 0, ops.TUNE_OVERLAP_PROLOGUE)
-    nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc))
+    nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc, named))
     ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
@@ -350,18 +372,18 @@ def run_b200(args, rank, world, local):
     def decode(out, q, bt, cl):
         if w.window:
             ops.paged_attention_decode_window(out, q, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
-                                              w.sm_scale, ks, vs, workspace=ws, device_error=err)
+                                              w.sm_scale, ks, vs, workspace=ws, device_error=err, cache_dtype=named)
         else:
             ops.paged_attention_decode(out, q, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs, workspace=ws,
-                                       device_error=err)
+                                       device_error=err, cache_dtype=named)
 
     def step(q=q, k_new=k_new, v_new=v_new, bt=bt, cl=cl, slots=slots, overlap=True):
         if args.unfused:
-            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err, cache_dtype=named)
             decode(out, q, bt, cl)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err, tuning=tuning if overlap else None)
+                                  workspace=ws, device_error=err, tuning=tuning if overlap else None, cache_dtype=named)
 
     def barrier():
         if world > 1:
@@ -391,13 +413,13 @@ def run_b200(args, rank, world, local):
     ev_start.record(stream)
     for k in range(args.steps):
         if args.unfused:
-            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err)
+            ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err, cache_dtype=named)
             att[k][0].record(stream)
             decode(out, q, bt, cl)
             att[k][1].record(stream)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err, tuning=tuning)
+                                  workspace=ws, device_error=err, tuning=tuning, cache_dtype=named)
     ev_end.record(stream)
     torch.cuda.synchronize()
     barrier()

@@ -11,12 +11,13 @@
  * Layouts (row-major, innermost last):
  *   key / value (new rows)   [num_tokens, n_kv, head_dim]          act dtype
  *   key_cache / value_cache  [num_blocks, block_size, n_kv, head_dim] cache dtype
+ *                            (INT4: [..., head_dim / 2] bytes)
  *   query / out              [num_seqs, n_q, head_dim]             act dtype
  *   block_tables             int32 [num_seqs, max_blocks_per_seq]
  *   context_lens             int32 [num_seqs]
  *   slot_mapping             int64 [num_tokens]
- *   k_scale / v_scale        INT8:     float [num_blocks, block_size, n_kv]
- *                            FP8 E4M3: float [n_kv]
+ *   k_scale / v_scale        INT8, INT4:     float [num_blocks, block_size, n_kv]
+ *                            FP8 E4M3, E5M2: float [n_kv]
  * A physical block holds the K (or V) rows of block_size consecutive tokens
  * for all KV heads: "Chapter 18 - KV-Cache Optimization Strategies", How
  * PagedAttention Works (Physical KV Block figure: [block_size, G, d_k]).
@@ -35,7 +36,11 @@ typedef enum {
   PKV_F32 = 0,      /* IEEE float32 */
   PKV_BF16 = 1,     /* bfloat16 */
   PKV_INT8 = 2,     /* int8 codes, one float scale per (token, head); cache only */
-  PKV_FP8_E4M3 = 3  /* OCP E4M3 bytes, one float scale per KV head; cache only */
+  PKV_FP8_E4M3 = 3, /* OCP E4M3 bytes, one float scale per KV head; cache only */
+  PKV_FP8_E5M2 = 4, /* OCP E5M2 bytes, one float scale per KV head; cache only */
+  PKV_INT4 = 5      /* signed 4-bit codes, two per byte (element 2j in the low
+                       nibble of byte j), one float scale per (token, KV head);
+                       cache only, pools [num_blocks, block_size, n_kv, head_dim/2] */
 } pkv_dtype;
 
 typedef enum {
@@ -65,8 +70,8 @@ typedef enum {
  *
  *   key, value          device, [num_tokens, n_kv, head_dim], act_dtype (F32 or BF16)
  *   key_cache, value_cache device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
- *   k_scale, v_scale    INT8: device, written, one scale per (slot, head);
- *                       FP8_E4M3: device, read, one scale per KV head;
+ *   k_scale, v_scale    INT8 / INT4: device, written, one scale per (slot, head);
+ *                       FP8_E4M3 / FP8_E5M2: device, read, one scale per KV head;
  *                       F32/BF16: must be NULL
  *   slot_mapping        device int64 [num_tokens]
  *   device_error        optional device int32 (NULL = not reported)
@@ -75,9 +80,11 @@ typedef enum {
  * (bit copies).  INT8: per (token, head) absmax quantiser of "KV Cache
  * Engineering for LLM Serving", section 8, at 8 bits in IEEE float32:
  * scale = max|x| / 127, code = clamp(rint(x / scale), -127, 127) (ties to
- * even); an all-zero row stores scale 0 and codes 0.  FP8_E4M3: code =
- * E4M3(x / scale_h) rounded to nearest-even, saturating at +-448; scale_h == 0
- * stores code 0.  head_dim must be 64, 128 or 256; pointers 16-byte aligned.
+ * even); an all-zero row stores scale 0 and codes 0.  INT4: the same rule at 4
+ * bits, scale = max|x| / 7, codes -7..7 packed two per byte.  FP8_E4M3: code =
+ * E4M3(x / scale_h) rounded to nearest-even, saturating at +-448; FP8_E5M2
+ * likewise at +-57344; scale_h == 0 stores code 0.  head_dim must be 64, 128
+ * or 256; pointers 16-byte aligned.
  * Slots of one call must be distinct, and must not lie in blocks shared by
  * several sequences (copy-on-write is the caller's job: Chapter 18, Prefix
  * Caching).
@@ -105,8 +112,8 @@ size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int h
  *   score_p = sm_scale * <query[s,h,:], K_p[kv,:]>
  *   out[s,h,:] = sum_p softmax(score)_p * V_p[kv,:]
  *   lse_out[s,h] = log(sum_p exp(score_p))             (natural log; optional)
- * K_p / V_p are dequantised for INT8 (code * scale[block,row,kv]) and
- * FP8_E4M3 (value * scale[kv]) caches.  L == 0 gives out = 0, lse = -inf.
+ * K_p / V_p are dequantised for INT8 / INT4 (code * scale[block,row,kv]) and
+ * FP8 (value * scale[kv]) caches.  L == 0 gives out = 0, lse = -inf.
  * Entries of block_tables past ceil(L / block_size) are never read, and rows of
  * the last block past L never enter the softmax.
  *
@@ -121,14 +128,14 @@ size_t pkv_paged_attention_workspace_size(int num_seqs, int n_q, int n_kv, int h
  *                      One workspace serves calls of any shape in stream order;
  *                      calls that may run concurrently need separate ones.
  *
- * A BF16/INT8/FP8 call makes two launches on `stream`: the decode kernel and,
+ * A call on a BF16 or quantised cache makes two launches on `stream`: the decode kernel and,
  * queued behind it with programmatic stream serialisation, the merge of
  * sequences whose blocks were split over several CTAs.
  *
  * Supported: block_size 16; act F32 with an F32 cache (head_dim 32..256, a
  * multiple of 32); act BF16 with a BF16 cache (head_dim 64 or 128); act BF16
- * or F32 with an INT8 or FP8_E4M3 cache (head_dim 128); n_q a multiple of n_kv
- * with n_q / n_kv <= 64.  Pointers 16-byte aligned.
+ * or F32 with an INT8, INT4, FP8_E4M3 or FP8_E5M2 cache (head_dim 128); n_q a
+ * multiple of n_kv with n_q / n_kv <= 64.  Pointers 16-byte aligned.
  */
 pkv_status pkv_paged_attention_decode(void* out, const void* query, const void* key_cache, const void* value_cache,
                                       const float* k_scale, const float* v_scale, const int32_t* block_tables,
@@ -338,16 +345,17 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const
  * diverges, only the affected block is duplicated ("Chapter 18 - KV-Cache
  * Optimization Strategies", Prefix Caching; KV-cache overview page t13_4,
  * copy-on-write paragraph).  For each pair p: block block_mapping[2p+1] of the
- * K and V pools (and, for INT8, of k_scale / v_scale) <- block block_mapping[2p].
+ * K and V pools (and, for INT8 / INT4, of k_scale / v_scale) <- block block_mapping[2p].
  *
  *   key_cache, value_cache  device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
- *   k_scale, v_scale        INT8 only: device [num_blocks, block_size, n_kv]; NULL otherwise
+ *   k_scale, v_scale        INT8 / INT4: device [num_blocks, block_size, n_kv]; NULL otherwise
  *                           (FP8 per-head scales belong to no block)
  *   block_mapping           device (or mapped host) int64 [num_pairs, 2] = (src, dst)
  * Destinations must be distinct and no block may be both a source and a
  * destination in one call (all pairs run in parallel).  Out-of-range block ids
- * set PKV_DEVERR_BLOCK_RANGE and the pair is skipped.  n_kv * head_dim * bytes
- * must be a multiple of 16.
+ * set PKV_DEVERR_BLOCK_RANGE and the pair is skipped.  The bytes of one row
+ * (n_kv * head_dim * bytes per value, half a byte for INT4) must be a multiple
+ * of 16.
  */
 pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,
                            const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
@@ -359,7 +367,7 @@ pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, f
  * Blocks not needed now move to a larger, slower tier and come back when they
  * are needed again ("KV Cache Engineering for LLM Serving", section 12, Cache
  * Offloading from GPU).  For each pair p: block block_mapping[2p+1] of the dst
- * pools <- block block_mapping[2p] of the src pools (K, V and INT8 scales).
+ * pools <- block block_mapping[2p] of the src pools (K, V and INT8 / INT4 scales).
  * Either side may be page-locked host memory mapped into the device address
  * space (cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped): the
  * kernel reads or writes it directly over the host link.  Same layouts,

@@ -8,7 +8,7 @@ formula did not survive extraction) and notes 2 bytes for BF16, 1 for FP8.
 """
 from __future__ import annotations
 
-BYTES_PER_VALUE = {"f32": 4, "bf16": 2, "int8": 1, "fp8_e4m3": 1}
+BYTES_PER_VALUE = {"f32": 4, "bf16": 2, "int8": 1, "fp8_e4m3": 1, "fp8_e5m2": 1, "int4": 0.5}
 
 
 def cache_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, bytes_per_value: float) -> float:
@@ -32,8 +32,8 @@ def tokens_in_pool(pool_bytes: float, bytes_per_token: float) -> int:
 
 
 def scale_bytes_per_token(cache_dtype: str, kv_heads: int) -> int:
-    """Per-token scale metadata read with the codes: one fp32 per (token, head) for K and V with int8."""
-    return 2 * kv_heads * 4 if cache_dtype == "int8" else 0
+    """Per-token scale metadata read with the codes: one fp32 per (token, head) for K and V with int8 / int4."""
+    return 2 * kv_heads * 4 if cache_dtype in ("int8", "int4") else 0
 
 
 def decode_kv_bytes(w, unique: bool = True) -> int:

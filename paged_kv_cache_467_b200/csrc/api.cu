@@ -44,7 +44,9 @@ int device_smem_optin() {
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-static bool valid_dtype(int d) { return d >= PKV_F32 && d <= PKV_FP8_E4M3; }
+static bool valid_dtype(int d) { return d >= PKV_F32 && d <= PKV_INT4; }
+static bool row_scaled(int d) { return d == PKV_INT8 || d == PKV_INT4; }
+static bool head_scaled(int d) { return d == PKV_FP8_E4M3 || d == PKV_FP8_E5M2; }
 
 // Shape rules of the decode kernels; PKV_OK when the tensor-core path or the
 // F32 path can run it.
@@ -94,7 +96,7 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   if (num_seqs == 0) return PKV_OK;
   if (!out || !query || !key_cache || !value_cache || !block_tables || !context_lens) return PKV_ERR_INVALID_ARG;
   if (!aligned16(out) || !aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache)) return PKV_ERR_INVALID_ARG;
-  const bool quant = cache_dtype == PKV_INT8 || cache_dtype == PKV_FP8_E4M3;
+  const bool quant = row_scaled(cache_dtype) || head_scaled(cache_dtype);
   if (quant && (!k_scale || !v_scale || !aligned16(k_scale) || !aligned16(v_scale))) return PKV_ERR_INVALID_ARG;
   if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
   if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
@@ -173,7 +175,7 @@ static pkv_status move_plan(const void* src_k, const void* src_v, const float* s
   if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
   if (num_pairs > 0 && (!pairs || !src_k || !src_v || !dst_k || !dst_v)) return PKV_ERR_INVALID_ARG;
   const size_t elem = cache_dtype == PKV_F32 ? 4 : (cache_dtype == PKV_BF16 ? 2 : 1);
-  const size_t row = (size_t)n_kv * head_dim * elem;
+  const size_t row = cache_dtype == PKV_INT4 ? (size_t)n_kv * head_dim / 2 : (size_t)n_kv * head_dim * elem;
   if (row % 16 != 0) return PKV_ERR_UNSUPPORTED;
   if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v)) return PKV_ERR_INVALID_ARG;
   src[0] = src_k;
@@ -182,7 +184,7 @@ static pkv_status move_plan(const void* src_k, const void* src_v, const float* s
   dst[1] = dst_v;
   bpb[0] = bpb[1] = row * block_size;
   *npools = 2;
-  const bool int8 = cache_dtype == PKV_INT8;
+  const bool int8 = row_scaled(cache_dtype);
   if (int8 != (src_ks && src_vs && dst_ks && dst_vs)) return PKV_ERR_INVALID_ARG;
   if (int8) {
     if (!aligned16(src_ks) || !aligned16(src_vs) || !aligned16(dst_ks) || !aligned16(dst_vs)) return PKV_ERR_INVALID_ARG;
@@ -217,7 +219,7 @@ pkv_status pkv_kv_cache_write(const void* key, const void* value, void* key_cach
   if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PKV_ERR_INVALID_ARG;
   if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
     return PKV_ERR_INVALID_ARG;
-  const bool quant = cache_dtype == PKV_INT8 || cache_dtype == PKV_FP8_E4M3;
+  const bool quant = row_scaled(cache_dtype) || head_scaled(cache_dtype);
   if (quant && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
   if (!quant && (k_scale || v_scale)) return PKV_ERR_INVALID_ARG;
   return launch_cache_write(key, value, key_cache, value_cache, k_scale, v_scale, slot_mapping, num_tokens, n_kv,
@@ -348,7 +350,7 @@ pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* ke
                                     void* workspace, size_t workspace_bytes, int32_t* device_error,
                                     const pkv_decode_tuning* tuning, void* stream) {
   if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
-  if (cache_dtype == PKV_FP8_E4M3 && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+  if (head_scaled(cache_dtype) && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
   return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
                      context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream, key,

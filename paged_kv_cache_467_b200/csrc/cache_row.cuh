@@ -6,14 +6,17 @@
 // Serving", section 8, at 8 bits with one float32 scale per (token, head):
 // scale = max|x| / 127, code = clamp(rint(x / scale), -127, 127), divisions
 // IEEE round-to-nearest, rint ties-to-even; an all-zero row stores scale 0.
-// FP8 stores the E4M3 value of x / scale_h, nearest-even, saturated at 448.
+// INT4 is the same quantiser at 4 bits (scale = max|x| / 7, codes -7..7), two
+// codes per byte: element 2j in the low nibble of byte j, two's complement.
+// FP8 stores the E4M3 (or E5M2) value of x / scale_h, nearest-even, saturated
+// at the largest finite value (448, or 57344).
 #pragma once
 
 #include "pkv_device.cuh"
 
 namespace pkv {
 
-enum WriteKind : int { WK_COPY = 0, WK_INT8 = 1, WK_FP8 = 2 };
+enum WriteKind : int { WK_COPY = 0, WK_INT8 = 1, WK_FP8 = 2, WK_E5M2 = 3, WK_INT4 = 4 };
 
 template <int BYTES>
 __device__ __forceinline__ void copy_lane(void* dst, const void* src) {
@@ -73,6 +76,26 @@ __device__ __forceinline__ void write_row(const void* src_row, void* cache, floa
   } else {
     float x[EPL];
     load_lane<BF16, EPL>(x, static_cast<const uint8_t*>(src_row) + lane * EPL * AB);
+    if constexpr (KIND == WK_INT4) {
+      float amax = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      amax = warp_max(amax);
+      const float scale = __fdiv_rn(amax, 7.0f);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        float q = scale == 0.f ? 0.f : rintf(__fdiv_rn(x[e], scale));
+        q = fminf(fmaxf(q, -7.f), 7.f);
+        packed |= ((uint32_t)(int)q & 0xFu) << (4 * e);
+      }
+      if (lane == 0) scales[dst_row] = scale;
+      uint8_t* dst = static_cast<uint8_t*>(cache) + dst_row * (D / 2) + lane * (EPL / 2);
+      if constexpr (EPL == 2) *dst = (uint8_t)packed;
+      else if constexpr (EPL == 4) *reinterpret_cast<uint16_t*>(dst) = (uint16_t)packed;
+      else *reinterpret_cast<uint32_t*>(dst) = packed;
+      return;
+    }
     uint8_t code[EPL];
     if constexpr (KIND == WK_INT8) {
       float amax = 0.f;
@@ -90,8 +113,10 @@ __device__ __forceinline__ void write_row(const void* src_row, void* cache, floa
     } else {
       const float scale = __ldg(scales + h);
 #pragma unroll
+      constexpr __nv_fp8_interpretation_t fmt = KIND == WK_E5M2 ? __NV_E5M2 : __NV_E4M3;
+#pragma unroll
       for (int e = 0; e < EPL; ++e)
-        code[e] = scale == 0.f ? (uint8_t)0 : (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(x[e], scale), __NV_SATFINITE, __NV_E4M3);
+        code[e] = scale == 0.f ? (uint8_t)0 : (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(x[e], scale), __NV_SATFINITE, fmt);
     }
     store_bytes<EPL>(static_cast<uint8_t*>(cache) + dst_row * D + lane * EPL, code);
   }

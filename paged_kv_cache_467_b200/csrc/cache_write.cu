@@ -92,6 +92,10 @@ pkv_status launch_cache_write(const void* key, const void* value, void* key_cach
     return bf16 ? launch_kind<true, WK_INT8>(p, head_dim, stream) : launch_kind<false, WK_INT8>(p, head_dim, stream);
   if (cache == PKV_FP8_E4M3)
     return bf16 ? launch_kind<true, WK_FP8>(p, head_dim, stream) : launch_kind<false, WK_FP8>(p, head_dim, stream);
+  if (cache == PKV_FP8_E5M2)
+    return bf16 ? launch_kind<true, WK_E5M2>(p, head_dim, stream) : launch_kind<false, WK_E5M2>(p, head_dim, stream);
+  if (cache == PKV_INT4)
+    return bf16 ? launch_kind<true, WK_INT4>(p, head_dim, stream) : launch_kind<false, WK_INT4>(p, head_dim, stream);
   return bf16 ? launch_kind<true, WK_COPY>(p, head_dim, stream) : launch_kind<false, WK_COPY>(p, head_dim, stream);
 }
 

@@ -219,9 +219,12 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
 template <int CACHE, int D>
 struct TcTraits {
   static constexpr int kElem = CACHE == TC_BF16 ? 2 : 1;
-  static constexpr int kChunks = D * kElem / 128;  // 128-byte chunks per head row
-  static constexpr int kTile = kChunks * 2048;     // one head's 16-row tile
-  static constexpr int kSteps = D / 16;            // k-steps of Q.K and m-tiles of P.V
+  // bytes of one TMA box row: a 128-byte chunk, or an INT4 head row (64 bytes)
+  static constexpr int kChunkBytes = CACHE == TC_INT4 ? D / 2 : 128;
+  static constexpr int kChunks = CACHE == TC_INT4 ? 1 : D * kElem / 128;  // chunks per head row
+  static constexpr int kBox = kChunkBytes * 16;                            // one chunk of 16 rows
+  static constexpr int kTile = kChunks * kBox;                             // one head's 16-row tile
+  static constexpr int kSteps = D / 16;  // k-steps of Q.K and m-tiles of P.V
 };
 
 // Write one finished (or merged) row pair: heads 2c, 2c+1 of this lane.
@@ -388,11 +391,11 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
 #pragma unroll
               for (int ch = 0; ch < Tr::kChunks; ++ch) {
                 const int c1 = (hgk * p.HPC + hl) * Tr::kChunks + ch;
-                tma_load_3d(st + (hl * Tr::kChunks + ch) * 2048, &kmap, 0, c1, row, &full[stage]);
-                tma_load_3d(st + (p.HPC + hl) * Tr::kTile + ch * 2048, &vmap, 0, c1, row, &full[stage]);
+                tma_load_3d(st + (hl * Tr::kChunks + ch) * Tr::kBox, &kmap, 0, c1, row, &full[stage]);
+                tma_load_3d(st + (p.HPC + hl) * Tr::kTile + ch * Tr::kBox, &vmap, 0, c1, row, &full[stage]);
               }
             }
-            if constexpr (CACHE == TC_INT8) {
+            if constexpr (tc_row_scaled(CACHE)) {
               const size_t sb = (size_t)(ph >= 0 ? ph : 0) * kBlockSize * p.n_kv;
               const uint32_t bytes = 64u * p.n_kv;
               uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
@@ -461,7 +464,11 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       }
       const size_t dst_row = ((size_t)phys * kBlockSize + pos % kBlockSize) * p.n_kv + kv;
       const size_t src_row = (size_t)ss * p.n_kv + kv;
-      constexpr int kind = CACHE == TC_BF16 ? WK_COPY : (CACHE == TC_INT8 ? WK_INT8 : WK_FP8);
+      constexpr int kind = CACHE == TC_BF16   ? WK_COPY
+                           : CACHE == TC_INT8 ? WK_INT8
+                           : CACHE == TC_INT4 ? WK_INT4
+                           : CACHE == TC_E5M2 ? WK_E5M2
+                                              : WK_FP8;
       if (p.act_bf16) {
         write_row<true, kind, D / 32>(static_cast<const uint8_t*>(p.new_key) + src_row * D * 2, p.key_cache, p.k_scale,
                                       dst_row, kv, p.n_kv, lane);
@@ -527,6 +534,17 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         // MMA B fragment: dims ks*16 + 2c, +1 and ks*16 + 2c + 8, +9
         qraw[ks][0] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c) / 2) : 0u;
         qraw[ks][1] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c + 8) / 2) : 0u;
+      } else if constexpr (CACHE == TC_INT4) {
+        // k-step ks = 2w + h pairs dims 32c + 8w + 2h + {0, 4} and {1, 5} (the
+        // nibble pairs of the INT4 word w of lane column c); one 16-byte load
+        // of dims 32c + 8w .. + 7 serves ks = 2w and 2w + 1
+        if (ks & 1) continue;
+        const uint4 w = q_ok ? __ldg(reinterpret_cast<const uint4*>(q32 + (32 * c + 4 * ks) / 2))
+                             : make_uint4(0u, 0u, 0u, 0u);
+        qraw[ks][0] = prmt(w.x, w.z, 0x5410);
+        qraw[ks][1] = prmt(w.x, w.z, 0x7632);
+        qraw[ks + 1][0] = prmt(w.y, w.w, 0x5410);
+        qraw[ks + 1][1] = prmt(w.y, w.w, 0x7632);
       } else {
         // k-step ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
         const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
@@ -535,10 +553,12 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         qraw[ks][1] = w.y;
       }
     }
-    if constexpr (CACHE == TC_FP8) {
-      // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256)
-      raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
-      raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
+    if constexpr (tc_fp8(CACHE)) {
+      // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256), or
+      // E5M2 values exactly (an E5M2 byte is the top byte of its f16)
+      constexpr float fold = CACHE == TC_FP8 ? 256.f : 1.f;
+      raw_k_scale = __ldg(p.k_scale + kv) * fold;
+      raw_v_scale = __ldg(p.v_scale + kv) * fold;
     }
   };
 
@@ -559,6 +579,24 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         if (ks & 1) mma_bf16(sb, af, qf[ks][0], qf[ks][1]);
         else mma_bf16(sa, af, qf[ks][0], qf[ks][1]);
       }
+    } else if constexpr (CACHE == TC_INT4) {
+      // lane (g, c) reads the 16-byte chunk c (dims 32c .. 32c+31) of rows g and
+      // g+8; 64-byte rows under the 64-byte swizzle: chunk c of row r sits at
+      // chunk c ^ ((r >> 1) & 3), the same for rows g and g+8
+      const uint32_t kb = kt + g * 64 + ((uint32_t)(c ^ ((g >> 1) & 3)) << 4);
+      const uint4 r0 = lds128(kb), r1 = lds128(kb + 512);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int w = ks >> 1, h = ks & 1;
+        const uint32_t x0 = (&r0.x)[w] ^ 0x88888888u, x1 = (&r1.x)[w] ^ 0x88888888u;
+        uint32_t af[4];
+        af[0] = i4x2_to_f16x2(x0 >> (8 * h));
+        af[1] = i4x2_to_f16x2(x1 >> (8 * h));
+        af[2] = i4x2_to_f16x2(x0 >> (8 * h + 4));
+        af[3] = i4x2_to_f16x2(x1 >> (8 * h + 4));
+        if (ks & 1) mma_f16(sb, af, qf[ks][0], qf[ks][1]);
+        else mma_f16(sa, af, qf[ks][0], qf[ks][1]);
+      }
     } else {
       // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each)
       uint4 kr[2][2];
@@ -578,6 +616,12 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           af[1] = i8x2_to_f16x2(x1, 0x4140);
           af[2] = i8x2_to_f16x2(x0, 0x4342);
           af[3] = i8x2_to_f16x2(x1, 0x4342);
+        } else if constexpr (CACHE == TC_E5M2) {
+          // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, as the f16 top bytes
+          af[0] = prmt(w0, 0u, 0x1404);
+          af[1] = prmt(w1, 0u, 0x1404);
+          af[2] = prmt(w0, 0u, 0x3424);
+          af[3] = prmt(w1, 0u, 0x3424);
         } else {
           // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, values / 256
           af[0] = e4m3x2_hi_to_f16x2_div256(prmt(w0, 0u, 0x1404));
@@ -593,14 +637,14 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     float sc0 = p.scale_log2, sc1 = p.scale_log2;
     vsc[0] = vsc[1] = 1.f;
     const int kvh = hg * p.HPC + head_local;
-    if constexpr (CACHE == TC_INT8) {
+    if constexpr (tc_row_scaled(CACHE)) {
       const float* ksm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile);
       const float* vsm = ksm + kBlockSize * p.n_kv;
       sc0 *= ksm[t0 * p.n_kv + kvh];
       sc1 *= ksm[t1 * p.n_kv + kvh];
       vsc[0] = vsm[t0 * p.n_kv + kvh];
       vsc[1] = vsm[t1 * p.n_kv + kvh];
-    } else if constexpr (CACHE == TC_FP8) {
+    } else if constexpr (tc_fp8(CACHE)) {
       sc0 *= head_k_scale;
       sc1 *= head_k_scale;
     }
@@ -619,7 +663,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     if constexpr (CACHE == TC_BF16) {
       pb0 = movmatrix_trans(pack_bf16(pr[0], pr[1]));
       pb1 = movmatrix_trans(pack_bf16(pr[2], pr[3]));
-    } else if constexpr (CACHE == TC_INT8) {
+    } else if constexpr (tc_row_scaled(CACHE)) {
       pb0 = movmatrix_trans(pack_f16(ok0 ? pr[0] * vsc[0] : 0.f, ok0 ? pr[1] * vsc[0] : 0.f));
       pb1 = movmatrix_trans(pack_f16(ok1 ? pr[2] * vsc[1] : 0.f, ok1 ? pr[3] * vsc[1] : 0.f));
     } else {
@@ -644,6 +688,27 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         af[3] &= mhi;
         mma_bf16(acc[mt], af, pb0, pb1);
       }
+    } else if constexpr (CACHE == TC_INT4) {
+      // lane (g, c) reads dims 16g .. 16g+15 (8 bytes at byte 8g, in chunk g/2)
+      // of token rows 2c, 2c+1, 2c+8, 2c+9 (64-byte rows, 64-byte swizzle)
+      auto row8 = [&](int r) {
+        return lds64(vt + r * 64 + ((uint32_t)((g >> 1) ^ ((r >> 1) & 3)) << 4) + (g & 1) * 8);
+      };
+      const uint2 x0 = row8(2 * c), y0 = row8(2 * c + 1), x1 = row8(2 * c + 8), y1 = row8(2 * c + 9);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        // dims 16g + 2mt (+1): byte mt of the 8, low (high) nibble; tokens side by side
+        const int wi = mt >> 2, b = mt & 3;
+        const uint32_t sel = b | (b << 4) | ((4 + b) << 8) | ((4 + b) << 12);
+        const uint32_t z0 = prmt((&x0.x)[wi], (&y0.x)[wi], sel) ^ 0x88888888u;
+        const uint32_t z1 = prmt((&x1.x)[wi], (&y1.x)[wi], sel) ^ 0x88888888u;
+        uint32_t af[4];
+        af[0] = i4x2_to_f16x2(z0) & mlo;
+        af[1] = i4x2_to_f16x2(z0 >> 4) & mlo;
+        af[2] = i4x2_to_f16x2(z1) & mhi;
+        af[3] = i4x2_to_f16x2(z1 >> 4) & mhi;
+        mma_f16(acc[mt], af, pb0, pb1);
+      }
     } else {
       // lane (g, c) reads chunk g of token rows 2c, 2c+1, 2c+8, 2c+9
       const uint4 x0 = lds128(vt + voff);
@@ -667,10 +732,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           const uint32_t A = 2 * (mt & 1);
           const uint32_t s0 = ((4 + A) << 12) | ((4 + A) << 8) | (A << 4) | A;
           const uint32_t s1 = s0 + 0x1111u;
-          af[0] = e4m3x2_hi_to_f16x2_div256(prmt((&x0.x)[wi], (&y0.x)[wi], s0));
-          af[1] = e4m3x2_hi_to_f16x2_div256(prmt((&x0.x)[wi], (&y0.x)[wi], s1));
-          af[2] = e4m3x2_hi_to_f16x2_div256(prmt((&x1.x)[wi], (&y1.x)[wi], s0));
-          af[3] = e4m3x2_hi_to_f16x2_div256(prmt((&x1.x)[wi], (&y1.x)[wi], s1));
+          af[0] = prmt((&x0.x)[wi], (&y0.x)[wi], s0);
+          af[1] = prmt((&x0.x)[wi], (&y0.x)[wi], s1);
+          af[2] = prmt((&x1.x)[wi], (&y1.x)[wi], s0);
+          af[3] = prmt((&x1.x)[wi], (&y1.x)[wi], s1);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            if constexpr (CACHE == TC_FP8) af[k] = e4m3x2_hi_to_f16x2_div256(af[k]);
+            else af[k] &= 0xFF00FF00u;  // E5M2 bytes are the f16 top bytes; clear the duplicated low bytes
+          }
         }
         af[0] &= mlo;
         af[1] &= mlo;
@@ -788,17 +858,31 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           const int kv = hg * p.HPC + head_local;
           const bool q_ok = qc * 8 + g < p.G;
           const size_t qoff = ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
+          const float* qrow = reinterpret_cast<const float*>(p.query) + qoff;
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
-            const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
-            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (q_ok) w = __ldg(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.query) + qoff + d0));
-            qf[ks][0] = pack_f16(w.x, w.y);
-            qf[ks][1] = pack_f16(w.z, w.w);
+            if constexpr (CACHE == TC_INT4) {
+              // dims 32c + 8w + 2h + {0, 4} and {1, 5} for ks = 2w + h (as fetch_query)
+              const int d0 = 32 * c + 8 * (ks >> 1) + 2 * (ks & 1);
+              float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
+              if (q_ok) {
+                lo = __ldg(reinterpret_cast<const float2*>(qrow + d0));
+                hi = __ldg(reinterpret_cast<const float2*>(qrow + d0 + 4));
+              }
+              qf[ks][0] = pack_f16(lo.x, hi.x);
+              qf[ks][1] = pack_f16(lo.y, hi.y);
+            } else {
+              const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+              float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (q_ok) w = __ldg(reinterpret_cast<const float4*>(qrow + d0));
+              qf[ks][0] = pack_f16(w.x, w.y);
+              qf[ks][1] = pack_f16(w.z, w.w);
+            }
           }
-          if constexpr (CACHE == TC_FP8) {
-            raw_k_scale = __ldg(p.k_scale + kv) * 256.f;
-            raw_v_scale = __ldg(p.v_scale + kv) * 256.f;
+          if constexpr (tc_fp8(CACHE)) {
+            constexpr float fold = CACHE == TC_FP8 ? 256.f : 1.f;
+            raw_k_scale = __ldg(p.k_scale + kv) * fold;
+            raw_v_scale = __ldg(p.v_scale + kv) * fold;
           }
         }
       }
@@ -830,7 +914,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
         lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
       }
-      const float post = (CACHE == TC_FP8) ? head_v_scale : 1.f;
+      const float post = tc_fp8(CACHE) ? head_v_scale : 1.f;
       const float inv0 = post / lt0, inv1 = post / lt1;
       const float lse0 = m0 + log2f(lt0), lse1 = m1 + log2f(lt1);
       const bool contained = P[u] >= a && P[u + 1] <= b;
@@ -899,17 +983,23 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Rank-3 view of a cache pool [num_blocks * 16 rows][n_kv * head_dim * elem bytes]
 // as (128-byte chunk elements, chunk index, row), box = 1 chunk x 16 rows.
-static pkv_status make_kv_map(CUtensorMap* map, const void* base, int elem, int n_kv, int head_dim, int64_t rows) {
+// Rank-3 view of a pool: (elements of one chunk, chunk index, token row).  A
+// chunk is 128 bytes (BF16 / INT8 / FP8 rows), or a whole 64-byte INT4 head row
+// (64-byte swizzle).
+static pkv_status make_kv_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes_i,
+                              int64_t rows) {
   auto fn = encode_fn();
   if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
-  const cuuint64_t row_bytes = (cuuint64_t)n_kv * head_dim * elem;
-  cuuint64_t dims[3] = {(cuuint64_t)(128 / elem), row_bytes / 128, (cuuint64_t)rows};
-  cuuint64_t strides[2] = {128, row_bytes};
-  cuuint32_t box[3] = {(cuuint32_t)(128 / elem), 1, (cuuint32_t)kBlockSize};
+  const cuuint64_t row_bytes = (cuuint64_t)row_bytes_i;
+  const cuuint64_t cb = (cuuint64_t)chunk_bytes;
+  cuuint64_t dims[3] = {cb / elem, row_bytes / cb, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {cb, row_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(cb / elem), 1, (cuuint32_t)kBlockSize};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  chunk_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return driver_fail((int)r, "cuTensorMapEncodeTiled");
   return PKV_OK;
 }
@@ -978,11 +1068,14 @@ static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CU
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream) {
   const int elem = plan.cache_kind == TC_BF16 ? 2 : 1;
+  const bool int4 = plan.cache_kind == TC_INT4;
+  const int row_bytes = int4 ? s.n_kv * s.head_dim / 2 : s.n_kv * s.head_dim * elem;
+  const int chunk_bytes = int4 ? s.head_dim / 2 : 128;
   const int64_t rows = a.num_blocks * kBlockSize;
   CUtensorMap km, vm;
-  pkv_status st = make_kv_map(&km, a.key_cache, elem, s.n_kv, s.head_dim, rows);
+  pkv_status st = make_kv_map(&km, a.key_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
-  st = make_kv_map(&vm, a.value_cache, elem, s.n_kv, s.head_dim, rows);
+  st = make_kv_map(&vm, a.value_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
 
   TcParams prm;
@@ -1030,6 +1123,8 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
     return launch_one<TC_BF16, 128>(plan, km, vm, prm, stream);
   }
   if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, prm, stream);
+  if (plan.cache_kind == TC_INT4) return launch_one<TC_INT4, 128>(plan, km, vm, prm, stream);
+  if (plan.cache_kind == TC_E5M2) return launch_one<TC_E5M2, 128>(plan, km, vm, prm, stream);
   return launch_one<TC_FP8, 128>(plan, km, vm, prm, stream);
 }
 
@@ -1037,13 +1132,18 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan) {
   TcPlan pl{};
-  pl.cache_kind = s.cache == PKV_BF16 ? TC_BF16 : (s.cache == PKV_INT8 ? TC_INT8 : TC_FP8);
+  pl.cache_kind = s.cache == PKV_BF16        ? TC_BF16
+                  : s.cache == PKV_INT8      ? TC_INT8
+                  : s.cache == PKV_INT4      ? TC_INT4
+                  : s.cache == PKV_FP8_E5M2 ? TC_E5M2
+                                             : TC_FP8;
   const int elem = pl.cache_kind == TC_BF16 ? 2 : 1;
-  pl.chunks = s.head_dim * elem / 128;
+  pl.chunks = pl.cache_kind == TC_INT4 ? 1 : s.head_dim * elem / 128;
+  const size_t tile_bytes = pl.cache_kind == TC_INT4 ? (size_t)s.head_dim / 2 * 16 : (size_t)pl.chunks * 2048;
   pl.G = s.n_q / s.n_kv;
   pl.QC = (pl.G + 7) / 8;
   const int want_hpc = tuning ? tuning->heads_per_cta : 0;
-  const size_t scale_bytes = pl.cache_kind == TC_INT8 ? 2 * 64 * (size_t)s.n_kv : 0;
+  const size_t scale_bytes = tc_row_scaled(pl.cache_kind) ? 2 * 64 * (size_t)s.n_kv : 0;
   if (want_hpc > 0) {
     if (s.n_kv % want_hpc != 0 || want_hpc * pl.QC > kMaxConsumerWarps) return PKV_ERR_INVALID_ARG;
     pl.HPC = want_hpc;
@@ -1064,7 +1164,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.HG = s.n_kv / pl.HPC;
   pl.NCW = pl.HPC * pl.QC;
   pl.units = s.num_seqs * pl.HG;
-  pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * pl.chunks * 2048 + scale_bytes);
+  pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * tile_bytes + scale_bytes);
   pl.stage_bytes = (uint32_t)align_up(pl.tx_bytes, 1024);
 
   const int sms = device_sm_count();

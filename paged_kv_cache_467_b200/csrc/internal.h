@@ -17,7 +17,9 @@ constexpr int kTargetCtasPerSm = 4;
 constexpr size_t kSmemPerSm = 233472;  // 228 KB of shared memory per SM
 
 // Cache kinds of the tensor-core decode kernel.
-enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2 };
+enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2, TC_E5M2 = 3, TC_INT4 = 4 };
+__host__ __device__ constexpr bool tc_fp8(int c) { return c == TC_FP8 || c == TC_E5M2; }          // one scale per KV head
+__host__ __device__ constexpr bool tc_row_scaled(int c) { return c == TC_INT8 || c == TC_INT4; }  // one scale per (token, head)
 
 struct DecodeShape {
   int num_seqs, n_q, n_kv, head_dim, block_size;

@@ -192,6 +192,23 @@ __device__ __forceinline__ uint32_t e4m3x2_hi_to_f16x2_div256(uint32_t t) {
   return ((t >> 1) & 0x3F803F80u) | (t & 0x80008000u);
 }
 
+// Two 4-bit codes held as offset-binary nibbles (code + 8) at bits [3:0] and
+// [19:16] of t (other bits ignored) -> f16x2 of the codes, exactly: the nibble
+// n ORed into the mantissa of 1024.0 (0x6400) reads as 1024 + n, and
+// subtracting 1032 leaves n - 8.
+__device__ __forceinline__ uint32_t i4x2_to_f16x2(uint32_t t) {
+  const uint32_t h = (t & 0x000F000Fu) | 0x64006400u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __half2half2(__ushort_as_half(0x6408)));  // 0x6408 = 1032.0
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

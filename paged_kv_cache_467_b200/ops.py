@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
-PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3 = 0, 1, 2, 3
+PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3, PKV_FP8_E5M2, PKV_INT4 = 0, 1, 2, 3, 4, 5
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype", 3: "workspace missing or too small", 4: "CUDA error"}
 DEVERR_SLOT_RANGE, DEVERR_BLOCK_RANGE, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
@@ -26,6 +26,8 @@ _CACHE_DTYPES = {
     "bf16": PKV_BF16,
     "int8": PKV_INT8,
     "fp8_e4m3": PKV_FP8_E4M3,
+    "fp8_e5m2": PKV_FP8_E5M2,
+    "int4": PKV_INT4,  # pools hold uint8 bytes, two codes each: pass cache_dtype="int4"
 }
 
 
@@ -124,6 +126,8 @@ def act_code(t: torch.Tensor) -> int:
 
 
 def cache_code(t: torch.Tensor, cache_dtype: str | None = None) -> int:
+    """Cache dtype code from an explicit name, else from the pool's torch dtype
+    (uint8 pools are E4M3 unless named; an INT4 pool must be named "int4")."""
     if cache_dtype is not None:
         return _CACHE_DTYPES[cache_dtype]
     if t.dtype == torch.float32:
@@ -134,16 +138,20 @@ def cache_code(t: torch.Tensor, cache_dtype: str | None = None) -> int:
         return PKV_INT8
     if t.dtype in (torch.uint8, torch.float8_e4m3fn):
         return PKV_FP8_E4M3
+    if t.dtype == torch.float8_e5m2:
+        return PKV_FP8_E5M2
     raise TypeError(f"unsupported cache dtype {t.dtype}")
 
 
-def kv_cache_write(key, value, key_cache, value_cache, slot_mapping, k_scale=None, v_scale=None, device_error=None):
+def kv_cache_write(key, value, key_cache, value_cache, slot_mapping, k_scale=None, v_scale=None, device_error=None,
+                   cache_dtype: str | None = None):
     """Append rows of ``key``/``value`` [T, n_kv, d] at ``slot_mapping`` [T] (int64)."""
     T, n_kv, d = key.shape
     num_blocks, block_size = key_cache.shape[0], key_cache.shape[1]
     st = lib.pkv_kv_cache_write(
         _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(slot_mapping),
-        T, n_kv, d, block_size, num_blocks, act_code(key), cache_code(key_cache), _ptr(device_error), _stream(key.device),
+        T, n_kv, d, block_size, num_blocks, act_code(key), cache_code(key_cache, cache_dtype), _ptr(device_error),
+        _stream(key.device),
     )
     _check(st, "pkv_kv_cache_write")
 
@@ -188,11 +196,12 @@ def paged_attention_decode(
     workspace=None,
     device_error=None,
     tuning: DecodeTuning | None = None,
+    cache_dtype: str | None = None,
 ):
     """Decode attention of ``query`` [S, n_q, d] over a paged cache into ``out``."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ccode = cache_code(key_cache)
+    ccode = cache_code(key_cache, cache_dtype)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:
@@ -214,11 +223,11 @@ def paged_attention_decode(
 
 def paged_decode_step(out, query, key, value, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
                       sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None, workspace=None,
-                      device_error=None, tuning: DecodeTuning | None = None):
+                      device_error=None, tuning: DecodeTuning | None = None, cache_dtype: str | None = None):
     """One fused decode step: append ``key``/``value`` [S, n_kv, d] as token L-1 of each sequence, then attend."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ccode = cache_code(key_cache)
+    ccode = cache_code(key_cache, cache_dtype)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:
@@ -241,7 +250,7 @@ def paged_decode_step(out, query, key, value, key_cache, value_cache, block_tabl
 
 def paged_attention_decode_static(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
                                   sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None,
-                                  device_error=None):
+                                  device_error=None, cache_dtype: str | None = None):
     """pkv_paged_attention_decode_static: decode with the library's own scratch (no workspace argument)."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
@@ -250,7 +259,7 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     st = lib.pkv_paged_attention_decode_static(
         _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
-        float(sm_scale), act_code(query), cache_code(key_cache), _ptr(lse_out), _ptr(device_error),
+        float(sm_scale), act_code(query), cache_code(key_cache, cache_dtype), _ptr(lse_out), _ptr(device_error),
         _stream(query.device),
     )
     if st != 0:
@@ -258,34 +267,42 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     return out
 
 
-def copy_blocks(key_cache, value_cache, block_mapping, k_scale=None, v_scale=None, device_error=None, stream=None):
+def copy_blocks(key_cache, value_cache, block_mapping, k_scale=None, v_scale=None, device_error=None, stream=None,
+                cache_dtype: str | None = None):
     """Copy-on-write block copies inside one pool; ``block_mapping`` int64 [P, 2] = (src, dst)."""
     nb, bs, n_kv, d = key_cache.shape
+    code = cache_code(key_cache, cache_dtype)
+    if code == PKV_INT4:
+        d *= 2
     st = lib.pkv_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_mapping),
-                             block_mapping.shape[0], n_kv, d, bs, nb, cache_code(key_cache), _ptr(device_error),
+                             block_mapping.shape[0], n_kv, d, bs, nb, code, _ptr(device_error),
                              stream if stream is not None else _stream(key_cache.device))
     _check(st, "pkv_copy_blocks")
 
 
 def swap_blocks(src_key, src_value, dst_key, dst_value, block_mapping, src_k_scale=None, src_v_scale=None,
-                dst_k_scale=None, dst_v_scale=None, device_error=None, device=None):
+                dst_k_scale=None, dst_v_scale=None, device_error=None, device=None, cache_dtype: str | None = None):
     """Move blocks between two pools (either may be pinned host memory); (src, dst) pairs."""
     snb, bs, n_kv, d = src_key.shape
+    code = cache_code(src_key, cache_dtype)
+    if code == PKV_INT4:
+        d *= 2
     dev = device if device is not None else (src_key.device if src_key.is_cuda else dst_key.device)
     st = lib.pkv_swap_blocks(_ptr(src_key), _ptr(src_value), _ptr(src_k_scale), _ptr(src_v_scale), snb,
                              _ptr(dst_key), _ptr(dst_value), _ptr(dst_k_scale), _ptr(dst_v_scale), dst_key.shape[0],
-                             _ptr(block_mapping), block_mapping.shape[0], n_kv, d, bs, cache_code(src_key),
+                             _ptr(block_mapping), block_mapping.shape[0], n_kv, d, bs, code,
                              _ptr(device_error), _stream(dev))
     _check(st, "pkv_swap_blocks")
 
 
 def paged_attention_decode_window(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
                                   window: int, sinks: int = 0, sm_scale: float | None = None, k_scale=None,
-                                  v_scale=None, lse_out=None, workspace=None, device_error=None):
+                                  v_scale=None, lse_out=None, workspace=None, device_error=None,
+                                  cache_dtype: str | None = None):
     """Decode attention over positions [0, sinks) and [L - window, L) of each sequence."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ccode = cache_code(key_cache)
+    ccode = cache_code(key_cache, cache_dtype)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:
@@ -331,11 +348,12 @@ def quest_select(query, page_min, page_max, block_tables, context_lens, max_cont
 
 def paged_attention_decode_pages(out, query, key_cache, value_cache, block_tables, context_lens, max_context_len: int,
                                  pages, sm_scale: float | None = None, k_scale=None, v_scale=None, lse_out=None,
-                                 workspace=None, device_error=None, tuning: DecodeTuning | None = None):
+                                 workspace=None, device_error=None, tuning: DecodeTuning | None = None,
+                                 cache_dtype: str | None = None):
     """Decode attention over the logical pages listed in ``pages`` [S, n_kv, k] for each KV head."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    ccode = cache_code(key_cache)
+    ccode = cache_code(key_cache, cache_dtype)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:

@@ -31,7 +31,8 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-DTYPES = ("f32", "bf16", "int8", "fp8_e4m3")
+DTYPES = ("f32", "bf16", "int8", "fp8_e4m3", "fp8_e5m2", "int4")
+FP8_MAX = {"fp8_e4m3": 448.0, "fp8_e5m2": 57344.0}  # largest finite value of each format
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
@@ -214,7 +215,8 @@ class DecodeWorkload:
         return k, v
 
     def fp8_head_scales(self) -> tuple[np.ndarray, np.ndarray]:
-        """Static per-KV-head scales for an E4M3 cache: absmax of the head / 448.
+        """Static per-KV-head scales for an FP8 cache: absmax of the head / the
+        format's largest finite value (448 for E4M3, 57344 for E5M2).
 
         Calibration input handed to the cache writer; computed over every row
         the workload will ever write (prefix, histories, appended rows).
@@ -233,7 +235,8 @@ class DecodeWorkload:
             if k.size:
                 amax_k = np.maximum(amax_k, np.abs(k).max(axis=(0, 2)))
                 amax_v = np.maximum(amax_v, np.abs(v).max(axis=(0, 2)))
-        return (amax_k / np.float32(448.0)).astype(np.float32), (amax_v / np.float32(448.0)).astype(np.float32)
+        top = np.float32(FP8_MAX.get(self.cache_dtype, 448.0))
+        return (amax_k / top).astype(np.float32), (amax_v / top).astype(np.float32)
 
     # --------------------------------------------------------------- bytes
     def kv_bytes_read(self) -> int:
@@ -370,7 +373,7 @@ def prefix_sharing(seed: int = 3) -> DecodeWorkload:
 
 
 def quantized(cache_dtype: str = "int8", seed: int = 4) -> DecodeWorkload:
-    """Batch 256, 32 q / 8 KV heads, L ~ U[1024, 8192], int8 or fp8 cache, 1% K outliers x10."""
+    """Batch 256, 32 q / 8 KV heads, L ~ U[1024, 8192], a quantised cache, 1% K outliers x10."""
     lengths = _uniform_lengths(seed, 256, 1024, 8192)
     return make_workload(
         f"quantized_b256_32q8kv_d128_{cache_dtype}",
@@ -399,5 +402,7 @@ CONFIGS = {
     "prefix": prefix_sharing,
     "int8": lambda: quantized("int8"),
     "fp8": lambda: quantized("fp8_e4m3", seed=5),
+    "fp8_e5m2": lambda: quantized("fp8_e5m2", seed=6),
+    "int4": lambda: quantized("int4", seed=7),
     "window": sliding_window,
 }

@@ -21,9 +21,24 @@ TOL = {
     "bf16": (2e-2, 2e-3),
     "int8": (3e-2, 3e-3),
     "fp8_e4m3": (3e-2, 3e-3),
+    "fp8_e5m2": (3e-2, 3e-3),
+    "int4": (3e-2, 3e-3),
 }
 
-_TORCH_CACHE = {"f32": torch.float32, "bf16": torch.bfloat16, "int8": torch.int8, "fp8_e4m3": torch.uint8}
+_TORCH_CACHE = {"f32": torch.float32, "bf16": torch.bfloat16, "int8": torch.int8, "fp8_e4m3": torch.uint8,
+                "fp8_e5m2": torch.float8_e5m2, "int4": torch.uint8}
+FP8 = ("fp8_e4m3", "fp8_e5m2")
+ROW_SCALED = ("int8", "int4")
+
+
+def named(w):
+    """cache_dtype keyword for the binding: pools whose torch dtype does not name the format."""
+    return "int4" if w.cache_dtype == "int4" else None
+
+
+def row_width(w):
+    """Last dimension of a pool: head_dim values, or head_dim / 2 bytes for int4."""
+    return w.head_dim // 2 if w.cache_dtype == "int4" else w.head_dim
 _TORCH_ACT = {"f32": torch.float32, "bf16": torch.bfloat16}
 
 
@@ -41,7 +56,7 @@ class GpuState:
 
 
 def _poisoned_cache(w, device):
-    shape = (w.num_blocks, w.block_size, w.n_kv, w.head_dim)
+    shape = (w.num_blocks, w.block_size, w.n_kv, row_width(w))
     dt = _TORCH_CACHE[w.cache_dtype]
     if w.cache_dtype in ("f32", "bf16"):
         kc = torch.full(shape, float("nan"), dtype=dt, device=device)
@@ -49,9 +64,12 @@ def _poisoned_cache(w, device):
     elif w.cache_dtype == "int8":
         kc = torch.full(shape, 77, dtype=dt, device=device)
         vc = torch.full(shape, -77, dtype=dt, device=device)
+    elif w.cache_dtype == "int4":
+        kc = torch.full(shape, 0x77, dtype=dt, device=device)  # codes 7, 7
+        vc = torch.full(shape, 0x99, dtype=dt, device=device)  # codes -7, -7
     else:
-        kc = torch.full(shape, 0x7F, dtype=dt, device=device)  # E4M3 NaN code
-        vc = torch.full(shape, 0x7F, dtype=dt, device=device)
+        kc = torch.full(shape, 0x7F, dtype=torch.uint8, device=device).view(dt)  # a NaN code of both FP8 formats
+        vc = torch.full(shape, 0x7F, dtype=torch.uint8, device=device).view(dt)
     return kc, vc
 
 
@@ -70,10 +88,10 @@ def fill_gpu(w: workloads.DecodeWorkload, device="cuda", fp8_scales=None, chunk_
 
     kc, vc = _poisoned_cache(w, device)
     ks = vs = None
-    if w.cache_dtype == "int8":
+    if w.cache_dtype in ROW_SCALED:
         ks = torch.full((w.num_blocks, w.block_size, w.n_kv), float("nan"), dtype=torch.float32, device=device)
         vs = torch.full_like(ks, float("nan"))
-    elif w.cache_dtype == "fp8_e4m3":
+    elif w.cache_dtype in FP8:
         if fp8_scales is None:
             fp8_scales = w.fp8_head_scales()
         ks = torch.from_numpy(fp8_scales[0]).to(device)
@@ -84,7 +102,8 @@ def fill_gpu(w: workloads.DecodeWorkload, device="cuda", fp8_scales=None, chunk_
         if len(slots) == 0:
             return
         ops.kv_cache_write(_rows(k, w, device), _rows(v, w, device), kc, vc,
-                           torch.from_numpy(np.asarray(slots, dtype=np.int64)).to(device), ks, vs, err)
+                           torch.from_numpy(np.asarray(slots, dtype=np.int64)).to(device), ks, vs, err,
+                           cache_dtype=named(w))
 
     if w.shared_prefix_tokens:
         pk, pv = w.prefix_kv()
@@ -122,6 +141,7 @@ def run_decode(w, st: GpuState, tuning=None, workspace=None, block_tables=None):
     ops.paged_attention_decode(
         out, st.query, st.key_cache, st.value_cache, st.block_tables if block_tables is None else block_tables,
         st.context_lens, w.max_context_len, w.sm_scale, st.k_scale, st.v_scale, lse, workspace, st.device_error, tuning,
+        cache_dtype=named(w),
     )
     torch.cuda.synchronize()
     return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
@@ -137,11 +157,14 @@ def oracle_sequence(w, s, fp8_scales=None, window=0, sinks=0):
     """
     L = int(w.context_lens[s])
     nb = max(workloads.blocks_for(L, w.block_size), 1)
-    shape = (nb, w.block_size, w.n_kv, w.head_dim)
+    shape = (nb, w.block_size, w.n_kv, row_width(w))
     if w.cache_dtype == "int8":
         kc, vc = np.zeros(shape, np.int8), np.zeros(shape, np.int8)
         ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
-    elif w.cache_dtype == "fp8_e4m3":
+    elif w.cache_dtype == "int4":
+        kc, vc = np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+        ks, vs = np.zeros(shape[:3], np.float32), np.zeros(shape[:3], np.float32)
+    elif w.cache_dtype in FP8:
         kc, vc = np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
         ks, vs = fp8_scales if fp8_scales is not None else w.fp8_head_scales()
     else:
@@ -160,10 +183,13 @@ def gpu_sequence_rows(w, st: GpuState, s):
     L = int(w.context_lens[s])
     nb = workloads.blocks_for(L, w.block_size)
     blocks = torch.from_numpy(w.block_tables[s, :nb].astype(np.int64)).to(st.key_cache.device)
-    k = st.key_cache.index_select(0, blocks).reshape(-1, w.n_kv, w.head_dim)[:L]
-    v = st.value_cache.index_select(0, blocks).reshape(-1, w.n_kv, w.head_dim)[:L]
+    kc, vc = st.key_cache, st.value_cache
+    if kc.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
+        kc, vc = kc.view(torch.uint8), vc.view(torch.uint8)
+    k = kc.index_select(0, blocks).reshape(-1, w.n_kv, row_width(w))[:L]
+    v = vc.index_select(0, blocks).reshape(-1, w.n_kv, row_width(w))[:L]
     res = [k.cpu(), v.cpu()]
-    if w.cache_dtype == "int8":
+    if w.cache_dtype in ROW_SCALED:
         res += [st.k_scale.index_select(0, blocks).reshape(-1, w.n_kv)[:L].cpu(),
                 st.v_scale.index_select(0, blocks).reshape(-1, w.n_kv)[:L].cpu()]
     return res
@@ -174,8 +200,8 @@ def assert_rows_bit_exact(w, st, s, oracle_rows):
     kc, vc, ks, vs = oracle_rows
     L = int(w.context_lens[s])
     got = gpu_sequence_rows(w, st, s)
-    want_k = kc.reshape(-1, w.n_kv, w.head_dim)[:L]
-    want_v = vc.reshape(-1, w.n_kv, w.head_dim)[:L]
+    want_k = kc.reshape(-1, w.n_kv, row_width(w))[:L]
+    want_v = vc.reshape(-1, w.n_kv, row_width(w))[:L]
     if w.cache_dtype == "bf16":
         gk = got[0].view(torch.int16).numpy()
         wk = torch.from_numpy(want_k.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy()
@@ -188,7 +214,7 @@ def assert_rows_bit_exact(w, st, s, oracle_rows):
     else:
         assert np.array_equal(got[0].numpy().view(np.uint8), want_k.view(np.uint8))
         assert np.array_equal(got[1].numpy().view(np.uint8), want_v.view(np.uint8))
-        if w.cache_dtype == "int8":
+        if w.cache_dtype in ROW_SCALED:
             assert np.array_equal(got[2].numpy().view(np.int32), ks.reshape(-1, w.n_kv)[:L].view(np.int32))
             assert np.array_equal(got[3].numpy().view(np.int32), vs.reshape(-1, w.n_kv)[:L].view(np.int32))
 
@@ -219,6 +245,7 @@ def run_decode_step(w, st: GpuState, workspace=None):
     out = torch.full((w.num_seqs, w.n_q, w.head_dim), float("nan"), dtype=_TORCH_ACT[w.act_dtype], device=st.query.device)
     lse = torch.full((w.num_seqs, w.n_q), float("nan"), dtype=torch.float32, device=st.query.device)
     ops.paged_decode_step(out, st.query, k, v, st.key_cache, st.value_cache, st.block_tables, st.context_lens,
-                          w.max_context_len, w.sm_scale, st.k_scale, st.v_scale, lse, workspace, st.device_error)
+                          w.max_context_len, w.sm_scale, st.k_scale, st.v_scale, lse, workspace, st.device_error,
+                          cache_dtype=named(w))
     torch.cuda.synchronize()
     return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)

@@ -37,10 +37,12 @@ def _host(t):
     t = t.cpu()
     if t.dtype == torch.bfloat16:
         t = t.view(torch.int16)
+    elif t.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
+        t = t.view(torch.uint8)
     return t.numpy().copy()
 
 
-@pytest.mark.parametrize("cache", ["bf16", "int8", "fp8_e4m3", "f32"])
+@pytest.mark.parametrize("cache", ["bf16", "int8", "fp8_e4m3", "f32", "fp8_e5m2", "int4"])
 def test_copy_blocks_bit_exact(cache):
     ops = _ops()
     act = "f32" if cache == "f32" else "bf16"
@@ -48,14 +50,16 @@ def test_copy_blocks_bit_exact(cache):
                                 act_dtype=act, cache_dtype=cache, extra_blocks=20)
     st = fill_gpu(w)
     pairs = _pairs(w.num_blocks, 17, seed=9)
+    row_scaled = cache in ("int8", "int4")
     pools = [_host(st.key_cache), _host(st.value_cache)]
-    if cache == "int8":
+    if row_scaled:
         pools += [_host(st.k_scale), _host(st.v_scale)]
     oracle.copy_blocks(pools, pairs)
-    scales = (st.k_scale, st.v_scale) if cache == "int8" else (None, None)  # fp8 scales are per head, not per block
-    ops.copy_blocks(st.key_cache, st.value_cache, torch.from_numpy(pairs).cuda(), *scales, st.device_error)
+    scales = (st.k_scale, st.v_scale) if row_scaled else (None, None)  # fp8 scales are per head, not per block
+    ops.copy_blocks(st.key_cache, st.value_cache, torch.from_numpy(pairs).cuda(), *scales, st.device_error,
+                    cache_dtype="int4" if cache == "int4" else None)
     torch.cuda.synchronize()
-    got = [_host(st.key_cache), _host(st.value_cache)] + ([_host(st.k_scale), _host(st.v_scale)] if cache == "int8" else [])
+    got = [_host(st.key_cache), _host(st.value_cache)] + ([_host(st.k_scale), _host(st.v_scale)] if row_scaled else [])
     for g, want in zip(got, pools):
         assert np.array_equal(g.view(np.uint8), want.view(np.uint8))
     assert int(st.device_error.item()) == 0

@@ -28,6 +28,9 @@ CASES = [
     ([40, 17, 64, 5, 1, 16, 33, 700], 32, 8, 128, "bf16", "int8"),
     ([300, 129, 48, 1000], 64, 8, 128, "f32", "int8"),
     ([40, 17, 64, 5, 1, 16, 33, 700], 32, 8, 128, "bf16", "fp8_e4m3"),
+    ([40, 17, 64, 5, 1, 16, 33, 700], 32, 8, 128, "bf16", "fp8_e5m2"),
+    ([40, 17, 64, 5, 1, 16, 33, 700], 32, 8, 128, "bf16", "int4"),
+    ([300, 129, 48, 1000], 64, 8, 128, "f32", "int4"),
     ([40, 17, 64, 5, 0], 8, 2, 64, "f32", "f32"),
 ]
 

@@ -45,7 +45,8 @@ def check_all(w, st, out, lse, seqs=None, fp8_scales=None, rows=True):
 
 # ------------------------------------------------------------------ cache writer
 @pytest.mark.parametrize("act,cache", [("f32", "f32"), ("bf16", "bf16"), ("bf16", "int8"), ("f32", "int8"),
-                                       ("bf16", "fp8_e4m3"), ("f32", "fp8_e4m3")])
+                                       ("bf16", "fp8_e4m3"), ("f32", "fp8_e4m3"), ("bf16", "fp8_e5m2"),
+                                       ("f32", "fp8_e5m2"), ("bf16", "int4"), ("f32", "int4")])
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_cache_write_bit_exact(act, cache, d):
     w = _wl([40, 17, 64, 5, 33], 8, 2, d, act, cache, seed=d, outlier_fraction=0.02 if cache != "f32" else 0.0)
@@ -62,8 +63,10 @@ def test_cache_write_bit_exact(act, cache, d):
         assert torch.isnan(kc.float()).all()
     elif cache == "int8":
         assert (kc == 77).all()
+    elif cache == "int4":
+        assert (kc == 0x77).all()
     else:
-        assert (kc == 0x7F).all()
+        assert (kc.view(torch.uint8) == 0x7F).all()
 
 
 def test_cache_write_skip_and_range_flag():
@@ -115,7 +118,7 @@ def test_decode_bf16_shapes(shape):
 
 
 @pytest.mark.parametrize("shape", [([40, 17, 64, 5, 1, 16, 33, 700], 32, 8, 128), ([300, 129, 48, 1000], 64, 8, 128)])
-@pytest.mark.parametrize("cache", ["int8", "fp8_e4m3"])
+@pytest.mark.parametrize("cache", ["int8", "fp8_e4m3", "fp8_e5m2", "int4"])
 def test_decode_quantized_shapes(shape, cache):
     lengths, n_q, n_kv, d = shape
     w = _wl(lengths, n_q, n_kv, d, cache=cache, seed=7, outlier_fraction=0.01)
@@ -250,10 +253,10 @@ def test_prefix_sharing_config():
     assert int(st.device_error.item()) == 0
 
 
-@pytest.mark.parametrize("cache", ["int8", "fp8_e4m3"])
+@pytest.mark.parametrize("cache", ["int8", "fp8_e4m3", "fp8_e5m2", "int4"])
 def test_quantized_config_sampled(cache):
-    w = workloads.quantized(cache, seed=4 if cache == "int8" else 5)
-    scales = w.fp8_head_scales() if cache == "fp8_e4m3" else None
+    w = workloads.quantized(cache, seed={"int8": 4, "fp8_e4m3": 5, "fp8_e5m2": 6, "int4": 7}[cache])
+    scales = w.fp8_head_scales() if cache.startswith("fp8") else None
     st = fill_gpu(w, fp8_scales=scales)
     out, lse = run_decode(w, st)
     errs = check_all(w, st, out, lse, seqs=range(0, 256, 37), fp8_scales=scales)
@@ -267,3 +270,14 @@ def test_quantized_config_sampled(cache):
     qerr = np.abs(out[0] - sdpa_reference(q[0], K, V, w.sm_scale)).max()
     print(f"{cache}: max/mean abs err vs dequantised oracle {max(e[0] for e in errs):.3e}/{np.mean([e[1] for e in errs]):.3e}; "
           f"vs unquantised seq 0 {qerr:.3e}")
+
+
+@pytest.mark.parametrize("cache", ["int8", "fp8_e4m3", "fp8_e5m2", "int4"])
+def test_decode_quantized_f32_queries(cache):
+    """float32 queries and outputs over a quantised cache (queries rounded to
+    f16 for the tensor cores: the quantised tolerance covers it)."""
+    w = _wl([40, 17, 64, 5, 1, 300], 32, 8, 128, act="f32", cache=cache, seed=8, outlier_fraction=0.01)
+    st = fill_gpu(w)
+    out, lse = run_decode(w, st)
+    check_all(w, st, out, lse, fp8_scales=st.fp8_scales)
+    assert int(st.device_error.item()) == 0
