@@ -326,9 +326,10 @@ def run_b200(args, rank, world, local):
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
     shape = (w.num_blocks, bs, nkv, d)
     # q/K/V ~ N(0,1) synthetic cache, filled on the device (the writer is exercised by the step's append)
-    if w.cache_dtype == "bf16":
-        kc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
-        vc = torch.randn(shape, device=dev, generator=gen).to(torch.bfloat16)
+    act = torch.float32 if w.act_dtype == "f32" else torch.bfloat16
+    if w.cache_dtype in ("bf16", "f32"):
+        kc = torch.randn(shape, device=dev, generator=gen).to(act)
+        vc = torch.randn(shape, device=dev, generator=gen).to(act)
         ks = vs = None
     else:
         pool_dtype = {"int8": torch.int8, "fp8_e4m3": torch.uint8, "fp8_e5m2": torch.float8_e5m2,
@@ -349,9 +350,9 @@ def run_b200(args, rank, world, local):
             kk = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
             vv = torch.randn((sl.numel(), nkv, d), device=dev, generator=gen).to(torch.bfloat16)
             ops.kv_cache_write(kk, vv, kc, vc, sl, ks, vs, cache_dtype=named)
-    q = torch.randn((S, nq, d), device=dev, generator=gen).to(torch.bfloat16)
-    k_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
-    v_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    q = torch.randn((S, nq, d), device=dev, generator=gen).to(act)
+    k_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(act)
+    v_new = torch.randn((S, nkv, d), device=dev, generator=gen).to(act)
     slots = torch.from_numpy(w.new_token_slots()).to(dev)
     bt = torch.from_numpy(w.block_tables).to(dev)
     cl = torch.from_numpy(w.context_lens).to(dev)
@@ -497,8 +498,10 @@ def run_b200(args, rank, world, local):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": traffic,
-                "kernel": "decode_tc_kernel + decode_merge_kernel (pkv_paged_attention_decode)" if args.unfused
-                else "decode_tc_kernel with fused append + decode_merge_kernel (pkv_paged_decode_step)",
+                "kernel": ("decode_f32_kernel" if w.cache_dtype == "f32" else "decode_tc_kernel")
+                + (" + decode_merge_kernel (pkv_paged_attention_decode)" if args.unfused and w.cache_dtype != "f32"
+                   else " with fused append" + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
+                   + " (pkv_paged_decode_step)" if not args.unfused else " (pkv_paged_attention_decode)"),
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "bytes_per_launch": kv_bytes,
                 "launch_ms": att_ms,

@@ -703,14 +703,16 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const uint32_t z0 = prmt((&x0.x)[wi], (&y0.x)[wi], sel) ^ 0x88888888u;
         const uint32_t z1 = prmt((&x1.x)[wi], (&y1.x)[wi], sel) ^ 0x88888888u;
         uint32_t af[4];
-        af[0] = i4x2_to_f16x2(z0) & mlo;
-        af[1] = i4x2_to_f16x2(z0 >> 4) & mlo;
-        af[2] = i4x2_to_f16x2(z1) & mhi;
-        af[3] = i4x2_to_f16x2(z1 >> 4) & mhi;
+        // codes are finite and masked tokens carry P = 0: no V mask needed
+        af[0] = i4x2_to_f16x2(z0);
+        af[1] = i4x2_to_f16x2(z0 >> 4);
+        af[2] = i4x2_to_f16x2(z1);
+        af[3] = i4x2_to_f16x2(z1 >> 4);
         mma_f16(acc[mt], af, pb0, pb1);
       }
     } else {
       // lane (g, c) reads chunk g of token rows 2c, 2c+1, 2c+8, 2c+9
+      const uint32_t mlo5 = mlo & 0xFF00FF00u, mhi5 = mhi & 0xFF00FF00u;
       const uint4 x0 = lds128(vt + voff);
       const uint4 y0 = lds128(vt + (voff ^ 16) + 128);
       const uint4 x1 = lds128(vt + voff + 1024);
@@ -736,16 +738,20 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           af[1] = prmt((&x0.x)[wi], (&y0.x)[wi], s1);
           af[2] = prmt((&x1.x)[wi], (&y1.x)[wi], s0);
           af[3] = prmt((&x1.x)[wi], (&y1.x)[wi], s1);
+          if constexpr (CACHE == TC_FP8) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            if constexpr (CACHE == TC_FP8) af[k] = e4m3x2_hi_to_f16x2_div256(af[k]);
-            else af[k] &= 0xFF00FF00u;  // E5M2 bytes are the f16 top bytes; clear the duplicated low bytes
+            for (int k = 0; k < 4; ++k) af[k] = e4m3x2_hi_to_f16x2_div256(af[k]);
+          } else {
+            // E5M2 bytes are the f16 top bytes: clear the duplicated low bytes, and
+            // the rows past the attended ones (their codes may be inf or NaN)
+            af[0] &= mlo5;
+            af[1] &= mlo5;
+            af[2] &= mhi5;
+            af[3] &= mhi5;
           }
         }
-        af[0] &= mlo;
-        af[1] &= mlo;
-        af[2] &= mhi;
-        af[3] &= mhi;
+        // INT8 and E4M3 values decode finite whatever the bytes, and masked
+        // tokens carry P = 0, so they need no V mask
         mma_f16(acc[mt], af, pb0, pb1);
       }
     }
