@@ -370,8 +370,26 @@ def run_b200(args, rank, world, local):
     if w.window:
         args.unfused = True  # the windowed decode has no fused-append entry point
 
+    prefix_blocks = w.shared_prefix_tokens // bs
+    if prefix_blocks:
+        # the shared prefix is attended once for all sequences, then each sequence's own blocks
+        nws = max(nws, ops.shared_prefix_workspace_size(S, nq, nkv, d, bs, prefix_blocks))
+        ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
+
+    def fused(out, q, k_new, v_new, bt, cl, tun):
+        if prefix_blocks:
+            ops.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, cl, w.max_context_len, prefix_blocks,
+                                                     key=k_new, value=v_new, sm_scale=w.sm_scale, workspace=ws,
+                                                     device_error=err)
+        else:
+            ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
+                                  workspace=ws, device_error=err, tuning=tun, cache_dtype=named)
+
     def decode(out, q, bt, cl):
-        if w.window:
+        if prefix_blocks:
+            ops.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, cl, w.max_context_len, prefix_blocks,
+                                                     sm_scale=w.sm_scale, workspace=ws, device_error=err)
+        elif w.window:
             ops.paged_attention_decode_window(out, q, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
                                               w.sm_scale, ks, vs, workspace=ws, device_error=err, cache_dtype=named)
         else:
@@ -383,8 +401,7 @@ def run_b200(args, rank, world, local):
             ops.kv_cache_write(k_new, v_new, kc, vc, slots, ks, vs, err, cache_dtype=named)
             decode(out, q, bt, cl)
         else:
-            ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err, tuning=tuning if overlap else None, cache_dtype=named)
+            fused(out, q, k_new, v_new, bt, cl, tuning if overlap else None)
 
     def barrier():
         if world > 1:
@@ -419,8 +436,7 @@ def run_b200(args, rank, world, local):
             decode(out, q, bt, cl)
             att[k][1].record(stream)
         else:
-            ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
-                                  workspace=ws, device_error=err, tuning=tuning, cache_dtype=named)
+            fused(out, q, k_new, v_new, bt, cl, tuning)
     ev_end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -498,18 +514,21 @@ def run_b200(args, rank, world, local):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": traffic,
-                "kernel": ("decode_f32_kernel" if w.cache_dtype == "f32" else "decode_tc_kernel")
-                + (" + decode_merge_kernel (pkv_paged_attention_decode)" if args.unfused and w.cache_dtype != "f32"
-                   else " with fused append" + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
-                   + " (pkv_paged_decode_step)" if not args.unfused else " (pkv_paged_attention_decode)"),
+                "kernel": ("prefix_attn_kernel + " if prefix_blocks else "")
+                + ("decode_f32_kernel" if w.cache_dtype == "f32" else "decode_tc_kernel")
+                + ("" if args.unfused else " with fused append")
+                + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
+                + (" (pkv_paged_attention_decode_shared_prefix)" if prefix_blocks
+                   else " (pkv_paged_attention_decode)" if args.unfused else " (pkv_paged_decode_step)"),
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "bytes_per_launch": kv_bytes,
                 "launch_ms": att_ms,
             },
             "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
-            # decode kernel + merge of split sequences (+ the cache write when unfused)
-            "gpu_launches": ((1 if w.cache_dtype == "f32" else 2) + (1 if args.unfused else 0)) * args.steps,
+            # decode kernel + merge of split sequences (+ the prefix pass, + the cache write when unfused)
+            "gpu_launches": ((1 if w.cache_dtype == "f32" else 2) + (1 if prefix_blocks else 0)
+                             + (1 if args.unfused else 0)) * args.steps,
             "step": ("append, then decode + merge of split sequences" if args.unfused
                      else "append fused into the decode kernel, then the merge of split sequences")
             + ("" if args.no_overlap or args.unfused else "; prologue overlaps the previous step (programmatic launch)"),

@@ -191,6 +191,38 @@ pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const
                                              size_t workspace_bytes, int32_t* device_error, void* stream);
 
 /*
+ * Decode for a batch whose sequences all begin with the same physical blocks:
+ * a shared prompt prefix stored once ("Chapter 18 - KV-Cache Optimization
+ * Strategies", Prefix Caching; "KV Cache Engineering for LLM Serving", section
+ * 11).  The first prefix_blocks entries of every block table must name the same
+ * blocks (the caller's contract, as for shared blocks in general; row 0's are
+ * the ones read).  The prefix is attended once per KV head for the queries of
+ * all sequences together (a dense tensor-core pass), and each sequence's own
+ * positions [prefix_blocks * block_size, L) are attended starting from that
+ * state, so the result equals pkv_paged_attention_decode's.
+ *
+ *   key, value        optional new rows [num_seqs, n_kv, head_dim] (act dtype):
+ *                     appended as token L-1 first, as in pkv_paged_decode_step;
+ *                     NULL for a plain decode
+ *   prefix_blocks     >= 1; every context length must exceed prefix_blocks *
+ *                     block_size (else PKV_DEVERR_CONTEXT_LEN and undefined output)
+ *   workspace         pkv_shared_prefix_workspace_size bytes
+ * BF16 cache and activations, head_dim 64 or 128.  Three launches on `stream`
+ * (prefix pass, decode, merge), each queued behind the previous one with
+ * programmatic serialisation.
+ */
+size_t pkv_shared_prefix_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                        int prefix_blocks);
+pkv_status pkv_paged_attention_decode_shared_prefix(void* out, const void* query, const void* key, const void* value,
+                                                    void* key_cache, void* value_cache, const int32_t* block_tables,
+                                                    int max_blocks_per_seq, const int32_t* context_lens,
+                                                    int max_context_len, int num_seqs, int n_q, int n_kv,
+                                                    int head_dim, int block_size, int64_t num_blocks, float sm_scale,
+                                                    int prefix_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                                    float* lse_out, void* workspace, size_t workspace_bytes,
+                                                    int32_t* device_error, void* stream);
+
+/*
  * Quest, query-aware sparse reads ("KV Cache Engineering for LLM Serving",
  * section 7).  A page is one cache block.  Each page keeps the element-wise
  * minimum and maximum of its keys; a query scores a page by

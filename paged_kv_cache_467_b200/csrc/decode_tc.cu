@@ -66,6 +66,12 @@ struct TcParams {
   // past the count) to read instead of every block; one KV head per unit
   const int32_t* pages;
   int k_pages;
+  // shared-prefix decode: logical blocks < skip_blocks were attended by the
+  // prefix pass; the piece holding a unit's first block starts from its state
+  int skip_blocks;
+  const float* pre_o;    // [n_kv][rows][pre_splits][D]
+  const float* pre_lse;  // [n_kv][rows][pre_splits], base 2
+  int pre_splits, pre_rows;
   int G, QC, HPC, HG, NCW, stages, units;
   float scale_log2;
   int act_bf16;
@@ -108,6 +114,14 @@ __device__ __forceinline__ AttendSet attend_set(const TcParams& p, int L) {
   a.nb = a.sink_blocks = a.win_first = nbl;
   a.s_eff = L;
   a.lo_w = 0;
+  if (p.skip_blocks > 0) {  // positions [skip_blocks * 16, L) only
+    a.s_eff = 0;
+    a.sink_blocks = 0;
+    a.win_first = min(p.skip_blocks, nbl);
+    a.lo_w = min(p.skip_blocks * kBlockSize, L);
+    a.nb = nbl - a.win_first;
+    return a;
+  }
   if (p.window > 0 && L > p.window) {
     a.lo_w = L - p.window;
     a.s_eff = min(p.sinks, L);
@@ -898,6 +912,40 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
+      if (p.pre_o != nullptr && j == 0) {
+        // the piece holding the unit's first block starts from the shared-prefix
+        // state of this lane's heads 2c, 2c+1: combined over the prefix splits
+        // (M = max lse_i, w_i = 2^(lse_i - M)); l is counted on lane g == 0 only
+        const int kvh = hg * p.HPC + head_local;
+        const int hq = qc * 8 + 2 * c;  // head of the group
+        const size_t r0 = (size_t)kvh * p.pre_rows + (size_t)s * p.G + hq;
+        float w0 = 0.f, w1 = 0.f;
+        if (head0_ok) {
+          for (int k = 0; k < p.pre_splits; ++k) m0 = fmaxf(m0, __ldcg(p.pre_lse + r0 * p.pre_splits + k));
+        }
+        if (head1_ok) {
+          for (int k = 0; k < p.pre_splits; ++k) m1 = fmaxf(m1, __ldcg(p.pre_lse + (r0 + 1) * p.pre_splits + k));
+        }
+        for (int k = 0; k < p.pre_splits; ++k) {
+          const float e0 = head0_ok ? ex2(__ldcg(p.pre_lse + r0 * p.pre_splits + k) - m0) : 0.f;
+          const float e1 = head1_ok ? ex2(__ldcg(p.pre_lse + (r0 + 1) * p.pre_splits + k) - m1) : 0.f;
+          w0 += e0;
+          w1 += e1;
+          const float* o0 = p.pre_o + (r0 * p.pre_splits + k) * D;
+          const float* o1 = p.pre_o + ((r0 + 1) * p.pre_splits + k) * D;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+            for (int hi = 0; hi < 2; ++hi) {
+              const int dd = d_of<CACHE, D>(mt, hi, g);
+              if (head0_ok) acc[mt][2 * hi] += e0 * __ldcg(o0 + dd);
+              if (head1_ok) acc[mt][2 * hi + 1] += e1 * __ldcg(o1 + dd);
+            }
+          }
+        }
+        l0 = g == 0 ? w0 : 0.f;
+        l1 = g == 0 ? w1 : 0.f;
+      }
     }
 
     const int uend = P[u + 1];
@@ -992,7 +1040,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // Rank-3 view of a pool: (elements of one chunk, chunk index, token row).  A
 // chunk is 128 bytes (BF16 / INT8 / FP8 rows), or a whole 64-byte INT4 head row
 // (64-byte swizzle).
-static pkv_status make_kv_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes_i,
+pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes_i,
                               int64_t rows) {
   auto fn = encode_fn();
   if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
@@ -1079,10 +1127,18 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   const int chunk_bytes = int4 ? s.head_dim / 2 : 128;
   const int64_t rows = a.num_blocks * kBlockSize;
   CUtensorMap km, vm;
-  pkv_status st = make_kv_map(&km, a.key_cache, elem, chunk_bytes, row_bytes, rows);
+  pkv_status st = make_pool_map(&km, a.key_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
-  st = make_kv_map(&vm, a.value_cache, elem, chunk_bytes, row_bytes, rows);
+  st = make_pool_map(&vm, a.value_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
+  PrefixState pre = a.prefix;
+  if (a.skip_blocks > 0 && a.prefix_ws) {
+    // shared prefix first; the decode over the sequences' own blocks then
+    // starts from its state (queued with programmatic serialisation)
+    st = launch_prefix(s, km, vm, a.query, a.block_tables, a.num_blocks, a.skip_blocks, a.sm_scale, a.prefix_ws,
+                       a.device_error, &pre, stream);
+    if (st != PKV_OK) return st;
+  }
 
   TcParams prm;
   prm.out = a.out;
@@ -1112,6 +1168,11 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.sinks = a.sinks;
   prm.pages = a.pages;
   prm.k_pages = a.k_pages;
+  prm.skip_blocks = a.skip_blocks;
+  prm.pre_o = pre.o;
+  prm.pre_lse = pre.lse;
+  prm.pre_splits = pre.splits;
+  prm.pre_rows = pre.rows;
   prm.G = plan.G;
   prm.QC = plan.QC;
   prm.HPC = plan.HPC;

@@ -1,6 +1,7 @@
 // Host-side declarations shared by the .cu files of libpkv (not installed).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -43,6 +44,17 @@ struct TcPlan {
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
 
+// Shared-prefix pass (prefix.cu): per (KV head, query row = s * G + head in
+// group, split) a normalised partial output and its base-2 lse, which the
+// decode kernel over each sequence's own blocks starts from.
+constexpr int kMaxPrefixSplits = 64;
+struct PrefixState {
+  const float* o = nullptr;    // [n_kv][rows][splits][head_dim]
+  const float* lse = nullptr;  // [n_kv][rows][splits]
+  int splits = 0;
+  int rows = 0;
+};
+
 struct TcArgs {
   void* out;
   const void* query;
@@ -69,9 +81,20 @@ struct TcArgs {
   // Quest decode only: [num_seqs, n_kv, k_pages] logical pages to read
   const int32_t* pages = nullptr;
   int k_pages = 0;
+  // shared-prefix decode only: the first skip_blocks logical blocks of every
+  // sequence were attended by the prefix pass, whose state each unit starts from
+  int skip_blocks = 0;
+  PrefixState prefix;
+  void* prefix_ws = nullptr;  // scratch of the prefix pass (prefix_workspace_bytes)
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);
+
+size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks);
+pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes, int64_t rows);
+pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const void* query,
+                         const int32_t* block_tables, int64_t num_blocks, int prefix_blocks, float sm_scale,
+                         void* prefix_ws, int32_t* device_error, PrefixState* state, cudaStream_t stream);
 
 pkv_status launch_decode_f32(const DecodeShape& s, const TcArgs& a, cudaStream_t stream);
 

@@ -87,6 +87,11 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attention_decode_pages_ex.argtypes = (lib.pkv_paged_attention_decode_pages.argtypes[:-1]
                                                         + [ctypes.POINTER(DecodeTuning), vp])
     lib.pkv_paged_attention_decode_pages_ex.restype = i32
+    lib.pkv_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.pkv_shared_prefix_workspace_size.restype = sz
+    lib.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
+                                                             i32, i32, i64, f32, i32, i32, i32, vp, vp, sz, vp, vp]
+    lib.pkv_paged_attention_decode_shared_prefix.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_cuda_error.argtypes = []
@@ -372,4 +377,35 @@ def paged_attention_decode_pages(out, query, key_cache, value_cache, block_table
     else:
         st = lib.pkv_paged_attention_decode_pages_ex(*args, ctypes.byref(tuning), _stream(query.device))
     _check(st, "pkv_paged_attention_decode_pages")
+    return out
+
+
+def shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks) -> int:
+    n = lib.pkv_shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks)
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(2, "pkv_shared_prefix_workspace_size")
+    return int(n)
+
+
+def paged_attention_decode_shared_prefix(out, query, key_cache, value_cache, block_tables, context_lens,
+                                         max_context_len: int, prefix_blocks: int, key=None, value=None,
+                                         sm_scale: float | None = None, lse_out=None, workspace=None,
+                                         device_error=None):
+    """Decode with the first ``prefix_blocks`` blocks shared by every sequence: one dense pass over the
+    prefix for all queries, then each sequence's own blocks; ``key``/``value`` append token L-1 first."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = shared_prefix_workspace_size(S, n_q, n_kv, d, block_size, prefix_blocks)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.pkv_paged_attention_decode_shared_prefix(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+        block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
+        float(sm_scale), int(prefix_blocks), act_code(query), cache_code(key_cache), _ptr(lse_out), _ptr(workspace),
+        ws_bytes, _ptr(device_error), _stream(query.device),
+    )
+    _check(st, "pkv_paged_attention_decode_shared_prefix")
     return out
