@@ -69,9 +69,9 @@ struct TcParams {
   // shared-prefix decode: logical blocks < skip_blocks were attended by the
   // prefix pass; the piece holding a unit's first block starts from its state
   int skip_blocks;
-  const float* pre_o;    // [n_kv][rows][pre_splits][D]
-  const float* pre_lse;  // [n_kv][rows][pre_splits], base 2
-  int pre_splits, pre_rows;
+  const float* pre_o;    // [n_kv][rows][D], normalised
+  const float* pre_lse;  // [n_kv][rows], base 2
+  int pre_rows;
   int G, QC, HPC, HG, NCW, stages, units;
   float scale_log2;
   int act_bf16;
@@ -914,37 +914,24 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       l0 = l1 = 0.f;
       if (p.pre_o != nullptr && j == 0) {
         // the piece holding the unit's first block starts from the shared-prefix
-        // state of this lane's heads 2c, 2c+1: combined over the prefix splits
-        // (M = max lse_i, w_i = 2^(lse_i - M)); l is counted on lane g == 0 only
+        // state (normalised o, base-2 lse) of this lane's heads 2c, 2c+1: m = lse,
+        // acc = o, l = 1, the sum counted on lane g == 0 only
         const int kvh = hg * p.HPC + head_local;
-        const int hq = qc * 8 + 2 * c;  // head of the group
-        const size_t r0 = (size_t)kvh * p.pre_rows + (size_t)s * p.G + hq;
-        float w0 = 0.f, w1 = 0.f;
-        if (head0_ok) {
-          for (int k = 0; k < p.pre_splits; ++k) m0 = fmaxf(m0, __ldcg(p.pre_lse + r0 * p.pre_splits + k));
-        }
-        if (head1_ok) {
-          for (int k = 0; k < p.pre_splits; ++k) m1 = fmaxf(m1, __ldcg(p.pre_lse + (r0 + 1) * p.pre_splits + k));
-        }
-        for (int k = 0; k < p.pre_splits; ++k) {
-          const float e0 = head0_ok ? ex2(__ldcg(p.pre_lse + r0 * p.pre_splits + k) - m0) : 0.f;
-          const float e1 = head1_ok ? ex2(__ldcg(p.pre_lse + (r0 + 1) * p.pre_splits + k) - m1) : 0.f;
-          w0 += e0;
-          w1 += e1;
-          const float* o0 = p.pre_o + (r0 * p.pre_splits + k) * D;
-          const float* o1 = p.pre_o + ((r0 + 1) * p.pre_splits + k) * D;
+        const size_t r0 = (size_t)kvh * p.pre_rows + (size_t)s * p.G + qc * 8 + 2 * c;
+        const float* o0 = p.pre_o + r0 * D;
 #pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
+        for (int mt = 0; mt < KS; ++mt) {
 #pragma unroll
-            for (int hi = 0; hi < 2; ++hi) {
-              const int dd = d_of<CACHE, D>(mt, hi, g);
-              if (head0_ok) acc[mt][2 * hi] += e0 * __ldcg(o0 + dd);
-              if (head1_ok) acc[mt][2 * hi + 1] += e1 * __ldcg(o1 + dd);
-            }
+          for (int hi = 0; hi < 2; ++hi) {
+            const int dd = d_of<CACHE, D>(mt, hi, g);
+            if (head0_ok) acc[mt][2 * hi] = __ldcg(o0 + dd);
+            if (head1_ok) acc[mt][2 * hi + 1] = __ldcg(o0 + D + dd);
           }
         }
-        l0 = g == 0 ? w0 : 0.f;
-        l1 = g == 0 ? w1 : 0.f;
+        if (head0_ok) m0 = __ldcg(p.pre_lse + r0);
+        if (head1_ok) m1 = __ldcg(p.pre_lse + r0 + 1);
+        l0 = (g == 0 && head0_ok) ? 1.f : 0.f;
+        l1 = (g == 0 && head1_ok) ? 1.f : 0.f;
       }
     }
 
@@ -1171,7 +1158,6 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.skip_blocks = a.skip_blocks;
   prm.pre_o = pre.o;
   prm.pre_lse = pre.lse;
-  prm.pre_splits = pre.splits;
   prm.pre_rows = pre.rows;
   prm.G = plan.G;
   prm.QC = plan.QC;

@@ -45,13 +45,14 @@ struct TcPlan {
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
 
 // Shared-prefix pass (prefix.cu): per (KV head, query row = s * G + head in
-// group, split) a normalised partial output and its base-2 lse, which the
-// decode kernel over each sequence's own blocks starts from.
+// group) the normalised output over the prefix and its base-2 lse (the
+// prefix's splits already combined), which the decode kernel over each
+// sequence's own blocks starts from.
 constexpr int kMaxPrefixSplits = 64;
 struct PrefixState {
-  const float* o = nullptr;    // [n_kv][rows][splits][head_dim]
-  const float* lse = nullptr;  // [n_kv][rows][splits]
-  int splits = 0;
+  const float* o = nullptr;    // [n_kv][rows][head_dim]
+  const float* lse = nullptr;  // [n_kv][rows]
+  int splits = 0;              // splits of the prefix pass (combined into o / lse)
   int rows = 0;
 };
 

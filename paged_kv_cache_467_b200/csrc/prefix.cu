@@ -5,10 +5,11 @@
 // per KV head for the queries of all sequences together: the scores are a
 // dense [S*G x 16] x [16 x d] product per block instead of S separate
 // [G x 16] ones, and the prefix is read once per query tile instead of once
-// per sequence.  The result is a normalised partial output and its base-2
-// log-sum-exp per (query row, split of the prefix); the decode kernel over
-// each sequence's own blocks starts from it (softmax states merge exactly:
-// M = max lse_i, o = sum 2^(lse_i - M) o_i / sum 2^(lse_i - M)).
+// per sequence.  The pass is split along the prefix; each split leaves a
+// normalised partial output and its base-2 log-sum-exp per query row, a small
+// second launch combines the splits (softmax states merge exactly:
+// M = max lse_i, o = sum 2^(lse_i - M) o_i / sum 2^(lse_i - M)), and the
+// decode kernel over each sequence's own blocks starts from that state.
 //
 // CTA = 4 warps x 16 query rows of one KV head, one split of the prefix.  Q
 // fragments stay in registers; K and V blocks come through a ring of TMA
@@ -151,21 +152,27 @@ __global__ void __launch_bounds__(kPrefixWarps * 32) prefix_attn_kernel(const __
     mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
     mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
     mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-    const float al_a = ex2f(m_a - mn_a), al_b = ex2f(m_b - mn_b);
-    m_a = mn_a;
-    m_b = mn_b;
+    // lazy rescale: the reference max moves (and the accumulators are
+    // rescaled) only when a score exceeds it by more than 2^8, so P <= 2^8
+    if (__any_sync(0xffffffffu, mx_a > m_a + 8.f || mx_b > m_b + 8.f)) {
+      const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+      const float al_a = ex2f(m_a - mn_a), al_b = ex2f(m_b - mn_b);
+      m_a = mn_a;
+      m_b = mn_b;
+      l_a *= al_a;
+      l_b *= al_b;
+#pragma unroll
+      for (int dt = 0; dt < D / 8; ++dt) {
+        o[dt][0] *= al_a;
+        o[dt][1] *= al_a;
+        o[dt][2] *= al_b;
+        o[dt][3] *= al_b;
+      }
+    }
     float pa[4] = {ex2f(s0[0] - m_a), ex2f(s0[1] - m_a), ex2f(s1[0] - m_a), ex2f(s1[1] - m_a)};
     float pb[4] = {ex2f(s0[2] - m_b), ex2f(s0[3] - m_b), ex2f(s1[2] - m_b), ex2f(s1[3] - m_b)};
-    l_a = l_a * al_a + (pa[0] + pa[1] + pa[2] + pa[3]);
-    l_b = l_b * al_b + (pb[0] + pb[1] + pb[2] + pb[3]);
-#pragma unroll
-    for (int dt = 0; dt < D / 8; ++dt) {
-      o[dt][0] *= al_a;
-      o[dt][1] *= al_a;
-      o[dt][2] *= al_b;
-      o[dt][3] *= al_b;
-    }
+    l_a += (pa[0] + pa[1] + pa[2] + pa[3]);
+    l_b += (pb[0] + pb[1] + pb[2] + pb[3]);
     // P as the A operand: (row g, tokens 2c, 2c+1), (row g+8, ...), (row g, 2c+8, 2c+9), (row g+8, ...)
     uint32_t pf[4] = {pack_bf16(pa[0], pa[1]), pack_bf16(pb[0], pb[1]), pack_bf16(pa[2], pa[3]),
                       pack_bf16(pb[2], pb[3])};
@@ -216,24 +223,68 @@ __global__ void __launch_bounds__(kPrefixWarps * 32) prefix_attn_kernel(const __
   }
 }
 
-// Splits of the prefix so that the grid covers the GPU about twice, each split
-// at least 4 blocks long.
+// Splits of the prefix so that about four CTAs run on every SM (the pass is
+// latency-bound: more resident warps hide more of each block's MMA and
+// softmax chain), each split at least 4 blocks long.
 static void prefix_grid(int rows, int n_kv, int prefix_blocks, int* splits, int* per_split) {
   const int tiles = (rows + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
-  const int want = std::max(1, (2 * std::max(1, device_sm_count())) / std::max(1, tiles * n_kv));
+  const int want = std::max(1, (4 * std::max(1, device_sm_count())) / std::max(1, tiles * n_kv));
   int sp = std::max(1, std::min(want, prefix_blocks / 4));
   sp = std::min(sp, kMaxPrefixSplits);
   *per_split = (prefix_blocks + sp - 1) / sp;
   *splits = (prefix_blocks + *per_split - 1) / *per_split;
 }
 
+// The splits' states combined per (KV head, query row): one CTA of 256 threads
+// per 8 rows, a thread per (row, 4 dims), the splits' loads independent.
+struct CombineParams {
+  const float* part_o;
+  const float* part_lse;
+  float* o;    // [n_kv * rows][D]
+  float* lse;  // [n_kv * rows]
+  int total_rows, splits;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) prefix_combine_kernel(const CombineParams p) {
+  grid_launch_dependents();
+  grid_wait_prerequisites();
+  constexpr int V = D / 4;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const int r = idx / V, v = idx - r * V;
+  if (r >= p.total_rows) return;
+  const float* lse = p.part_lse + (size_t)r * p.splits;
+  float M = -INFINITY;
+#pragma unroll 8
+  for (int k = 0; k < p.splits; ++k) M = fmaxf(M, __ldcg(lse + k));
+  float wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int k = 0; k < p.splits; ++k) {
+    const float w = ex2f(__ldcg(lse + k) - M);
+    const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((size_t)r * p.splits + k) * D) + v);
+    wsum += w;
+    acc.x += w * o.x;
+    acc.y += w * o.y;
+    acc.z += w * o.z;
+    acc.w += w * o.w;
+  }
+  const float inv = 1.f / wsum;
+  reinterpret_cast<float4*>(p.o + (size_t)r * D)[v] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (v == 0) p.lse[r] = M + log2f(wsum);
+}
+
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
 size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks) {
   const int rows = num_seqs * (n_q / n_kv);
   int splits = 1, per = 1;
   prefix_grid(rows, n_kv, prefix_blocks, &splits, &per);
-  const size_t o = (size_t)n_kv * rows * splits * head_dim * 4;
-  const size_t l = (size_t)n_kv * rows * splits * 4;
-  return (o + 255) / 256 * 256 + (l + 255) / 256 * 256;
+  const size_t part_o = (size_t)n_kv * rows * splits * head_dim * 4;
+  const size_t part_l = (size_t)n_kv * rows * splits * 4;
+  const size_t o = (size_t)n_kv * rows * head_dim * 4;
+  const size_t l = (size_t)n_kv * rows * 4;
+  return align256(part_o) + align256(part_l) + align256(o) + align256(l);
 }
 
 pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const void* query,
@@ -252,11 +303,21 @@ pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUte
   p.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
   prefix_grid(p.rows, s.n_kv, prefix_blocks, &p.splits, &p.per_split);
   uint8_t* ws = static_cast<uint8_t*>(prefix_ws);
+  const size_t part_o = align256((size_t)s.n_kv * p.rows * p.splits * s.head_dim * 4);
+  const size_t part_l = align256((size_t)s.n_kv * p.rows * p.splits * 4);
+  const size_t comb_o = align256((size_t)s.n_kv * p.rows * s.head_dim * 4);
   p.part_o = reinterpret_cast<float*>(ws);
-  p.part_lse = reinterpret_cast<float*>(ws + ((size_t)s.n_kv * p.rows * p.splits * s.head_dim * 4 + 255) / 256 * 256);
-  state->o = p.part_o;
-  state->lse = p.part_lse;
-  state->splits = p.splits;
+  p.part_lse = reinterpret_cast<float*>(ws + part_o);
+  CombineParams cp;
+  cp.part_o = p.part_o;
+  cp.part_lse = p.part_lse;
+  cp.o = reinterpret_cast<float*>(ws + part_o + part_l);
+  cp.lse = reinterpret_cast<float*>(ws + part_o + part_l + comb_o);
+  cp.total_rows = s.n_kv * p.rows;
+  cp.splits = p.splits;
+  state->o = cp.o;
+  state->lse = cp.lse;
+  state->splits = 1;
   state->rows = p.rows;
 
   const int tiles = (p.rows + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
@@ -279,9 +340,31 @@ pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUte
     if (e != cudaSuccess) return cuda_fail(e, "prefix_attn_kernel launch");
     return PKV_OK;
   };
-  if (s.head_dim == 128) return run(prefix_attn_kernel<128>);
-  if (s.head_dim == 64) return run(prefix_attn_kernel<64>);
-  return PKV_ERR_UNSUPPORTED;
+  auto combine = [&](auto kern) -> pkv_status {
+    const long long threads = (long long)cp.total_rows * (s.head_dim / 4);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
+    cfg.blockDim = dim3(256);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, cp);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "prefix_combine_kernel launch");
+    return PKV_OK;
+  };
+  pkv_status st = PKV_ERR_UNSUPPORTED;
+  if (s.head_dim == 128) {
+    st = run(prefix_attn_kernel<128>);
+    if (st == PKV_OK) st = combine(prefix_combine_kernel<128>);
+  } else if (s.head_dim == 64) {
+    st = run(prefix_attn_kernel<64>);
+    if (st == PKV_OK) st = combine(prefix_combine_kernel<64>);
+  }
+  return st;
 }
 
 }  // namespace pkv
