@@ -530,6 +530,12 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   float head_k_scale = 1.f, head_v_scale = 1.f;
 
   uint32_t qf[KS][2];
+  // INT8 / INT4: the queries as two 8-bit parts per dim for m16n8k32 MMAs
+  // (q ~ qscale * (h + l / 254)), the per-column scales, and for INT4 the sums
+  // of the parts times 8 (the stored codes are offset by 8)
+  uint32_t qh[4][2], ql[4][2];
+  float qs0 = 0.f, qs1 = 0.f;
+  int ch0 = 0, ch1 = 0, cl0 = 0, cl1 = 0;
   float acc[KS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
@@ -599,18 +605,43 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       // chunk c ^ ((r >> 1) & 3), the same for rows g and g+8
       const uint32_t kb = kt + g * 64 + ((uint32_t)(c ^ ((g >> 1) & 3)) << 4);
       const uint4 r0 = lds128(kb), r1 = lds128(kb + 512);
+      // k-step kk: word kk of the chunk, its even nibbles (offset-binary codes
+      // + 8, as unsigned bytes) and its odd nibbles, against the query parts
+      int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        const int w = ks >> 1, h = ks & 1;
-        const uint32_t x0 = (&r0.x)[w] ^ 0x88888888u, x1 = (&r1.x)[w] ^ 0x88888888u;
-        uint32_t af[4];
-        af[0] = i4x2_to_f16x2(x0 >> (8 * h));
-        af[1] = i4x2_to_f16x2(x1 >> (8 * h));
-        af[2] = i4x2_to_f16x2(x0 >> (8 * h + 4));
-        af[3] = i4x2_to_f16x2(x1 >> (8 * h + 4));
-        if (ks & 1) mma_f16(sb, af, qf[ks][0], qf[ks][1]);
-        else mma_f16(sa, af, qf[ks][0], qf[ks][1]);
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t x0 = (&r0.x)[kk] ^ 0x88888888u, x1 = (&r1.x)[kk] ^ 0x88888888u;
+        const uint32_t af[4] = {x0 & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu, (x0 >> 4) & 0x0F0F0F0Fu,
+                                (x1 >> 4) & 0x0F0F0F0Fu};
+        mma_u8s8(ah, af, qh[kk][0], qh[kk][1]);
+        mma_u8s8(al, af, ql[kk][0], ql[kk][1]);
       }
+      // sum (code + 8) q = sum code q + 8 sum q: the offsets come back out exactly
+      sa[0] = ((float)(ah[0] - ch0) + (float)(al[0] - cl0) * (1.f / 254.f)) * qs0;
+      sa[1] = ((float)(ah[1] - ch1) + (float)(al[1] - cl1) * (1.f / 254.f)) * qs1;
+      sa[2] = ((float)(ah[2] - ch0) + (float)(al[2] - cl0) * (1.f / 254.f)) * qs0;
+      sa[3] = ((float)(ah[3] - ch1) + (float)(al[3] - cl1) * (1.f / 254.f)) * qs1;
+    } else if constexpr (CACHE == TC_INT8) {
+      // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each); k-step
+      // kk takes the bytes of dims 32c + 8kk + {0..3} and {4..7} as they are stored
+      uint4 kr[2][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        kr[0][h] = lds128(kt + (koff ^ (h << 4)));
+        kr[1][h] = lds128(kt + (koff ^ (h << 4)) + 1024);
+      }
+      int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int h = kk >> 1, wv = (kk & 1) * 2;
+        const uint32_t af[4] = {(&kr[0][h].x)[wv], (&kr[1][h].x)[wv], (&kr[0][h].x)[wv + 1], (&kr[1][h].x)[wv + 1]};
+        mma_s8s8(ah, af, qh[kk][0], qh[kk][1]);
+        mma_s8s8(al, af, ql[kk][0], ql[kk][1]);
+      }
+      sa[0] = ((float)ah[0] + (float)al[0] * (1.f / 254.f)) * qs0;
+      sa[1] = ((float)ah[1] + (float)al[1] * (1.f / 254.f)) * qs1;
+      sa[2] = ((float)ah[2] + (float)al[2] * (1.f / 254.f)) * qs0;
+      sa[3] = ((float)ah[3] + (float)al[3] * (1.f / 254.f)) * qs1;
     } else {
       // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each)
       uint4 kr[2][2];
@@ -624,13 +655,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const int h = ks >> 2, k = ks & 3;
         const uint32_t w0 = (&kr[0][h].x)[k], w1 = (&kr[1][h].x)[k];
         uint32_t af[4];
-        if constexpr (CACHE == TC_INT8) {
-          const uint32_t x0 = w0 ^ 0x80808080u, x1 = w1 ^ 0x80808080u;
-          af[0] = i8x2_to_f16x2(x0, 0x4140);
-          af[1] = i8x2_to_f16x2(x1, 0x4140);
-          af[2] = i8x2_to_f16x2(x0, 0x4342);
-          af[3] = i8x2_to_f16x2(x1, 0x4342);
-        } else if constexpr (CACHE == TC_E5M2) {
+        if constexpr (CACHE == TC_E5M2) {
           // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, as the f16 top bytes
           af[0] = prmt(w0, 0u, 0x1404);
           af[1] = prmt(w1, 0u, 0x1404);
@@ -865,7 +890,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           qf[ks][0] = qraw[ks][0];
           qf[ks][1] = qraw[ks][1];
         }
-      } else {
+      } else if constexpr (tc_fp8(CACHE)) {  // INT8 / INT4 quantise their queries below
         if (p.act_bf16) {
           fetch_query(u);
 #pragma unroll
@@ -908,6 +933,85 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       }
       head_k_scale = raw_k_scale;
       head_v_scale = raw_v_scale;
+      if constexpr (tc_row_scaled(CACHE)) {
+        // this lane's 32 dims 32c .. 32c+31 of query head g, quantised per head:
+        // t = q * 127 / max|q|, h = rint(t), l = rint((t - h) * 254), both in
+        // [-127, 127], so q = max|q| / 127 * (h + l / 254) to 1 part in 32000
+        const int kvq = hg * p.HPC + head_local;
+        const bool q_ok = qc * 8 + g < p.G;
+        const size_t qoff = ((size_t)s * p.n_q + kvq * p.G + qc * 8 + g) * D + 32 * c;
+        float x[32];
+        if (p.act_bf16) {
+          const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.query) + qoff);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 w = q_ok ? __ldg(q4 + i) : make_uint4(0u, 0u, 0u, 0u);
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              x[8 * i + 2 * k] = __uint_as_float(wv[k] << 16);
+              x[8 * i + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
+            }
+          }
+        } else {
+          const float4* q4 = reinterpret_cast<const float4*>(static_cast<const float*>(p.query) + qoff);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 w = q_ok ? __ldg(q4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[4 * i] = w.x;
+            x[4 * i + 1] = w.y;
+            x[4 * i + 2] = w.z;
+            x[4 * i + 3] = w.w;
+          }
+        }
+        float amax = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(x[e]));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        const float inv = amax > 0.f ? 127.f / amax : 0.f;
+        int hsum = 0, lsum = 0;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          int hv[8], lv[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float t = x[8 * kk + e] * inv;
+            const float hq = rintf(t);
+            hv[e] = (int)hq;
+            lv[e] = (int)rintf((t - hq) * 254.f);
+            hsum += hv[e];
+            lsum += lv[e];
+          }
+          if constexpr (CACHE == TC_INT8) {
+            // k-step kk: dims 32c + 8kk + {0..3} and {4..7}, as the stored bytes
+            qh[kk][0] = pack_s8x4(hv[0], hv[1], hv[2], hv[3]);
+            qh[kk][1] = pack_s8x4(hv[4], hv[5], hv[6], hv[7]);
+            ql[kk][0] = pack_s8x4(lv[0], lv[1], lv[2], lv[3]);
+            ql[kk][1] = pack_s8x4(lv[4], lv[5], lv[6], lv[7]);
+          } else {
+            // k-step kk: even and odd nibbles of the INT4 word kk (dims 32c + 8kk + {0,2,4,6}, {1,3,5,7})
+            qh[kk][0] = pack_s8x4(hv[0], hv[2], hv[4], hv[6]);
+            qh[kk][1] = pack_s8x4(hv[1], hv[3], hv[5], hv[7]);
+            ql[kk][0] = pack_s8x4(lv[0], lv[2], lv[4], lv[6]);
+            ql[kk][1] = pack_s8x4(lv[1], lv[3], lv[5], lv[7]);
+          }
+        }
+        hsum += __shfl_xor_sync(0xffffffffu, hsum, 1);
+        hsum += __shfl_xor_sync(0xffffffffu, hsum, 2);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+        lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+        // score columns are heads 2c and 2c+1: their values live on lanes 8c and 8c + 4
+        const float qsc = amax * (1.f / 127.f);
+        qs0 = __shfl_sync(0xffffffffu, qsc, 8 * c);
+        qs1 = __shfl_sync(0xffffffffu, qsc, 8 * c + 4);
+        if constexpr (CACHE == TC_INT4) {
+          ch0 = 8 * __shfl_sync(0xffffffffu, hsum, 8 * c);
+          ch1 = 8 * __shfl_sync(0xffffffffu, hsum, 8 * c + 4);
+          cl0 = 8 * __shfl_sync(0xffffffffu, lsum, 8 * c);
+          cl1 = 8 * __shfl_sync(0xffffffffu, lsum, 8 * c + 4);
+        }
+      }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
