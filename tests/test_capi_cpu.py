@@ -100,3 +100,49 @@ def test_workspace_size_host_paths(lib):
     if not torch.cuda.is_available():
         # sizing the tensor-core path needs the device's SM count
         assert lib.pkv_paged_attention_workspace_size(4, 8, 2, 128, 16, 1) == ctypes.c_size_t(-1).value
+
+
+def test_new_format_host_validation(lib):
+    # INT4 / E5M2 caches: row-scaled and head-scaled scale arrays are required
+    assert _write(lib, cache=5) == 1  # INT4 without scales
+    assert _write(lib, cache=4) == 1  # E5M2 without scales
+    assert _write(lib, cache=6) == 1  # no such dtype
+    assert _decode(lib, cache=5, ks=FAKE, vs=FAKE, d=64) == 2  # quantised caches need head_dim 128
+    assert _decode(lib, cache=4) == 1
+
+
+def test_window_pages_and_prefix_host_validation(lib):
+    a = dict(out=FAKE, q=FAKE, kc=FAKE, vc=FAKE, ks=None, vs=None, bt=FAKE, mb=8, cl=FAKE, mcl=100, S=2, nq=8, nkv=2,
+             d=128, bs=16, nb=16, scale=0.1)
+    common = [a[k] for k in ("out", "q", "kc", "vc", "ks", "vs", "bt", "mb", "cl", "mcl", "S", "nq", "nkv", "d", "bs",
+                             "nb", "scale")]
+    # window / sinks must be >= 0
+    assert lib.pkv_paged_attention_decode_window(*common, -1, 0, 1, 1, None, FAKE, 1 << 20, None, None) == 1
+    # a page list needs at least one entry per (sequence, KV head)
+    assert lib.pkv_paged_attention_decode_pages(*common, FAKE, 0, 1, 1, None, FAKE, 1 << 20, None, None) == 1
+    assert lib.pkv_paged_attention_decode_pages(*common, None, 4, 1, 1, None, FAKE, 1 << 20, None, None) == 1
+    # shared prefix: at least one block, shorter than every context, BF16 only
+    sp = lib.pkv_paged_attention_decode_shared_prefix
+
+    def shared(prefix, mcl=100, cache=1, key=None, value=None):
+        return sp(FAKE, FAKE, key, value, FAKE, FAKE, FAKE, 8, FAKE, mcl, 2, 8, 2, 128, 16, 16, 0.1, prefix, 1, cache,
+                  None, FAKE, 1 << 20, None, None)
+
+    assert shared(0) == 1
+    assert shared(7, mcl=100) == 1  # 7 blocks = 112 tokens: no private token left
+    assert shared(2, key=FAKE) == 1  # key without value
+    assert shared(2, cache=2) == 1  # INT8 without scales is rejected first
+    assert lib.pkv_shared_prefix_workspace_size(2, 8, 2, 128, 16, 0) == ctypes.c_size_t(-1).value
+
+
+def test_quest_host_validation(lib):
+    # summaries: BF16 / F32 caches, head_dim 64 or 128, block size 16
+    summ = lib.pkv_quest_page_summaries
+    assert summ(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 2, 2, 96, 16, 16, 1, 0, None, None) == 2
+    assert summ(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 2, 2, 128, 16, 16, 2, 0, None, None) == 2
+    assert summ(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 0, 2, 128, 16, 16, 1, 0, None, None) == 0  # nothing to do
+    sel = lib.pkv_quest_select
+    # k_pages >= 1, the score buffer is required, query heads a multiple of KV heads
+    assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 8, 2, 128, 16, 16, 1, 1, 0, FAKE, FAKE, None, None) == 1
+    assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 8, 2, 128, 16, 16, 1, 1, 4, FAKE, None, None, None) == 1
+    assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 6, 4, 128, 16, 16, 1, 1, 4, FAKE, FAKE, None, None) == 1
