@@ -349,6 +349,43 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const int per = max(1, (total + (int)gridDim.x - 1) / (int)gridDim.x);
   const int a = min((int)blockIdx.x * per, total);
   const int b = min(a + per, total);
+  // Producer lanes look up the physical blocks of 32 consecutive entries of
+  // the range: block i (lane's) of unit u, its KV head group, whether it is
+  // the unit's last block; -1 (bad = true) for an entry out of the pool.
+  auto lookup = [&](int base, int& phys, int& hg, int& unit_last, bool& bad) {
+    const int i = base + lane;
+    phys = -1;
+    hg = 0;
+    unit_last = 0;
+    bad = false;
+    if (i < b) {
+      const int u = upper_bound_smem(P, units + 1, i) - 1;
+      const int s = u / p.HG;
+      hg = u - s * p.HG;
+      unit_last = (i + 1 == P[u + 1]);
+      const int Ls = seq_len(p, s, false);
+      int lb;
+      if (p.pages) {
+        lb = __ldg(p.pages + ((size_t)s * p.n_kv + hg) * p.k_pages + (i - P[u]));
+        if (lb < 0 || (long long)lb * kBlockSize >= Ls) lb = -1;  // not a page of this sequence
+      } else {
+        lb = logical_block(attend_set(p, Ls), i - P[u]);
+      }
+      phys = lb < 0 ? -1 : __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + lb);
+      if (phys < 0 || (long long)phys >= p.num_blocks) {
+        bad = true;
+        phys = -1;
+      }
+    }
+  };
+  // The first lookup reads only block_tables (and context_lens): it may run
+  // before the wait below (page lists may come from the previous kernel).
+  int phys0 = -1, hg0 = 0, last0 = 0;
+  bool bad0 = false, early = false;
+  if (warp == p.NCW && a < b && !p.pages) {
+    lookup(a, phys0, hg0, last0, bad0);
+    early = true;
+  }
   // Everything above read only context_lens and block_tables.  Under a
   // programmatic launch the previous kernel may still be running: wait for it
   // before touching queries, new rows, the cache, the workspace or outputs.
@@ -360,27 +397,17 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     int it = 0;
     bool abort = false, appended = false;
     for (int base = a; base < b && !abort; base += 32) {
-      const int i = base + lane;
-      int phys = -1, hg = 0, unit_last = 0;
-      if (i < b) {
-        const int u = upper_bound_smem(P, units + 1, i) - 1;
-        const int s = u / p.HG;
-        hg = u - s * p.HG;
-        unit_last = (i + 1 == P[u + 1]);
-        const int Ls = seq_len(p, s, false);
-        int lb;
-        if (p.pages) {
-          lb = __ldg(p.pages + ((size_t)s * p.n_kv + hg) * p.k_pages + (i - P[u]));
-          if (lb < 0 || (long long)lb * kBlockSize >= Ls) lb = -1;  // not a page of this sequence
-        } else {
-          lb = logical_block(attend_set(p, Ls), i - P[u]);
-        }
-        phys = lb < 0 ? -1 : __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + lb);
-        if (phys < 0 || (long long)phys >= p.num_blocks) {
-          flag_error(p.err, DEVERR_BLOCK_RANGE);
-          phys = -1;
-        }
+      int phys, hg, unit_last;
+      bool bad;
+      if (base == a && early) {
+        phys = phys0;
+        hg = hg0;
+        unit_last = last0;
+        bad = bad0;
+      } else {
+        lookup(base, phys, hg, unit_last, bad);
       }
+      if (bad) flag_error(p.err, DEVERR_BLOCK_RANGE);
       const int n = min(32, b - base);
       for (int k = 0; k < n; ++k) {
         const int ph = __shfl_sync(0xffffffffu, phys, k);
