@@ -367,8 +367,6 @@ def run_b200(args, rank, world, local):
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
 
-    if w.window:
-        args.unfused = True  # the windowed decode has no fused-append entry point
 
     prefix_blocks = w.shared_prefix_tokens // bs
     if prefix_blocks:
@@ -377,7 +375,10 @@ def run_b200(args, rank, world, local):
         ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
 
     def fused(out, q, k_new, v_new, bt, cl, tun):
-        if prefix_blocks:
+        if w.window:
+            ops.paged_decode_step_window(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
+                                         w.sm_scale, ks, vs, workspace=ws, device_error=err, cache_dtype=named)
+        elif prefix_blocks:
             ops.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, cl, w.max_context_len, prefix_blocks,
                                                      key=k_new, value=v_new, sm_scale=w.sm_scale, workspace=ws,
                                                      device_error=err)
@@ -519,6 +520,7 @@ def run_b200(args, rank, world, local):
                 + ("" if args.unfused else " with fused append")
                 + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
                 + (" (pkv_paged_attention_decode_shared_prefix)" if prefix_blocks
+                   else " (pkv_paged_decode_step_window)" if w.window and not args.unfused
                    else " (pkv_paged_attention_decode)" if args.unfused else " (pkv_paged_decode_step)"),
                 "peak_source": f"{peak_kind} hbm_gbs",
                 "bytes_per_launch": kv_bytes,
@@ -531,7 +533,8 @@ def run_b200(args, rank, world, local):
                              + (1 if args.unfused else 0)) * args.steps,
             "step": ("append, then decode + merge of split sequences" if args.unfused
                      else "append fused into the decode kernel, then the merge of split sequences")
-            + ("" if args.no_overlap or args.unfused else "; prologue overlaps the previous step (programmatic launch)"),
+            + ("" if args.no_overlap or args.unfused or w.window or prefix_blocks
+               else "; prologue overlaps the previous step (programmatic launch)"),
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:

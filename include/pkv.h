@@ -190,6 +190,19 @@ pkv_status pkv_paged_attention_decode_window(void* out, const void* query, const
                                              pkv_dtype cache_dtype, float* lse_out, void* workspace,
                                              size_t workspace_bytes, int32_t* device_error, void* stream);
 
+/* The fused step (append token L-1, then attend) with a sliding window and
+ * sinks: the new rows of pkv_paged_decode_step, the attended positions of
+ * pkv_paged_attention_decode_window (the appended token is always inside the
+ * window).  Same arguments, layouts and rules as those two calls. */
+pkv_status pkv_paged_decode_step_window(void* out, const void* query, const void* key, const void* value,
+                                        void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                        int n_kv, int head_dim, int block_size, int64_t num_blocks, float sm_scale,
+                                        int window, int sinks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                        float* lse_out, void* workspace, size_t workspace_bytes,
+                                        int32_t* device_error, void* stream);
+
 /*
  * Decode for a batch whose sequences all begin with the same physical blocks:
  * a shared prompt prefix stored once ("Chapter 18 - KV-Cache Optimization

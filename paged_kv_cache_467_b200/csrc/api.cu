@@ -412,6 +412,22 @@ pkv_status pkv_paged_decode_step(void* out, const void* query, const void* key, 
                                   workspace_bytes, device_error, nullptr, stream);
 }
 
+pkv_status pkv_paged_decode_step_window(void* out, const void* query, const void* key, const void* value,
+                                        void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                                        const int32_t* block_tables, int max_blocks_per_seq,
+                                        const int32_t* context_lens, int max_context_len, int num_seqs, int n_q,
+                                        int n_kv, int head_dim, int block_size, int64_t num_blocks, float sm_scale,
+                                        int window, int sinks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
+                                        float* lse_out, void* workspace, size_t workspace_bytes,
+                                        int32_t* device_error, void* stream) {
+  if (num_seqs > 0 && (!key || !value || !aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
+  if (head_scaled(cache_dtype) && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
+  return decode_impl(out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream, key,
+                     value, window, sinks);
+}
+
 pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,
                            const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,
                            int64_t num_blocks, pkv_dtype cache_dtype, int32_t* device_error, void* stream) {

@@ -87,6 +87,9 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attention_decode_pages_ex.argtypes = (lib.pkv_paged_attention_decode_pages.argtypes[:-1]
                                                         + [ctypes.POINTER(DecodeTuning), vp])
     lib.pkv_paged_attention_decode_pages_ex.restype = i32
+    lib.pkv_paged_decode_step_window.argtypes = (lib.pkv_paged_decode_step.argtypes[:19] + [i32, i32]
+                                                 + lib.pkv_paged_decode_step.argtypes[19:])
+    lib.pkv_paged_decode_step_window.restype = i32
     lib.pkv_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.pkv_shared_prefix_workspace_size.restype = sz
     lib.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
@@ -408,4 +411,28 @@ def paged_attention_decode_shared_prefix(out, query, key_cache, value_cache, blo
         ws_bytes, _ptr(device_error), _stream(query.device),
     )
     _check(st, "pkv_paged_attention_decode_shared_prefix")
+    return out
+
+
+def paged_decode_step_window(out, query, key, value, key_cache, value_cache, block_tables, context_lens,
+                             max_context_len: int, window: int, sinks: int = 0, sm_scale: float | None = None,
+                             k_scale=None, v_scale=None, lse_out=None, workspace=None, device_error=None,
+                             cache_dtype: str | None = None):
+    """The fused step (append token L-1, attend) over positions [0, sinks) and [L - window, L)."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    ccode = cache_code(key_cache, cache_dtype)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.pkv_paged_decode_step_window(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q,
+        n_kv, d, block_size, num_blocks, float(sm_scale), int(window), int(sinks), act_code(query), ccode,
+        _ptr(lse_out), _ptr(workspace), ws_bytes, _ptr(device_error), _stream(query.device),
+    )
+    _check(st, "pkv_paged_decode_step_window")
     return out

@@ -96,3 +96,32 @@ def test_window_covering_everything_equals_full_decode():
     assert np.array_equal(out, full) and np.array_equal(lse, lse_full)
     out0, lse0 = run_window(w, st, 0, 5)
     assert np.array_equal(out0, full) and np.array_equal(lse0, lse_full)
+
+
+@pytest.mark.parametrize("cache,act,d", [("bf16", "bf16", 128), ("int8", "bf16", 128), ("fp8_e5m2", "bf16", 128),
+                                         ("f32", "f32", 64)])
+def test_fused_window_step(cache, act, d):
+    """Append token L-1 and attend over the window and sinks in one call: the
+    appended rows are bit-exact and the outputs match the oracle."""
+    from paged_kv_cache_467_b200 import ops
+    from gpu_harness import assert_rows_bit_exact, named, new_rows
+
+    window, sinks = 200, 4
+    w = workloads.make_workload("w", seed=64, context_lens=LENGTHS, n_q=16, n_kv=4, head_dim=d, act_dtype=act,
+                                cache_dtype=cache, extra_blocks=3, outlier_fraction=0.01 if cache != "f32" else 0.0)
+    st = fill_gpu(w, append_new=False)
+    k, v = new_rows(w)
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    out = torch.full((w.num_seqs, w.n_q, w.head_dim), float("nan"), dtype=dt, device="cuda")
+    lse = torch.full((w.num_seqs, w.n_q), float("nan"), dtype=torch.float32, device="cuda")
+    ops.paged_decode_step_window(out, st.query, k, v, st.key_cache, st.value_cache, st.block_tables, st.context_lens,
+                                 w.max_context_len, window, sinks, w.sm_scale, st.k_scale, st.v_scale, lse,
+                                 device_error=st.device_error, cache_dtype=named(w))
+    torch.cuda.synchronize()
+    assert int(st.device_error.item()) == 0
+    got = out.float().cpu().numpy().astype(np.float64)
+    gl = lse.cpu().numpy().astype(np.float64)
+    check(w, st, got, gl, window, sinks)
+    for s in range(w.num_seqs):
+        _, _, rows = oracle_sequence(w, s, st.fp8_scales, window=window, sinks=sinks)
+        assert_rows_bit_exact(w, st, s, rows)
