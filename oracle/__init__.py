@@ -26,3 +26,5 @@ from .paged_attention import (  # noqa: F401
 from .block_ops import copy_blocks, swap_blocks  # noqa: F401,E402
 from .quest import (decode_over_pages, group_scores, page_scores, page_summaries, quest_decode,  # noqa: F401,E402
                     select_pages)
+from .kivi import (KIVI_BITS, kivi_cache_state, kivi_decode, kivi_decode_sequence,  # noqa: F401,E402
+                   kivi_dequantize_block, kivi_quantize_block)

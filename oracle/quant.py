@@ -163,3 +163,27 @@ def unpack_int4(packed) -> np.ndarray:
     out[..., 0::2] = np.where(lo >= 8, lo - 16, lo)
     out[..., 1::2] = np.where(hi >= 8, hi - 16, hi)
     return out
+
+
+def pack_int2(codes) -> np.ndarray:
+    """Signed 2-bit codes [..., d] (d a multiple of 4, values in [-2, 1]) -> bytes [..., d/4].
+
+    Storage reading for the 2-bit KIVI cache ("KV Cache Engineering", section 8;
+    "Chapter 18 - KV-Cache Optimization Strategies", KV-Cache Quantization
+    table): two's-complement bit pairs, the code of element 4j + m in bits
+    [2m, 2m + 1] of byte j.
+    """
+    c = np.asarray(codes, dtype=np.int64)
+    pairs = (c & 0x3).astype(np.uint8)
+    return (pairs[..., 0::4] | (pairs[..., 1::4] << 2) | (pairs[..., 2::4] << 4) | (pairs[..., 3::4] << 6)).astype(
+        np.uint8)
+
+
+def unpack_int2(packed) -> np.ndarray:
+    """Bytes [..., d/4] -> signed codes [..., d] (inverse of pack_int2)."""
+    b = np.asarray(packed, dtype=np.uint8).astype(np.int64)
+    out = np.empty(b.shape[:-1] + (4 * b.shape[-1],), dtype=np.int64)
+    for m in range(4):
+        v = (b >> (2 * m)) & 0x3
+        out[..., m::4] = np.where(v >= 2, v - 4, v)
+    return out

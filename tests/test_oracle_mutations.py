@@ -175,3 +175,42 @@ def test_e5m2_wrong_bias_is_caught(monkeypatch):
     monkeypatch.setattr(oq, "e5m2_value_table", lambda: t)
     _fails(fpins.test_e5m2_table_closed_forms)
     _fails(fpins.test_e5m2_table_matches_torch_float8)
+
+
+def test_kivi_keys_grouped_per_token_are_caught(monkeypatch):
+    import oracle.kivi as ok
+    import test_oracle_kivi as kpins
+
+    def per_token(k_rows, v_rows, bits=ok.KIVI_BITS):
+        k_rows = np.asarray(k_rows, np.float32)
+        kc, ksc, vc, vsc = real(k_rows, v_rows, bits)
+        for t in range(k_rows.shape[0]):
+            for h in range(k_rows.shape[1]):
+                codes, scale, _ = oq.absmax_quantize(k_rows[t, h], bits, np.float32)
+                kc[t, h] = codes
+                ksc[h] = scale  # the last token's scale stands for the block
+        return kc, ksc, vc, vsc
+
+    real = ok.kivi_quantize_block
+    monkeypatch.setattr(ok, "kivi_quantize_block", per_token)
+    _fails(kpins.test_two_bit_codes_closed_form)
+    _fails(kpins.test_key_groups_are_channels)
+
+
+def test_kivi_at_four_bits_is_caught(monkeypatch):
+    import oracle.kivi as ok
+    import test_oracle_kivi as kpins
+
+    real = ok.kivi_quantize_block
+    monkeypatch.setattr(ok, "kivi_quantize_block", lambda k, v, bits=4: real(k, v, 4))
+    _fails(kpins.test_two_bit_codes_closed_form)
+    _fails(kpins.test_round_trip_bounds)
+
+
+def test_kivi_residual_dropped_is_caught(monkeypatch):
+    import oracle.kivi as ok
+    import test_oracle_kivi as kpins
+
+    real = ok.kivi_decode
+    monkeypatch.setattr(ok, "kivi_decode", lambda q, b, rk, rv, s: real(q, b, rk[:0], rv[:0], s))
+    _fails(kpins.test_decode_is_attention_over_restored_rows)
