@@ -145,6 +145,8 @@ def oracle_step_sample(w, seqs, host_rows):
 
     from paged_kv_cache_467_b200 import accounting
 
+    if w.cache_dtype == "kivi2":
+        return oracle_kivi_step_sample(w, seqs, host_rows)
     per_token = accounting.cache_bytes(1, w.n_kv, w.head_dim, 1, accounting.BYTES_PER_VALUE[w.cache_dtype])
     per_token += accounting.scale_bytes_per_token(w.cache_dtype, w.n_kv)
     kv_bytes = 0
@@ -161,6 +163,30 @@ def oracle_step_sample(w, seqs, host_rows):
     return kv_bytes
 
 
+def oracle_kivi_step_sample(w, seqs, host_rows):
+    """One oracle KIVI step per sampled sequence: the new row joins the BF16
+    residual, a residual that became a full block is quantised, then the decode."""
+    import numpy as np
+
+    import oracle
+
+    from paged_kv_cache_467_b200 import accounting
+
+    kv_bytes = 0
+    per_block = accounting.kivi_block_bytes(w.n_kv, w.head_dim, w.block_size)
+    for s in seqs:
+        blocks, rk, rv, K, V, q = host_rows[s]
+        L = int(w.context_lens[s])
+        rk = np.concatenate([rk, K[L - 1 : L]])
+        rv = np.concatenate([rv, V[L - 1 : L]])
+        if rk.shape[0] == w.block_size:
+            blocks = blocks + [oracle.kivi_quantize_block(rk, rv)]
+            rk, rv = rk[:0], rv[:0]
+        oracle.kivi_decode(q, blocks, rk, rv, w.sm_scale)
+        kv_bytes += len(blocks) * per_block + rk.shape[0] * w.n_kv * w.head_dim * 2 * 2
+    return kv_bytes
+
+
 def prepare_oracle_rows(w, seqs, scales=None):
     import numpy as np
 
@@ -168,6 +194,13 @@ def prepare_oracle_rows(w, seqs, scales=None):
 
     rows = {}
     q = w.query()
+    if w.cache_dtype == "kivi2":
+        for s in seqs:
+            L = int(w.context_lens[s])
+            K, V = w.sequence_kv(s)
+            blocks, rk, rv = oracle.kivi_cache_state(K[: L - 1], V[: L - 1])
+            rows[s] = (blocks, rk, rv, K, V, q[s])
+        return rows
     for s in seqs:
         L = int(w.context_lens[s])
         nb = -(-L // w.block_size)
@@ -327,7 +360,25 @@ def run_b200(args, rank, world, local):
     shape = (w.num_blocks, bs, nkv, d)
     # q/K/V ~ N(0,1) synthetic cache, filled on the device (the writer is exercised by the step's append)
     act = torch.float32 if w.act_dtype == "f32" else torch.bfloat16
-    if w.cache_dtype in ("bf16", "f32"):
+    kivi = w.cache_dtype == "kivi2"
+    if kivi:
+        if args.unfused:
+            raise SystemExit("the 2-bit KIVI cache appends inside its residual pass: no unfused step")
+        # every pool block quantised from N(0,1) rows by the library's block quantiser,
+        # and N(0,1) residual rows (the partial last block of each sequence)
+        kc = torch.empty((w.num_blocks, bs, nkv, d // 4), device=dev, dtype=torch.uint8)
+        vc = torch.empty_like(kc)
+        ks = torch.empty((w.num_blocks, nkv, d), device=dev)
+        vs = torch.empty((w.num_blocks, bs, nkv), device=dev)
+        for b0 in range(0, w.num_blocks, 4096):
+            nblk = min(4096, w.num_blocks - b0)
+            kk = torch.randn((nblk, bs, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+            vv = torch.randn((nblk, bs, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+            dst = torch.arange(b0, b0 + nblk, device=dev, dtype=torch.int32)
+            ops.kivi_quantize_blocks(kk, vv, dst, kc, vc, ks, vs)
+        res_k = torch.randn((S, bs, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+        res_v = torch.randn((S, bs, nkv, d), device=dev, generator=gen).to(torch.bfloat16)
+    elif w.cache_dtype in ("bf16", "f32"):
         kc = torch.randn(shape, device=dev, generator=gen).to(act)
         vc = torch.randn(shape, device=dev, generator=gen).to(act)
         ks = vs = None
@@ -362,7 +413,10 @@ def run_b200(args, rank, world, local):
     # the kernel launched right before a step, so each step may overlap its
     # prologue with the previous step's tail (programmatic dependent launch).
     tuning = None if args.no_overlap else ops.DecodeTuning(0, 0, 0, ops.TUNE_OVERLAP_PROLOGUE)
-    nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc, named))
+    if kivi:
+        nws = ops.kivi_workspace_size(S, nq, nkv, d, bs)
+    else:
+        nws = ops.paged_attention_workspace_size(S, nq, nkv, d, bs, ops.cache_code(kc, named))
     ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     kv_bytes = accounting.decode_kv_bytes(w)
@@ -375,7 +429,10 @@ def run_b200(args, rank, world, local):
         ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
 
     def fused(out, q, k_new, v_new, bt, cl, tun):
-        if w.window:
+        if kivi:
+            ops.kivi_decode(out, q, res_k, res_v, kc, vc, ks, vs, bt, cl, w.max_context_len, key=k_new, value=v_new,
+                            sm_scale=w.sm_scale, workspace=ws, device_error=err)
+        elif w.window:
             ops.paged_decode_step_window(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
                                          w.sm_scale, ks, vs, workspace=ws, device_error=err, cache_dtype=named)
         elif prefix_blocks:
@@ -451,7 +508,7 @@ def run_b200(args, rank, world, local):
     # The step's inputs (query, new K/V rows, block tables, lengths, slots) live
     # in one pinned host buffer and cross to the device in one copy per step;
     # the output comes back in one copy, and the host waits for it.
-    parts = [q, k_new, v_new, bt, cl, slots]
+    parts = [q, k_new, v_new, bt, cl] + ([] if kivi else [slots])
     offs, total = [], 0
     for t in parts:
         offs.append(total)
@@ -463,7 +520,8 @@ def run_b200(args, rank, world, local):
         nbytes = t.numel() * t.element_size()
         h_in[o : o + nbytes].copy_(t.contiguous().view(torch.uint8).reshape(-1).cpu())
         views.append(d_in[o : o + nbytes].view(t.dtype).view(t.shape))
-    d_q, d_k, d_v, d_bt, d_cl, d_slots = views
+    d_q, d_k, d_v, d_bt, d_cl = views[:5]
+    d_slots = None if kivi else views[5]
     h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     h2d = total
     d2h = h_out.numel() * h_out.element_size()
@@ -515,7 +573,8 @@ def run_b200(args, rank, world, local):
                 "unit": "GB/s",
                 "frac": achieved / peak,
                 "traffic": traffic,
-                "kernel": ("prefix_attn_kernel + " if prefix_blocks else "")
+                "kernel": "kivi_residual_kernel + decode_tc_kernel<KIVI> + decode_merge_kernel (pkv_kivi_decode)"
+                if kivi else ("prefix_attn_kernel + " if prefix_blocks else "")
                 + ("decode_f32_kernel" if w.cache_dtype == "f32" else "decode_tc_kernel")
                 + ("" if args.unfused else " with fused append")
                 + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
@@ -529,16 +588,20 @@ def run_b200(args, rank, world, local):
             "e2e": {"value": whole_job_gbs(kv_bytes, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps},
             # decode kernel + merge of split sequences (+ the prefix pass, + the cache write when unfused)
-            "gpu_launches": ((1 if w.cache_dtype == "f32" else 2) + (1 if prefix_blocks else 0)
+            "gpu_launches": ((1 if w.cache_dtype == "f32" else 2) + (1 if prefix_blocks or kivi else 0)
                              + (1 if args.unfused else 0)) * args.steps,
-            "step": ("append, then decode + merge of split sequences" if args.unfused
+            "step": ("residual pass (append, quantise a completed block, attend the BF16 residual rows), then "
+                     "decode over the 2-bit blocks + merge of split sequences" if kivi
+                     else "append, then decode + merge of split sequences" if args.unfused
                      else "append fused into the decode kernel, then the merge of split sequences")
             + ("" if args.no_overlap or args.unfused or w.window or prefix_blocks
                else "; prologue overlaps the previous step (programmatic launch)"),
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            b, t, seqs = time_oracle(w, budget_s=12.0)
+            # the KIVI oracle quantises a sequence's blocks group by group before its
+            # timed step (seconds per sequence, untimed): a few sequences bound the run
+            b, t, seqs = time_oracle(w, budget_s=12.0, max_seqs=3 if kivi else None)
             line["cpu_baseline"] = {
                 "value": b / t / 1e9,
                 "unit": "GB/s",

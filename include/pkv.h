@@ -38,9 +38,13 @@ typedef enum {
   PKV_INT8 = 2,     /* int8 codes, one float scale per (token, head); cache only */
   PKV_FP8_E4M3 = 3, /* OCP E4M3 bytes, one float scale per KV head; cache only */
   PKV_FP8_E5M2 = 4, /* OCP E5M2 bytes, one float scale per KV head; cache only */
-  PKV_INT4 = 5      /* signed 4-bit codes, two per byte (element 2j in the low
+  PKV_INT4 = 5,     /* signed 4-bit codes, two per byte (element 2j in the low
                        nibble of byte j), one float scale per (token, KV head);
                        cache only, pools [num_blocks, block_size, n_kv, head_dim/2] */
+  PKV_KIVI2 = 6     /* 2-bit KIVI cache (pkv_kivi_* calls only): signed 2-bit
+                       codes, four per byte (element 4j + m in bits [2m, 2m+1]
+                       of byte j), K scaled per (block, KV head, channel), V per
+                       (token, KV head); pools [num_blocks, block_size, n_kv, head_dim/4] */
 } pkv_dtype;
 
 typedef enum {
@@ -384,6 +388,77 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const
                                              float* lse_out, int32_t* device_error, void* stream);
 
 /*
+ * 2-bit KIVI cache ("KV Cache Engineering for LLM Serving", section 8,
+ * Quantization: KIVI groups key values by channel and value-cache numbers by
+ * token, with a 2-bit cache; "Chapter 18 - KV-Cache Optimization Strategies",
+ * KV-Cache Quantization methods table).  Quantiser: the section's symmetric
+ * absmax one at 2 bits: scale = max |x| of the group (float), codes
+ * rint(x / scale) (ties to even) in {-1, 0, 1}, restored values code * scale;
+ * an all-zero group has scale 0 and codes 0.
+ *   K group: one channel of one KV head over the 16 tokens of a block
+ *   V group: the head_dim values of one token of one KV head
+ * A channel group needs its whole block, so only full blocks are quantised.
+ * Sequence s of length L keeps positions [0, 16 * floor(L / 16)) in the pool
+ * blocks named by its block table and the L % 16 positions of its partial
+ * last block, in order, in rows [0, L % 16) of its BF16 residual.
+ *
+ * Layouts (row-major, innermost last):
+ *   key_cache, value_cache  device uint8 [num_blocks, 16, n_kv, head_dim / 4]:
+ *                           element 4j + m of a row in bits [2m, 2m+1] of byte
+ *                           j, two's complement
+ *   k_scale                 device float [num_blocks, n_kv, head_dim]
+ *   v_scale                 device float [num_blocks, 16, n_kv]
+ *   residual_k, residual_v  device bf16 [num_seqs, 16, n_kv, head_dim]; row r of
+ *                           sequence s holds position 16 * floor(L / 16) + r
+ * BF16 activations, head_dim 128, block_size 16, n_q / n_kv <= 64.  All
+ * pointers 16-byte aligned.
+ */
+
+/* Workspace bytes of pkv_kivi_decode; (size_t)-1 for an unsupported shape. */
+size_t pkv_kivi_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size);
+
+/*
+ * Quantise whole 16-token blocks of K/V rows into the pools (prefill).
+ *   key_rows, value_rows  device bf16 [num_src_blocks, 16, n_kv, head_dim]
+ *   dst_blocks            device int32 [num_src_blocks]: physical block of
+ *                         each source block; -1 skips it, any other id outside
+ *                         [0, num_blocks) sets PKV_DEVERR_BLOCK_RANGE and skips it
+ * Destinations must be distinct.  One launch on `stream`.
+ */
+pkv_status pkv_kivi_quantize_blocks(const void* key_rows, const void* value_rows, const int32_t* dst_blocks,
+                                    int64_t num_src_blocks, void* key_cache, void* value_cache, float* k_scale,
+                                    float* v_scale, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    pkv_dtype act_dtype, int32_t* device_error, void* stream);
+
+/*
+ * Decode over a KIVI cache, optionally appending the step's token first.
+ *
+ *   key, value     optional device bf16 [num_seqs, n_kv, head_dim]: token
+ *                  L - 1 of each sequence (L = context_lens[s] >= 1, counted
+ *                  with it), written to residual row (L - 1) % 16; when that
+ *                  row is 15 the block is full and its 16 rows are quantised
+ *                  into physical block block_tables[s][(L - 1) / 16].  Both
+ *                  NULL for a plain decode.
+ *   query, out     device bf16 [num_seqs, n_q, head_dim]
+ *   lse_out        optional device float [num_seqs, n_q], natural log
+ *   workspace      pkv_kivi_workspace_size bytes (any contents)
+ * For each query head: softmax(sm_scale * q.k) over the dequantised keys of
+ * the full blocks and the residual rows, weighting the values likewise; a
+ * sequence with L == 0 gives out 0 and lse -inf.  Context lengths outside
+ * [0, min(max_context_len, max_blocks_per_seq * 16)] set
+ * PKV_DEVERR_CONTEXT_LEN; block-table entries outside [0, num_blocks) set
+ * PKV_DEVERR_BLOCK_RANGE (the block is skipped).  Three launches on `stream`
+ * (residual pass, decode over the full blocks, merge of split units), the
+ * last two queued with programmatic serialisation.
+ */
+pkv_status pkv_kivi_decode(void* out, const void* query, const void* key, const void* value, void* residual_k,
+                           void* residual_v, void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int max_context_len, int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                           int64_t num_blocks, float sm_scale, pkv_dtype act_dtype, float* lse_out, void* workspace,
+                           size_t workspace_bytes, int32_t* device_error, void* stream);
+
+/*
  * Copy whole physical blocks inside one pool: copy-on-write of shared blocks.
  *
  * Several block tables may point at one physical block; when a sequence
@@ -393,14 +468,16 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const
  * K and V pools (and, for INT8 / INT4, of k_scale / v_scale) <- block block_mapping[2p].
  *
  *   key_cache, value_cache  device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
- *   k_scale, v_scale        INT8 / INT4: device [num_blocks, block_size, n_kv]; NULL otherwise
- *                           (FP8 per-head scales belong to no block)
+ *   k_scale, v_scale        INT8 / INT4: device [num_blocks, block_size, n_kv]; KIVI2:
+ *                           k_scale [num_blocks, n_kv, head_dim], v_scale [num_blocks,
+ *                           block_size, n_kv]; NULL otherwise (FP8 per-head scales
+ *                           belong to no block)
  *   block_mapping           device (or mapped host) int64 [num_pairs, 2] = (src, dst)
  * Destinations must be distinct and no block may be both a source and a
  * destination in one call (all pairs run in parallel).  Out-of-range block ids
  * set PKV_DEVERR_BLOCK_RANGE and the pair is skipped.  The bytes of one row
- * (n_kv * head_dim * bytes per value, half a byte for INT4) must be a multiple
- * of 16.
+ * (n_kv * head_dim * bytes per value, half a byte for INT4, a quarter for
+ * KIVI2) must be a multiple of 16.
  */
 pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,
                            const int64_t* block_mapping, int64_t num_pairs, int n_kv, int head_dim, int block_size,

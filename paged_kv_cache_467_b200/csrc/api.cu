@@ -1,6 +1,8 @@
 // C ABI of libpkv: argument validation, launch planning and status codes.
 // Every check here runs on the host before anything is enqueued.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -187,10 +189,13 @@ static pkv_status move_plan(const void* src_k, const void* src_v, const float* s
                             int64_t num_pairs, int n_kv, int head_dim, int block_size, pkv_dtype cache_dtype,
                             const void* src[4], void* dst[4], size_t bpb[4], int* npools) {
   if (num_pairs < 0 || n_kv <= 0 || head_dim <= 0 || block_size <= 0) return PKV_ERR_INVALID_ARG;
-  if (!valid_dtype(cache_dtype)) return PKV_ERR_INVALID_ARG;
+  const bool kivi = cache_dtype == PKV_KIVI2;
+  if (!valid_dtype(cache_dtype) && !kivi) return PKV_ERR_INVALID_ARG;
   if (num_pairs > 0 && (!pairs || !src_k || !src_v || !dst_k || !dst_v)) return PKV_ERR_INVALID_ARG;
   const size_t elem = cache_dtype == PKV_F32 ? 4 : (cache_dtype == PKV_BF16 ? 2 : 1);
-  const size_t row = cache_dtype == PKV_INT4 ? (size_t)n_kv * head_dim / 2 : (size_t)n_kv * head_dim * elem;
+  const size_t row = cache_dtype == PKV_INT4 ? (size_t)n_kv * head_dim / 2
+                     : kivi                  ? (size_t)n_kv * head_dim / 4
+                                             : (size_t)n_kv * head_dim * elem;
   if (row % 16 != 0) return PKV_ERR_UNSUPPORTED;
   if (!aligned16(src_k) || !aligned16(src_v) || !aligned16(dst_k) || !aligned16(dst_v)) return PKV_ERR_INVALID_ARG;
   src[0] = src_k;
@@ -199,16 +204,18 @@ static pkv_status move_plan(const void* src_k, const void* src_v, const float* s
   dst[1] = dst_v;
   bpb[0] = bpb[1] = row * block_size;
   *npools = 2;
-  const bool int8 = row_scaled(cache_dtype);
-  if (int8 != (src_ks && src_vs && dst_ks && dst_vs)) return PKV_ERR_INVALID_ARG;
-  if (int8) {
+  const bool scaled = row_scaled(cache_dtype) || kivi;
+  if (scaled != (src_ks && src_vs && dst_ks && dst_vs)) return PKV_ERR_INVALID_ARG;
+  if (scaled) {
     if (!aligned16(src_ks) || !aligned16(src_vs) || !aligned16(dst_ks) || !aligned16(dst_vs)) return PKV_ERR_INVALID_ARG;
     if (((size_t)block_size * n_kv * 4) % 16 != 0) return PKV_ERR_UNSUPPORTED;
     src[2] = src_ks;
     src[3] = src_vs;
     dst[2] = dst_ks;
     dst[3] = dst_vs;
-    bpb[2] = bpb[3] = (size_t)block_size * n_kv * 4;
+    // KIVI: K scales per (head, channel) of the block, V per (token, head)
+    bpb[2] = kivi ? (size_t)n_kv * head_dim * 4 : (size_t)block_size * n_kv * 4;
+    bpb[3] = (size_t)block_size * n_kv * 4;
     *npools = 4;
   }
   return PKV_OK;
@@ -426,6 +433,95 @@ pkv_status pkv_paged_decode_step_window(void* out, const void* query, const void
                      context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
                      act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream, key,
                      value, window, sinks);
+}
+
+// ---------------------------------------------------------------- 2-bit KIVI cache
+static pkv_status check_kivi_shape(int num_seqs, int n_q, int n_kv, int head_dim, int block_size, pkv_dtype act) {
+  if (num_seqs < 0 || n_q <= 0 || n_kv <= 0 || head_dim <= 0 || block_size <= 0) return PKV_ERR_INVALID_ARG;
+  if (n_q % n_kv != 0 || (act != PKV_F32 && act != PKV_BF16)) return PKV_ERR_INVALID_ARG;
+  if (act != PKV_BF16 || head_dim != 128 || block_size != kBlockSize) return PKV_ERR_UNSUPPORTED;
+  if (n_q / n_kv > 64) return PKV_ERR_UNSUPPORTED;
+  return PKV_OK;
+}
+
+static pkv_status kivi_plan(int num_seqs, int n_q, int n_kv, TcPlan* plan, size_t* state_off, size_t* total) {
+  const DecodeShape s{num_seqs, n_q, n_kv, 128, kBlockSize, PKV_BF16, PKV_KIVI2};
+  pkv_status st = plan_tc(s, nullptr, plan);
+  if (st != PKV_OK) return st;
+  // the residual pass's state after the decode's scratch
+  *state_off = (plan->ws_total + 255) / 256 * 256;
+  *total = *state_off + kivi_state_bytes(num_seqs, n_q);
+  return PKV_OK;
+}
+
+size_t pkv_kivi_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size) {
+  if (check_kivi_shape(num_seqs, n_q, n_kv, head_dim, block_size, PKV_BF16) != PKV_OK) return (size_t)-1;
+  if (num_seqs == 0) return 0;
+  TcPlan plan;
+  size_t off = 0, total = 0;
+  if (kivi_plan(num_seqs, n_q, n_kv, &plan, &off, &total) != PKV_OK) return (size_t)-1;
+  return total;
+}
+
+pkv_status pkv_kivi_quantize_blocks(const void* key_rows, const void* value_rows, const int32_t* dst_blocks,
+                                    int64_t num_src_blocks, void* key_cache, void* value_cache, float* k_scale,
+                                    float* v_scale, int n_kv, int head_dim, int block_size, int64_t num_blocks,
+                                    pkv_dtype act_dtype, int32_t* device_error, void* stream) {
+  pkv_status st = check_kivi_shape(1, n_kv, n_kv, head_dim, block_size, act_dtype);
+  if (st != PKV_OK) return st;
+  if (num_src_blocks < 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (num_src_blocks * (int64_t)n_kv > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;
+  if (num_src_blocks == 0) return PKV_OK;
+  if (!key_rows || !value_rows || !dst_blocks || !key_cache || !value_cache || !k_scale || !v_scale)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(key_rows) || !aligned16(value_rows)) return PKV_ERR_INVALID_ARG;
+  return launch_kivi_quantize_blocks(key_rows, value_rows, dst_blocks, num_src_blocks, key_cache, value_cache,
+                                     k_scale, v_scale, n_kv, num_blocks, device_error,
+                                     static_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_kivi_decode(void* out, const void* query, const void* key, const void* value, void* residual_k,
+                           void* residual_v, void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                           const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                           int max_context_len, int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                           int64_t num_blocks, float sm_scale, pkv_dtype act_dtype, float* lse_out, void* workspace,
+                           size_t workspace_bytes, int32_t* device_error, void* stream) {
+  pkv_status st = check_kivi_shape(num_seqs, n_q, n_kv, head_dim, block_size, act_dtype);
+  if (st != PKV_OK) return st;
+  if (max_blocks_per_seq < 0 || max_context_len < 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
+  if (num_blocks * (int64_t)block_size > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  if ((int64_t)num_seqs * n_kv > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PKV_OK;
+  if (!out || !query || !residual_k || !residual_v || !key_cache || !value_cache || !k_scale || !v_scale ||
+      !block_tables || !context_lens)
+    return PKV_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(query) || !aligned16(residual_k) || !aligned16(residual_v) ||
+      !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(k_scale) || !aligned16(v_scale))
+    return PKV_ERR_INVALID_ARG;
+  if ((key == nullptr) != (value == nullptr)) return PKV_ERR_INVALID_ARG;
+  if (key && (!aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
+  if (max_blocks_per_seq == 0 && max_context_len > 0) return PKV_ERR_INVALID_ARG;
+  TcPlan plan;
+  size_t state_off = 0, need = 0;
+  st = kivi_plan(num_seqs, n_q, n_kv, &plan, &state_off, &need);
+  if (st != PKV_OK) return st;
+  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+
+  KiviArgs k{query, key, value, residual_k, residual_v, key_cache, value_cache, k_scale, v_scale, block_tables,
+             max_blocks_per_seq, context_lens,
+             (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * kBlockSize), num_blocks,
+             num_seqs, n_q, n_kv, sm_scale, device_error};
+  PrefixState state;
+  st = launch_kivi_residual(k, static_cast<uint8_t*>(workspace) + state_off, &state, strm);
+  if (st != PKV_OK) return st;
+
+  const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, act_dtype, PKV_KIVI2};
+  TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
+           max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error};
+  a.prefix = state;
+  plan.overlap_prologue = true;  // the decode's prologue overlaps the residual pass
+  return launch_tc(s, plan, a, strm);
 }
 
 pkv_status pkv_copy_blocks(void* key_cache, void* value_cache, float* k_scale, float* v_scale,

@@ -72,6 +72,7 @@ struct TcParams {
   const float* pre_o;    // [n_kv][rows][D], normalised
   const float* pre_lse;  // [n_kv][rows], base 2
   int pre_rows;
+  int whole_blocks;  // only full 16-token blocks are in the pool (2-bit KIVI cache)
   int G, QC, HPC, HG, NCW, stages, units;
   float scale_log2;
   int act_bf16;
@@ -110,7 +111,7 @@ struct AttendSet {
 
 __device__ __forceinline__ AttendSet attend_set(const TcParams& p, int L) {
   AttendSet a;
-  const int nbl = (L + kBlockSize - 1) / kBlockSize;
+  const int nbl = p.whole_blocks ? L / kBlockSize : (L + kBlockSize - 1) / kBlockSize;
   a.nb = a.sink_blocks = a.win_first = nbl;
   a.s_eff = L;
   a.lo_w = 0;
@@ -233,9 +234,10 @@ __device__ void build_prefix(const TcParams& p, int* P, int* wsum) {
 template <int CACHE, int D>
 struct TcTraits {
   static constexpr int kElem = CACHE == TC_BF16 ? 2 : 1;
-  // bytes of one TMA box row: a 128-byte chunk, or an INT4 head row (64 bytes)
-  static constexpr int kChunkBytes = CACHE == TC_INT4 ? D / 2 : 128;
-  static constexpr int kChunks = CACHE == TC_INT4 ? 1 : D * kElem / 128;  // chunks per head row
+  // bytes of one TMA box row: a 128-byte chunk, or a whole INT4 (64 bytes) or
+  // 2-bit (32 bytes) head row
+  static constexpr int kChunkBytes = CACHE == TC_INT4 ? D / 2 : CACHE == TC_KIVI ? D / 4 : 128;
+  static constexpr int kChunks = (CACHE == TC_INT4 || CACHE == TC_KIVI) ? 1 : D * kElem / 128;  // chunks per head row
   static constexpr int kBox = kChunkBytes * 16;                            // one chunk of 16 rows
   static constexpr int kTile = kChunks * kBox;                             // one head's 16-row tile
   static constexpr int kSteps = D / 16;  // k-steps of Q.K and m-tiles of P.V
@@ -245,6 +247,7 @@ struct TcTraits {
 template <int CACHE, int D>
 __device__ __forceinline__ int d_of(int mt, int hi, int g) {
   if constexpr (CACHE == TC_BF16) return mt * 16 + g + 8 * hi;
+  else if constexpr (CACHE == TC_KIVI) return g * 16 + 8 * (mt >> 2) + 4 * hi + (mt & 3);
   else return g * 16 + 2 * mt + hi;
 }
 
@@ -316,7 +319,7 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
 template <int CACHE, int D, int MAXW>
 __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
-                     const TcParams p) {
+                     const __grid_constant__ CUtensorMap smap, const TcParams p) {
   using Tr = TcTraits<CACHE, D>;
   constexpr int KS = Tr::kSteps;
   extern __shared__ uint8_t smem_raw[];
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   if (warp == p.NCW && lane == 0) {
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
+    if constexpr (CACHE == TC_KIVI) prefetch_tensormap(&smap);
   }
   build_prefix(p, P, wsum);  // ends with __syncthreads()
 
@@ -442,6 +446,14 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
               uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
               bulk_load(sc, p.k_scale + sb, bytes, &full[stage]);
               bulk_load(sc + bytes, p.v_scale + sb, bytes, &full[stage]);
+            } else if constexpr (CACHE == TC_KIVI) {
+              // the K scales of the CTA's heads (rows of 32 channels, 128-byte
+              // swizzle) and the V scales of the block's 16 tokens, all heads
+              const int phc = ph >= 0 ? ph : 0;
+              uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
+              tma_load_2d(sc, &smap, 0, (phc * p.n_kv + hgk * p.HPC) * (D / 32), &full[stage]);
+              bulk_load(sc + p.HPC * D * 4, p.v_scale + (size_t)phc * kBlockSize * p.n_kv, 64u * p.n_kv,
+                        &full[stage]);
             }
           }
         }
@@ -466,7 +478,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   const bool head0_ok = qc * 8 + 2 * c < p.G, head1_ok = qc * 8 + 2 * c + 1 < p.G;
 
   // Units with no blocks (empty sequences, empty page lists): out = 0,
-  // lse = -inf.  CTAs share the scan, 32 units per warp step.
+  // lse = -inf, or with a starting state (the KIVI residual pass) that state.
+  // CTAs share the scan, 32 units per warp step.
   for (int u0 = blockIdx.x * 32; u0 < units; u0 += gridDim.x * 32) {
     const int uu = u0 + lane;
     unsigned empty_units = __ballot_sync(0xffffffffu, uu < units && P[uu] == P[uu + 1]);
@@ -478,11 +491,13 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       for (int n = 0; n < 8; ++n) {
         if (qc * 8 + n >= p.G) break;
         const long long row = (long long)s * p.n_q + hg * QH + qbase_local + n;
+        const size_t pre_row = ((size_t)(hg * p.HPC + head_local) * p.pre_rows + (size_t)s * p.G + qc * 8 + n);
         for (int dd = lane; dd < D; dd += 32) {
-          if (p.act_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[row * D + dd] = __float2bfloat16_rn(0.f);
-          else reinterpret_cast<float*>(p.out)[row * D + dd] = 0.f;
+          const float v = p.pre_o ? __ldcg(p.pre_o + pre_row * D + dd) : 0.f;
+          if (p.act_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[row * D + dd] = __float2bfloat16_rn(v);
+          else reinterpret_cast<float*>(p.out)[row * D + dd] = v;
         }
-        if (p.lse_out && lane == 0) p.lse_out[row] = -INFINITY;
+        if (p.lse_out && lane == 0) p.lse_out[row] = p.pre_o ? __ldcg(p.pre_lse + pre_row) * kLn2 : -INFINITY;
       }
     }
   }
@@ -492,7 +507,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   // its range, so it writes those units' new rows (token L-1) into the cache
   // first, one warp per KV head, while the producer starts the ring.  The
   // proxy fence orders these generic stores before the TMA reads of the block.
-  if (p.new_key && qc == 0) {
+  if (CACHE != TC_KIVI && p.new_key && qc == 0) {
     for (int uu = upper_bound_smem(P, units + 1, a) - 1; uu < units && P[uu] < b; ++uu) {
       if (P[uu + 1] > b) break;  // ends past this range: another CTA appends it
       if (P[uu] == P[uu + 1]) continue;
@@ -510,7 +525,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
                            : CACHE == TC_INT4 ? WK_INT4
                            : CACHE == TC_E5M2 ? WK_E5M2
                                               : WK_FP8;
-      if (p.act_bf16) {
+      if constexpr (CACHE == TC_KIVI) {
+        // the KIVI residual pass appends (a row is quantised only with its block)
+      } else if (p.act_bf16) {
         write_row<true, kind, D / 32>(static_cast<const uint8_t*>(p.new_key) + src_row * D * 2, p.key_cache, p.k_scale,
                                       dst_row, kv, p.n_kv, lane);
         write_row<true, kind, D / 32>(static_cast<const uint8_t*>(p.new_value) + src_row * D * 2, p.value_cache,
@@ -648,6 +665,39 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       sa[1] = ((float)(ah[1] - ch1) + (float)(al[1] - cl1) * (1.f / 254.f)) * qs1;
       sa[2] = ((float)(ah[2] - ch0) + (float)(al[2] - cl0) * (1.f / 254.f)) * qs0;
       sa[3] = ((float)(ah[3] - ch1) + (float)(al[3] - cl1) * (1.f / 254.f)) * qs1;
+    } else if constexpr (CACHE == TC_KIVI) {
+      // 2-bit codes, 32-byte rows: lane (g, c) reads bytes 8c .. 8c+7 (dims
+      // 32c .. 32c+31) of rows g and g+8.  The block's per-channel K scales
+      // fold into the query: B = q * scale (f16) for the lane's channels, row
+      // 4 * head_local + c of the scale tile, whose 16-byte chunk kk sits at
+      // kk ^ (row & 7) under the 128-byte swizzle (conflict-free).
+      const uint2 r0 = lds64(kt + g * 32 + 8 * c), r1 = lds64(kt + (g + 8) * 32 + 8 * c);
+      const int srow = 4 * head_local + c;
+      const uint32_t ksb = smem_addr(st + 2 * p.HPC * Tr::kTile) + srow * 128;
+      float f[8][4];
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint4 w = lds128(ksb + ((uint32_t)(kk ^ (srow & 7)) << 4));
+        f[kk][0] = __uint_as_float(w.x);
+        f[kk][1] = __uint_as_float(w.y);
+        f[kk][2] = __uint_as_float(w.z);
+        f[kk][3] = __uint_as_float(w.w);
+      }
+      // k-step ks: word m = ks >> 2 of the row, byte pair (t, t + 2) with
+      // t = (ks >> 1) & 1, codes s0 = 2 (ks & 1) and s0 + 1 of each byte:
+      // dims 32c + 16m + 4t + s and 32c + 16m + 8 + 4t + s
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int m = ks >> 2, t = (ks >> 1) & 1, s0 = 2 * (ks & 1);
+        const uint32_t w0 = m ? r0.y : r0.x, w1 = m ? r1.y : r1.x;
+        const int sh = 2 * s0 + 8 * t;
+        const uint32_t af[4] = {i2x2_to_f16x2(w0 >> sh), i2x2_to_f16x2(w1 >> sh), i2x2_to_f16x2(w0 >> (sh + 2)),
+                                i2x2_to_f16x2(w1 >> (sh + 2))};
+        const uint32_t b0 = hmul2_u32(qf[ks][0], pack_f16(f[4 * m + t][s0], f[4 * m + t + 2][s0]));
+        const uint32_t b1 = hmul2_u32(qf[ks][1], pack_f16(f[4 * m + t][s0 + 1], f[4 * m + t + 2][s0 + 1]));
+        if (ks & 1) mma_f16(sb, af, b0, b1);
+        else mma_f16(sa, af, b0, b1);
+      }
     } else if constexpr (CACHE == TC_INT8) {
       // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each); k-step
       // kk takes the bytes of dims 32c + 8kk + {0..3} and {4..7} as they are stored
@@ -710,6 +760,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       sc1 *= ksm[t1 * p.n_kv + kvh];
       vsc[0] = vsm[t0 * p.n_kv + kvh];
       vsc[1] = vsm[t1 * p.n_kv + kvh];
+    } else if constexpr (CACHE == TC_KIVI) {
+      const float* vsm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile + p.HPC * D * 4);
+      vsc[0] = vsm[t0 * p.n_kv + kvh];
+      vsc[1] = vsm[t1 * p.n_kv + kvh];
     } else if constexpr (tc_fp8(CACHE)) {
       sc0 *= head_k_scale;
       sc1 *= head_k_scale;
@@ -729,7 +783,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     if constexpr (CACHE == TC_BF16) {
       pb0 = movmatrix_trans(pack_bf16(pr[0], pr[1]));
       pb1 = movmatrix_trans(pack_bf16(pr[2], pr[3]));
-    } else if constexpr (tc_row_scaled(CACHE)) {
+    } else if constexpr (tc_v_row_scaled(CACHE)) {
       pb0 = movmatrix_trans(pack_f16(ok0 ? pr[0] * vsc[0] : 0.f, ok0 ? pr[1] * vsc[0] : 0.f));
       pb1 = movmatrix_trans(pack_f16(ok1 ? pr[2] * vsc[1] : 0.f, ok1 ? pr[3] * vsc[1] : 0.f));
     } else {
@@ -753,6 +807,25 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         af[2] &= mhi;
         af[3] &= mhi;
         mma_bf16(acc[mt], af, pb0, pb1);
+      }
+    } else if constexpr (CACHE == TC_KIVI) {
+      // lane (g, c) reads word g (dims 16g .. 16g+15, byte j = dims 16g + 4j ..
+      // + 3) of token rows 2c, 2c+1, 2c+8, 2c+9 (32-byte rows).  Bytes (2J,
+      // 2J+1) of the row pair side by side; code s of byte 2J is dim 16g + 8J
+      // + s (m-tile row g), of byte 2J+1 dim 16g + 8J + 4 + s (row g+8)
+      const uint32_t vb = vt + 64 * c + 4 * g;
+      const uint32_t x0 = lds32(vb), y0 = lds32(vb + 32), x1 = lds32(vb + 256), y1 = lds32(vb + 288);
+#pragma unroll
+      for (int J = 0; J < 2; ++J) {
+        const uint32_t sel = J ? 0x7632u : 0x5410u;
+        const uint32_t z0 = prmt(x0, y0, sel), z1 = prmt(x1, y1, sel);
+#pragma unroll
+        for (int s2 = 0; s2 < 4; ++s2) {
+          // codes are finite and masked tokens carry P = 0: no V mask needed
+          const uint32_t af[4] = {i2x2_to_f16x2(z0 >> (2 * s2)), i2x2_to_f16x2(z0 >> (2 * s2 + 8)),
+                                  i2x2_to_f16x2(z1 >> (2 * s2)), i2x2_to_f16x2(z1 >> (2 * s2 + 8))};
+          mma_f16(acc[4 * J + s2], af, pb0, pb1);
+        }
       }
     } else if constexpr (CACHE == TC_INT4) {
       // lane (g, c) reads dims 16g .. 16g+15 (8 bytes at byte 8g, in chunk g/2)
@@ -1039,6 +1112,32 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           cl1 = 8 * __shfl_sync(0xffffffffu, lsum, 8 * c + 4);
         }
       }
+      if constexpr (CACHE == TC_KIVI) {
+        // this lane's dims 32c .. 32c+31 of query head g as f16 pairs in the
+        // order of the 2-bit K fragments (see block_scores); the block's
+        // channel scales multiply them per block
+        const int kvq = hg * p.HPC + head_local;
+        const bool q_ok = qc * 8 + g < p.G;
+        const size_t qoff = ((size_t)s * p.n_q + kvq * p.G + qc * 8 + g) * D + 32 * c;
+        const uint4* q4 = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.query) + qoff);
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 w = q_ok ? __ldg(q4 + i) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[8 * i + 2 * k] = __uint_as_float(wv[k] << 16);
+            x[8 * i + 2 * k + 1] = __uint_as_float(wv[k] & 0xFFFF0000u);
+          }
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int e = 16 * (ks >> 2) + 4 * ((ks >> 1) & 1) + 2 * (ks & 1);
+          qf[ks][0] = pack_f16(x[e], x[e + 8]);
+          qf[ks][1] = pack_f16(x[e + 1], x[e + 9]);
+        }
+      }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       m0 = m1 = -INFINITY;
@@ -1153,11 +1252,11 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Rank-3 view of a cache pool [num_blocks * 16 rows][n_kv * head_dim * elem bytes]
-// as (128-byte chunk elements, chunk index, row), box = 1 chunk x 16 rows.
-// Rank-3 view of a pool: (elements of one chunk, chunk index, token row).  A
-// chunk is 128 bytes (BF16 / INT8 / FP8 rows), or a whole 64-byte INT4 head row
-// (64-byte swizzle).
+// Rank-3 view of a cache pool [num_blocks * 16 rows][n_kv * head_dim * elem
+// bytes] as (elements of one chunk, chunk index, token row), box = 1 chunk x 16
+// rows.  A chunk is 128 bytes (BF16 / INT8 / FP8 rows, 128-byte swizzle), or a
+// whole head row: 64 bytes of INT4 (64-byte swizzle) or 32 bytes of 2-bit
+// codes (no swizzle).
 pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes_i,
                               int64_t rows) {
   auto fn = encode_fn();
@@ -1170,15 +1269,33 @@ pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  chunk_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  chunk_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : chunk_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                      : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return driver_fail((int)r, "cuTensorMapEncodeTiled");
   return PKV_OK;
 }
 
+// The 2-bit cache's K scales [num_blocks * n_kv * 4 rows][32 floats] as a
+// rank-2 map, box = 32 floats x (4 * heads_per_cta) rows, 128-byte swizzle.
+static pkv_status make_kivi_scale_map(CUtensorMap* map, const float* k_scale, int64_t num_blocks, int n_kv, int hpc) {
+  auto fn = encode_fn();
+  if (!fn) return driver_fail(-1, "cuTensorMapEncodeTiled entry point");
+  cuuint64_t dims[2] = {32, (cuuint64_t)num_blocks * n_kv * 4};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {32, (cuuint32_t)(4 * hpc)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(k_scale), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return driver_fail((int)r, "cuTensorMapEncodeTiled(k_scale)");
+  return PKV_OK;
+}
+
 template <int CACHE, int D, int MAXW>
-static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const TcParams& prm,
-                                 cudaStream_t stream) {
+static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
+                                 const TcParams& prm, cudaStream_t stream) {
   auto kern = decode_tc_kernel<CACHE, D, MAXW>;
   static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
   if ((int)plan.smem_bytes > configured_bytes) {
@@ -1196,7 +1313,7 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = plan.overlap_prologue ? 1 : 0;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, prm);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, sm, prm);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_tc_kernel launch");
 
@@ -1232,23 +1349,29 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
 // Up to 8 consumer warps use the variant whose launch bound leaves ~220
 // registers per thread; wider CTAs take the 16-warp variant.
 template <int CACHE, int D>
-static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const TcParams& prm,
-                             cudaStream_t stream) {
-  if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, prm, stream);
-  return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, prm, stream);
+static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
+                             const TcParams& prm, cudaStream_t stream) {
+  if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, sm, prm, stream);
+  return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, sm, prm, stream);
 }
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream) {
   const int elem = plan.cache_kind == TC_BF16 ? 2 : 1;
-  const bool int4 = plan.cache_kind == TC_INT4;
-  const int row_bytes = int4 ? s.n_kv * s.head_dim / 2 : s.n_kv * s.head_dim * elem;
-  const int chunk_bytes = int4 ? s.head_dim / 2 : 128;
+  const bool int4 = plan.cache_kind == TC_INT4, kivi = plan.cache_kind == TC_KIVI;
+  const int row_bytes = int4 ? s.n_kv * s.head_dim / 2 : kivi ? s.n_kv * s.head_dim / 4 : s.n_kv * s.head_dim * elem;
+  const int chunk_bytes = int4 ? s.head_dim / 2 : kivi ? s.head_dim / 4 : 128;
   const int64_t rows = a.num_blocks * kBlockSize;
-  CUtensorMap km, vm;
+  CUtensorMap km, vm, sm;
   pkv_status st = make_pool_map(&km, a.key_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
   st = make_pool_map(&vm, a.value_cache, elem, chunk_bytes, row_bytes, rows);
   if (st != PKV_OK) return st;
+  if (kivi) {
+    st = make_kivi_scale_map(&sm, a.k_scale, a.num_blocks, s.n_kv, plan.HPC);
+    if (st != PKV_OK) return st;
+  } else {
+    sm = km;  // unused
+  }
   PrefixState pre = a.prefix;
   if (a.skip_blocks > 0 && a.prefix_ws) {
     // shared prefix first; the decode over the sequences' own blocks then
@@ -1290,6 +1413,7 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.pre_o = pre.o;
   prm.pre_lse = pre.lse;
   prm.pre_rows = pre.rows;
+  prm.whole_blocks = kivi ? 1 : 0;
   prm.G = plan.G;
   prm.QC = plan.QC;
   prm.HPC = plan.HPC;
@@ -1303,13 +1427,14 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.tx_bytes = plan.tx_bytes;
 
   if (plan.cache_kind == TC_BF16) {
-    if (s.head_dim == 64) return launch_one<TC_BF16, 64>(plan, km, vm, prm, stream);
-    return launch_one<TC_BF16, 128>(plan, km, vm, prm, stream);
+    if (s.head_dim == 64) return launch_one<TC_BF16, 64>(plan, km, vm, sm, prm, stream);
+    return launch_one<TC_BF16, 128>(plan, km, vm, sm, prm, stream);
   }
-  if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, prm, stream);
-  if (plan.cache_kind == TC_INT4) return launch_one<TC_INT4, 128>(plan, km, vm, prm, stream);
-  if (plan.cache_kind == TC_E5M2) return launch_one<TC_E5M2, 128>(plan, km, vm, prm, stream);
-  return launch_one<TC_FP8, 128>(plan, km, vm, prm, stream);
+  if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, sm, prm, stream);
+  if (plan.cache_kind == TC_INT4) return launch_one<TC_INT4, 128>(plan, km, vm, sm, prm, stream);
+  if (plan.cache_kind == TC_E5M2) return launch_one<TC_E5M2, 128>(plan, km, vm, sm, prm, stream);
+  if (plan.cache_kind == TC_KIVI) return launch_one<TC_KIVI, 128>(plan, km, vm, sm, prm, stream);
+  return launch_one<TC_FP8, 128>(plan, km, vm, sm, prm, stream);
 }
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -1320,10 +1445,14 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
                   : s.cache == PKV_INT8      ? TC_INT8
                   : s.cache == PKV_INT4      ? TC_INT4
                   : s.cache == PKV_FP8_E5M2 ? TC_E5M2
+                  : s.cache == PKV_KIVI2    ? TC_KIVI
                                              : TC_FP8;
   const int elem = pl.cache_kind == TC_BF16 ? 2 : 1;
-  pl.chunks = pl.cache_kind == TC_INT4 ? 1 : s.head_dim * elem / 128;
-  const size_t tile_bytes = pl.cache_kind == TC_INT4 ? (size_t)s.head_dim / 2 * 16 : (size_t)pl.chunks * 2048;
+  const bool kivi = pl.cache_kind == TC_KIVI;
+  pl.chunks = (pl.cache_kind == TC_INT4 || kivi) ? 1 : s.head_dim * elem / 128;
+  const size_t tile_bytes = pl.cache_kind == TC_INT4 ? (size_t)s.head_dim / 2 * 16
+                            : kivi                   ? (size_t)s.head_dim / 4 * 16
+                                                     : (size_t)pl.chunks * 2048;
   pl.G = s.n_q / s.n_kv;
   pl.QC = (pl.G + 7) / 8;
   const int want_hpc = tuning ? tuning->heads_per_cta : 0;
@@ -1348,7 +1477,10 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.HG = s.n_kv / pl.HPC;
   pl.NCW = pl.HPC * pl.QC;
   pl.units = s.num_seqs * pl.HG;
-  pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * tile_bytes + scale_bytes);
+  // KIVI: the K scales of the CTA's heads (head_dim floats each) and the V
+  // scales of the block's tokens, all heads
+  const size_t kivi_scales = kivi ? (size_t)pl.HPC * s.head_dim * 4 + 64 * (size_t)s.n_kv : 0;
+  pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * tile_bytes + scale_bytes + kivi_scales);
   pl.stage_bytes = (uint32_t)align_up(pl.tx_bytes, 1024);
 
   const int sms = device_sm_count();

@@ -18,9 +18,12 @@ constexpr int kTargetCtasPerSm = 4;
 constexpr size_t kSmemPerSm = 233472;  // 228 KB of shared memory per SM
 
 // Cache kinds of the tensor-core decode kernel.
-enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2, TC_E5M2 = 3, TC_INT4 = 4 };
+enum TcCache : int { TC_BF16 = 0, TC_INT8 = 1, TC_FP8 = 2, TC_E5M2 = 3, TC_INT4 = 4, TC_KIVI = 5 };
 __host__ __device__ constexpr bool tc_fp8(int c) { return c == TC_FP8 || c == TC_E5M2; }          // one scale per KV head
 __host__ __device__ constexpr bool tc_row_scaled(int c) { return c == TC_INT8 || c == TC_INT4; }  // one scale per (token, head)
+// V scaled per (token, head): the row-scaled formats and the 2-bit KIVI cache,
+// whose K scales are per (block, head, channel)
+__host__ __device__ constexpr bool tc_v_row_scaled(int c) { return tc_row_scaled(c) || c == TC_KIVI; }
 
 struct DecodeShape {
   int num_seqs, n_q, n_kv, head_dim, block_size;
@@ -90,6 +93,36 @@ struct TcArgs {
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);
+
+// 2-bit KIVI cache (kivi.cu).  The residual pass appends the new rows (if
+// any) to the BF16 residual of each sequence, quantises a residual that became
+// a full block into the pool, and leaves per (KV head, row = s * G + head in
+// group) the normalised output and base-2 lse over the residual rows, which the
+// decode over the quantised full blocks starts from.
+struct KiviArgs {
+  const void* query;
+  const void* new_key;    // [num_seqs, n_kv, 128] bf16 or null
+  const void* new_value;
+  void* residual_k;       // [num_seqs, 16, n_kv, 128] bf16
+  void* residual_v;
+  void* key_cache;        // [num_blocks, 16, n_kv, 32] bytes
+  void* value_cache;
+  float* k_scale;         // [num_blocks, n_kv, 128]
+  float* v_scale;         // [num_blocks, 16, n_kv]
+  const int32_t* block_tables;
+  int max_blocks_per_seq;
+  const int32_t* context_lens;
+  int cap_len;
+  int64_t num_blocks;
+  int num_seqs, n_q, n_kv;
+  float sm_scale;
+  int32_t* device_error;
+};
+size_t kivi_state_bytes(int num_seqs, int n_q);
+pkv_status launch_kivi_residual(const KiviArgs& a, void* state_ws, PrefixState* state, cudaStream_t stream);
+pkv_status launch_kivi_quantize_blocks(const void* key_rows, const void* value_rows, const int32_t* dst_blocks,
+                                       int64_t n, void* key_cache, void* value_cache, float* k_scale, float* v_scale,
+                                       int n_kv, int64_t num_blocks, int32_t* device_error, cudaStream_t stream);
 
 size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks);
 pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes, int64_t rows);

@@ -81,6 +81,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// Tiled TMA load of one box of a rank-2 tensor map (same completion rules).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Contiguous bulk copy global -> shared (16-byte aligned, size a multiple of 16).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_addr(dst)),
@@ -222,6 +231,28 @@ __device__ __forceinline__ uint32_t i4x2_to_f16x2(uint32_t t) {
   __half2 v = *reinterpret_cast<const __half2*>(&h);
   v = __hsub2(v, __half2half2(__ushort_as_half(0x6408)));  // 0x6408 = 1032.0
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Two 2-bit two's-complement codes at bits [1:0] and [17:16] of t (other bits
+// ignored) -> f16x2 of the codes, exactly.  XOR with 2 turns a code c into
+// c + 2 in [0, 3]; ORed into the mantissa of 1024.0 it reads as 1026 + c, and
+// subtracting 1026 leaves c.  One LOP3 and one HSUB2.
+__device__ __forceinline__ uint32_t i2x2_to_f16x2(uint32_t t) {
+  const uint32_t h = (t & 0x00030003u) ^ 0x64026402u;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __half2half2(__ushort_as_half(0x6402)));  // 0x6402 = 1026.0
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {

@@ -17,7 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
-PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3, PKV_FP8_E5M2, PKV_INT4 = 0, 1, 2, 3, 4, 5
+PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3, PKV_FP8_E5M2, PKV_INT4, PKV_KIVI2 = 0, 1, 2, 3, 4, 5, 6
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype", 3: "workspace missing or too small", 4: "CUDA error"}
 DEVERR_SLOT_RANGE, DEVERR_BLOCK_RANGE, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 
@@ -28,6 +28,7 @@ _CACHE_DTYPES = {
     "fp8_e4m3": PKV_FP8_E4M3,
     "fp8_e5m2": PKV_FP8_E5M2,
     "int4": PKV_INT4,  # pools hold uint8 bytes, two codes each: pass cache_dtype="int4"
+    "kivi2": PKV_KIVI2,  # uint8 pools, four 2-bit codes a byte (block movers only; decode via kivi_decode)
 }
 
 
@@ -95,6 +96,13 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                                              i32, i32, i64, f32, i32, i32, i32, vp, vp, sz, vp, vp]
     lib.pkv_paged_attention_decode_shared_prefix.restype = i32
+    lib.pkv_kivi_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.pkv_kivi_workspace_size.restype = sz
+    lib.pkv_kivi_quantize_blocks.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]
+    lib.pkv_kivi_quantize_blocks.restype = i32
+    lib.pkv_kivi_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, i32,
+                                    i64, f32, i32, vp, vp, sz, vp, vp]
+    lib.pkv_kivi_decode.restype = i32
     lib.pkv_status_string.argtypes = [i32]
     lib.pkv_status_string.restype = ctypes.c_char_p
     lib.pkv_last_cuda_error.argtypes = []
@@ -282,6 +290,8 @@ def copy_blocks(key_cache, value_cache, block_mapping, k_scale=None, v_scale=Non
     code = cache_code(key_cache, cache_dtype)
     if code == PKV_INT4:
         d *= 2
+    elif code == PKV_KIVI2:
+        d *= 4
     st = lib.pkv_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_mapping),
                              block_mapping.shape[0], n_kv, d, bs, nb, code, _ptr(device_error),
                              stream if stream is not None else _stream(key_cache.device))
@@ -295,6 +305,8 @@ def swap_blocks(src_key, src_value, dst_key, dst_value, block_mapping, src_k_sca
     code = cache_code(src_key, cache_dtype)
     if code == PKV_INT4:
         d *= 2
+    elif code == PKV_KIVI2:
+        d *= 4
     dev = device if device is not None else (src_key.device if src_key.is_cuda else dst_key.device)
     st = lib.pkv_swap_blocks(_ptr(src_key), _ptr(src_value), _ptr(src_k_scale), _ptr(src_v_scale), snb,
                              _ptr(dst_key), _ptr(dst_value), _ptr(dst_k_scale), _ptr(dst_v_scale), dst_key.shape[0],
@@ -435,4 +447,47 @@ def paged_decode_step_window(out, query, key, value, key_cache, value_cache, blo
         _ptr(lse_out), _ptr(workspace), ws_bytes, _ptr(device_error), _stream(query.device),
     )
     _check(st, "pkv_paged_decode_step_window")
+    return out
+
+
+def kivi_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size) -> int:
+    n = lib.pkv_kivi_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size)
+    if n == ctypes.c_size_t(-1).value:
+        raise PkvError(2, "pkv_kivi_workspace_size")
+    return int(n)
+
+
+def kivi_quantize_blocks(key_rows, value_rows, dst_blocks, key_cache, value_cache, k_scale, v_scale,
+                         device_error=None):
+    """Quantise whole blocks ``key_rows``/``value_rows`` [n, 16, n_kv, d] (bf16) into the 2-bit pools
+    (uint8 [num_blocks, 16, n_kv, d / 4]) at physical blocks ``dst_blocks`` [n] (int32, -1 skips)."""
+    n, block_size, n_kv, d = key_rows.shape
+    st = lib.pkv_kivi_quantize_blocks(
+        _ptr(key_rows), _ptr(value_rows), _ptr(dst_blocks), n, _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
+        _ptr(v_scale), n_kv, d, block_size, key_cache.shape[0], act_code(key_rows), _ptr(device_error),
+        _stream(key_rows.device),
+    )
+    _check(st, "pkv_kivi_quantize_blocks")
+
+
+def kivi_decode(out, query, residual_k, residual_v, key_cache, value_cache, k_scale, v_scale, block_tables,
+                context_lens, max_context_len: int, key=None, value=None, sm_scale: float | None = None,
+                lse_out=None, workspace=None, device_error=None):
+    """Decode over a 2-bit KIVI cache (full blocks in the pools, the partial last block in the BF16
+    residual [S, 16, n_kv, d]); ``key``/``value`` [S, n_kv, d] append token L-1 first."""
+    S, n_q, d = query.shape
+    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if workspace is None:
+        nbytes = kivi_workspace_size(S, n_q, n_kv, d, block_size)
+        workspace = workspace_for(nbytes, query.device) if nbytes else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = lib.pkv_kivi_decode(
+        _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(residual_k), _ptr(residual_v), _ptr(key_cache),
+        _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables), block_tables.shape[1],
+        _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks, float(sm_scale),
+        act_code(query), _ptr(lse_out), _ptr(workspace), ws_bytes, _ptr(device_error), _stream(query.device),
+    )
+    _check(st, "pkv_kivi_decode")
     return out

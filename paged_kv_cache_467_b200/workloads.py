@@ -31,7 +31,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-DTYPES = ("f32", "bf16", "int8", "fp8_e4m3", "fp8_e5m2", "int4")
+DTYPES = ("f32", "bf16", "int8", "fp8_e4m3", "fp8_e5m2", "int4", "kivi2")
 FP8_MAX = {"fp8_e4m3": 448.0, "fp8_e5m2": 57344.0}  # largest finite value of each format
 
 
@@ -404,5 +404,6 @@ CONFIGS = {
     "fp8": lambda: quantized("fp8_e4m3", seed=5),
     "fp8_e5m2": lambda: quantized("fp8_e5m2", seed=6),
     "int4": lambda: quantized("int4", seed=7),
+    "kivi2": lambda: quantized("kivi2", seed=8),
     "window": sliding_window,
 }

@@ -146,3 +146,39 @@ def test_quest_host_validation(lib):
     assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 8, 2, 128, 16, 16, 1, 1, 0, FAKE, FAKE, None, None) == 1
     assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 8, 2, 128, 16, 16, 1, 1, 4, FAKE, None, None, None) == 1
     assert sel(FAKE, FAKE, FAKE, FAKE, 8, FAKE, 100, 2, 6, 4, 128, 16, 16, 1, 1, 4, FAKE, FAKE, None, None) == 1
+
+
+def _kivi_decode(lib, **kw):
+    a = dict(out=FAKE, q=FAKE, key=None, value=None, rk=FAKE, rv=FAKE, kc=FAKE, vc=FAKE, ks=FAKE, vs=FAKE, bt=FAKE,
+             mb=8, cl=FAKE, mcl=100, S=2, nq=8, nkv=2, d=128, bs=16, nb=16, scale=0.1, act=1, lse=None, ws=FAKE,
+             wsb=1 << 24, err=None)
+    a.update(kw)
+    return lib.pkv_kivi_decode(a["out"], a["q"], a["key"], a["value"], a["rk"], a["rv"], a["kc"], a["vc"], a["ks"],
+                               a["vs"], a["bt"], a["mb"], a["cl"], a["mcl"], a["S"], a["nq"], a["nkv"], a["d"],
+                               a["bs"], a["nb"], a["scale"], a["act"], a["lse"], a["ws"], a["wsb"], a["err"], None)
+
+
+def test_kivi_host_validation(lib):
+    none = ctypes.c_size_t(-1).value
+    assert lib.pkv_kivi_workspace_size(0, 8, 2, 128, 16) == 0
+    assert lib.pkv_kivi_workspace_size(2, 8, 2, 64, 16) == none  # head_dim 128 only
+    assert lib.pkv_kivi_workspace_size(2, 6, 4, 128, 16) == none
+    assert _kivi_decode(lib, S=0) == 0
+    assert _kivi_decode(lib, key=FAKE) == 1  # key without value
+    assert _kivi_decode(lib, key=FAKE, value=FAKE + 8) == 1  # misaligned
+    assert _kivi_decode(lib, rk=None) == 1  # the residual is required
+    assert _kivi_decode(lib, ks=FAKE + 4) == 1
+    assert _kivi_decode(lib, d=64) == 2
+    assert _kivi_decode(lib, act=0) == 2  # BF16 activations only
+    assert _kivi_decode(lib, act=2) == 1
+    assert _kivi_decode(lib, nq=6, nkv=4) == 1
+    assert _kivi_decode(lib, bs=32) == 2
+    assert _kivi_decode(lib, mb=0) == 1  # context but no table
+    q = lib.pkv_kivi_quantize_blocks
+    assert q(FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 1, None, None) == 0
+    assert q(None, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 1, None, None) == 1
+    assert q(FAKE, FAKE, FAKE, 3, FAKE, FAKE, None, FAKE, 2, 128, 16, 8, 1, None, None) == 1
+    assert q(FAKE + 2, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 1, None, None) == 1
+    assert q(FAKE, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 64, 16, 8, 1, None, None) == 2
+    assert q(FAKE, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 0, None, None) == 2
+    assert q(FAKE, FAKE, FAKE, -1, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 1, None, None) == 1
