@@ -366,10 +366,10 @@ def run_b200(args, rank, world, local):
             raise SystemExit("the 2-bit KIVI cache appends inside its residual pass: no unfused step")
         # every pool block quantised from N(0,1) rows by the library's block quantiser,
         # and N(0,1) residual rows (the partial last block of each sequence)
-        kc = torch.empty((w.num_blocks, bs, nkv, d // 4), device=dev, dtype=torch.uint8)
+        kc = torch.empty((w.num_blocks, nkv, bs, d // 4), device=dev, dtype=torch.uint8)
         vc = torch.empty_like(kc)
         ks = torch.empty((w.num_blocks, nkv, d), device=dev)
-        vs = torch.empty((w.num_blocks, bs, nkv), device=dev)
+        vs = torch.empty((w.num_blocks, nkv, bs), device=dev)
         for b0 in range(0, w.num_blocks, 4096):
             nblk = min(4096, w.num_blocks - b0)
             kk = torch.randn((nblk, bs, nkv, d), device=dev, generator=gen).to(torch.bfloat16)

@@ -41,10 +41,11 @@ typedef enum {
   PKV_INT4 = 5,     /* signed 4-bit codes, two per byte (element 2j in the low
                        nibble of byte j), one float scale per (token, KV head);
                        cache only, pools [num_blocks, block_size, n_kv, head_dim/2] */
-  PKV_KIVI2 = 6     /* 2-bit KIVI cache (pkv_kivi_* calls only): signed 2-bit
-                       codes, four per byte (element 4j + m in bits [2m, 2m+1]
-                       of byte j), K scaled per (block, KV head, channel), V per
-                       (token, KV head); pools [num_blocks, block_size, n_kv, head_dim/4] */
+  PKV_KIVI2 = 6     /* 2-bit KIVI cache (pkv_kivi_* calls and the block movers):
+                       signed 2-bit codes, four per byte (element 4j + m in bits
+                       [2m, 2m+1] of byte j), K scaled per (block, KV head,
+                       channel), V per (token, KV head); pools [num_blocks, n_kv,
+                       block_size, head_dim/4] (layout under pkv_kivi_decode) */
 } pkv_dtype;
 
 typedef enum {
@@ -403,11 +404,12 @@ pkv_status pkv_paged_attention_decode_static(void* out, const void* query, const
  * last block, in order, in rows [0, L % 16) of its BF16 residual.
  *
  * Layouts (row-major, innermost last):
- *   key_cache, value_cache  device uint8 [num_blocks, 16, n_kv, head_dim / 4]:
- *                           element 4j + m of a row in bits [2m, 2m+1] of byte
- *                           j, two's complement
+ *   key_cache, value_cache  device uint8 [num_blocks, n_kv, 16, head_dim / 4]
+ *                           (head-major inside a block: one (block, head) tile
+ *                           is 512 contiguous bytes): element 4j + m of a token
+ *                           row in bits [2m, 2m+1] of byte j, two's complement
  *   k_scale                 device float [num_blocks, n_kv, head_dim]
- *   v_scale                 device float [num_blocks, 16, n_kv]
+ *   v_scale                 device float [num_blocks, n_kv, 16]
  *   residual_k, residual_v  device bf16 [num_seqs, 16, n_kv, head_dim]; row r of
  *                           sequence s holds position 16 * floor(L / 16) + r
  * BF16 activations, head_dim 128, block_size 16, n_q / n_kv <= 64.  All
@@ -470,7 +472,7 @@ pkv_status pkv_kivi_decode(void* out, const void* query, const void* key, const 
  *   key_cache, value_cache  device, [num_blocks, block_size, n_kv, head_dim], cache_dtype
  *   k_scale, v_scale        INT8 / INT4: device [num_blocks, block_size, n_kv]; KIVI2:
  *                           k_scale [num_blocks, n_kv, head_dim], v_scale [num_blocks,
- *                           block_size, n_kv]; NULL otherwise (FP8 per-head scales
+ *                           n_kv, block_size]; NULL otherwise (FP8 per-head scales
  *                           belong to no block)
  *   block_mapping           device (or mapped host) int64 [num_pairs, 2] = (src, dst)
  * Destinations must be distinct and no block may be both a source and a

@@ -490,6 +490,7 @@ pkv_status pkv_kivi_decode(void* out, const void* query, const void* key, const 
   if (st != PKV_OK) return st;
   if (max_blocks_per_seq < 0 || max_context_len < 0 || num_blocks < 0) return PKV_ERR_INVALID_ARG;
   if (num_blocks * (int64_t)block_size > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  if (num_blocks * (int64_t)n_kv * 4 > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;  // K-scale rows (int32 TMA coordinate)
   if ((int64_t)num_seqs * n_kv > 0x7FFFFFFFLL) return PKV_ERR_UNSUPPORTED;
   if (num_seqs == 0) return PKV_OK;
   if (!out || !query || !residual_k || !residual_v || !key_cache || !value_cache || !k_scale || !v_scale ||

@@ -149,7 +149,9 @@ __device__ __forceinline__ int logical_block(const AttendSet& a, int j) {
 __device__ __forceinline__ uint32_t token_mask(const AttendSet& a, int L, int lb) {
   const int base = lb * kBlockSize;
   auto below = [](int n) -> uint32_t { return n <= 0 ? 0u : (n >= kBlockSize ? 0xFFFFu : (1u << n) - 1u); };
-  return below(L - base) & (below(a.s_eff - base) | (0xFFFFu & ~below(a.lo_w - base)));
+  uint32_t m = below(L - base);
+  if (a.s_eff < L || a.lo_w > 0) m &= below(a.s_eff - base) | (0xFFFFu & ~below(a.lo_w - base));
+  return m;
 }
 
 // Blocks of unit u (sequence length L): its attended set or, with a page list,
@@ -316,8 +318,8 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
   }
 }
 
-template <int CACHE, int D, int MAXW>
-__global__ void __launch_bounds__((MAXW + 1) * 32, 1)
+template <int CACHE, int D, int MAXW, int MINB>
+__global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
     decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                      const __grid_constant__ CUtensorMap smap, const TcParams p) {
   using Tr = TcTraits<CACHE, D>;
@@ -399,6 +401,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   if (warp == p.NCW) {
     if (a >= b) return;
     int it = 0;
+    int pstage = 0;       // ring stage of block `it`
+    uint32_t ppass = 0;   // parity of the ring pass of block `it`
     bool abort = false, appended = false;
     for (int base = a; base < b && !abort; base += 32) {
       int phys, hg, unit_last;
@@ -419,8 +423,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
         const int lastk = __shfl_sync(0xffffffffu, unit_last, k);
         int ok = 1;
         if (lane == 0) {
-          const int stage = it % p.stages;
-          if (it >= p.stages && !mbar_wait(&empty[stage], ((it / p.stages) & 1) ^ 1)) {
+          const int stage = pstage;
+          if (it >= p.stages && !mbar_wait(&empty[stage], ppass ^ 1u)) {
             flag_error(p.err, DEVERR_TIMEOUT);
             ok = 0;
           } else if (p.new_key && lastk && !appended && !(appended = mbar_wait(append_done, 0))) {
@@ -430,14 +434,29 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
           } else {
             uint8_t* st = smem + (size_t)stage * p.stage_bytes;
             mbar_arrive_expect_tx(&full[stage], p.tx_bytes);
-            const int row = ph * kBlockSize;  // -16 for a rejected entry: the TMA zero-fills it
+            if constexpr (CACHE == TC_KIVI) {
+              // head-major pools: the (block, head) tiles of the CTA's heads are
+              // contiguous, as are their K scales and V scales (a rejected entry
+              // reads block 0; its error bit is set)
+              const size_t tile0 = (size_t)(ph >= 0 ? ph : 0) * p.n_kv + hgk * p.HPC;
+              const uint32_t codes = p.HPC * Tr::kTile;
+              bulk_load(st, static_cast<const uint8_t*>(p.key_cache) + tile0 * Tr::kTile, codes, &full[stage]);
+              bulk_load(st + codes, static_cast<const uint8_t*>(p.value_cache) + tile0 * Tr::kTile, codes,
+                        &full[stage]);
+              // K scales: rows of 32 channels, 128-byte swizzle; V scales: 16 per head
+              uint8_t* sc = st + 2 * codes;
+              tma_load_2d(sc, &smap, 0, (int)(tile0 * (D / 32)), &full[stage]);
+              bulk_load(sc + p.HPC * D * 4, p.v_scale + tile0 * kBlockSize, 64u * p.HPC, &full[stage]);
+            } else {
+              const int row = ph * kBlockSize;  // -16 for a rejected entry: the TMA zero-fills it
 #pragma unroll 1
-            for (int hl = 0; hl < p.HPC; ++hl) {
+              for (int hl = 0; hl < p.HPC; ++hl) {
 #pragma unroll
-              for (int ch = 0; ch < Tr::kChunks; ++ch) {
-                const int c1 = (hgk * p.HPC + hl) * Tr::kChunks + ch;
-                tma_load_3d(st + (hl * Tr::kChunks + ch) * Tr::kBox, &kmap, 0, c1, row, &full[stage]);
-                tma_load_3d(st + (p.HPC + hl) * Tr::kTile + ch * Tr::kBox, &vmap, 0, c1, row, &full[stage]);
+                for (int ch = 0; ch < Tr::kChunks; ++ch) {
+                  const int c1 = (hgk * p.HPC + hl) * Tr::kChunks + ch;
+                  tma_load_3d(st + (hl * Tr::kChunks + ch) * Tr::kBox, &kmap, 0, c1, row, &full[stage]);
+                  tma_load_3d(st + (p.HPC + hl) * Tr::kTile + ch * Tr::kBox, &vmap, 0, c1, row, &full[stage]);
+                }
               }
             }
             if constexpr (tc_row_scaled(CACHE)) {
@@ -446,20 +465,16 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
               uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
               bulk_load(sc, p.k_scale + sb, bytes, &full[stage]);
               bulk_load(sc + bytes, p.v_scale + sb, bytes, &full[stage]);
-            } else if constexpr (CACHE == TC_KIVI) {
-              // the K scales of the CTA's heads (rows of 32 channels, 128-byte
-              // swizzle) and the V scales of the block's 16 tokens, all heads
-              const int phc = ph >= 0 ? ph : 0;
-              uint8_t* sc = st + 2 * p.HPC * Tr::kTile;
-              tma_load_2d(sc, &smap, 0, (phc * p.n_kv + hgk * p.HPC) * (D / 32), &full[stage]);
-              bulk_load(sc + p.HPC * D * 4, p.v_scale + (size_t)phc * kBlockSize * p.n_kv, 64u * p.n_kv,
-                        &full[stage]);
             }
           }
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { abort = true; break; }
         ++it;
+        if (++pstage == p.stages) {
+          pstage = 0;
+          ppass ^= 1u;
+        }
       }
     }
     // Never leave with copies in flight: wait for the last stages issued.
@@ -761,9 +776,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
       vsc[0] = vsm[t0 * p.n_kv + kvh];
       vsc[1] = vsm[t1 * p.n_kv + kvh];
     } else if constexpr (CACHE == TC_KIVI) {
-      const float* vsm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile + p.HPC * D * 4);
-      vsc[0] = vsm[t0 * p.n_kv + kvh];
-      vsc[1] = vsm[t1 * p.n_kv + kvh];
+      const float* vsm = reinterpret_cast<const float*>(st + 2 * p.HPC * Tr::kTile + p.HPC * D * 4) + head_local * 16;
+      vsc[0] = vsm[t0];
+      vsc[1] = vsm[t1];
     } else if constexpr (tc_fp8(CACHE)) {
       sc0 *= head_k_scale;
       sc1 *= head_k_scale;
@@ -900,6 +915,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
   // scores, one online-softmax update, then their P.V.  Two blocks give each
   // warp two independent MMA chains.  Returns false if a wait timed out.
   int it = 0;
+  int cstage = 0;      // ring stage of block `it`
+  uint32_t cpass = 0;  // parity of the ring pass of block `it`
   auto step = [&](auto nb_const) -> bool {
     constexpr int NB = decltype(nb_const)::value;
     const uint8_t* st[NB];
@@ -907,10 +924,18 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     uint32_t valid[NB];  // attended-row masks
 #pragma unroll
     for (int k = 0; k < NB; ++k) {
-      stage[k] = (it + k) % p.stages;
-      if (!mbar_wait(&full[stage[k]], ((it + k) / p.stages) & 1)) return false;
-      st[k] = smem + (size_t)stage[k] * p.stage_bytes;
-      if (p.pages)
+      int sk = cstage + k;
+      uint32_t pk = cpass;
+      if (sk >= p.stages) {
+        sk -= p.stages;
+        pk ^= 1u;
+      }
+      stage[k] = sk;
+      if (!mbar_wait(&full[sk], pk)) return false;
+      st[k] = smem + (size_t)sk * p.stage_bytes;
+      if constexpr (CACHE == TC_KIVI)
+        valid[k] = 0xFFFFu;  // full blocks only
+      else if (p.pages)
         valid[k] = (j + k + 1 == P[u + 1] - P[u]) ? token_mask(aset, L, last_page) : 0xFFFFu;
       else
         valid[k] = token_mask(aset, L, logical_block(aset, j + k));
@@ -1175,6 +1200,11 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, 1)
     i += nb;
     it += nb;
     j += nb;
+    cstage += nb;
+    if (cstage >= p.stages) {
+      cstage -= p.stages;
+      cpass ^= 1u;
+    }
 
     // ---- unit end: finish here, or hand a piece to the merge
     const bool unit_end = (i == uend);
@@ -1293,10 +1323,10 @@ static pkv_status make_kivi_scale_map(CUtensorMap* map, const float* k_scale, in
   return PKV_OK;
 }
 
-template <int CACHE, int D, int MAXW>
+template <int CACHE, int D, int MAXW, int MINB = 1>
 static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
                                  const TcParams& prm, cudaStream_t stream) {
-  auto kern = decode_tc_kernel<CACHE, D, MAXW>;
+  auto kern = decode_tc_kernel<CACHE, D, MAXW, MINB>;
   static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
   if ((int)plan.smem_bytes > configured_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
@@ -1347,10 +1377,15 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
 }
 
 // Up to 8 consumer warps use the variant whose launch bound leaves ~220
-// registers per thread; wider CTAs take the 16-warp variant.
+// registers per thread; wider CTAs take the 16-warp variant.  The 2-bit cache,
+// bound by dequantisation work, runs 3 CTAs of up to 4 consumer warps per SM
+// (launch bound: at most 136 registers a thread) for more warps in flight.
 template <int CACHE, int D>
 static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
                              const TcParams& prm, cudaStream_t stream) {
+  if constexpr (CACHE == TC_KIVI) {
+    if (plan.NCW <= 4) return launch_variant<CACHE, D, 4, kKiviCtasPerSm>(plan, km, vm, sm, prm, stream);
+  }
   if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, sm, prm, stream);
   return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, sm, prm, stream);
 }
@@ -1464,7 +1499,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     // Two consumer warps per CTA (2 KV heads when the group fits one warp) and
     // four CTAs per SM measured best for bf16 and int8; FP8, whose dequant is
     // heavier on the ALUs, does best with four warps per CTA and two CTAs.
-    const int warps = pl.cache_kind == TC_FP8 ? 4 : 2;
+    const int warps = (pl.cache_kind == TC_FP8 || kivi) ? 4 : 2;
     pl.HPC = 1;
     for (int h = std::min(s.n_kv, warps); h >= 1; --h) {
       if (s.n_kv % h == 0 && h * pl.QC <= warps) {
@@ -1477,9 +1512,8 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.HG = s.n_kv / pl.HPC;
   pl.NCW = pl.HPC * pl.QC;
   pl.units = s.num_seqs * pl.HG;
-  // KIVI: the K scales of the CTA's heads (head_dim floats each) and the V
-  // scales of the block's tokens, all heads
-  const size_t kivi_scales = kivi ? (size_t)pl.HPC * s.head_dim * 4 + 64 * (size_t)s.n_kv : 0;
+  // KIVI: the K scales (head_dim floats) and V scales (16 floats) of the CTA's heads
+  const size_t kivi_scales = kivi ? (size_t)pl.HPC * s.head_dim * 4 + 64 * (size_t)pl.HPC : 0;
   pl.tx_bytes = (uint32_t)(2 * (size_t)pl.HPC * tile_bytes + scale_bytes + kivi_scales);
   pl.stage_bytes = (uint32_t)align_up(pl.tx_bytes, 1024);
 
@@ -1494,7 +1528,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     // whole shared memory (~190 KB) of K/V in flight; fewer CTAs per SM only
     // when even 2 stages do not fit.
     stages = 2;
-    const int target_per_sm = pl.cache_kind == TC_FP8 ? 2 : kTargetCtasPerSm;
+    const int target_per_sm = pl.cache_kind == TC_FP8 ? 2 : (kivi && pl.NCW <= 4) ? kKiviCtasPerSm : kTargetCtasPerSm;
     for (int per = target_per_sm; per >= 1; --per) {
       const size_t budget = (size_t)kSmemPerSm / per - 1024;
       if (budget < fixed) continue;
@@ -1510,7 +1544,9 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.smem_bytes = (size_t)stages * pl.stage_bytes + fixed;
   if (pl.smem_bytes > (size_t)optin) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   // CTAs resident per SM from shared memory alone (1 KB reserved per CTA).
-  const int per_sm = std::max(1, std::min(pl.cache_kind == TC_FP8 ? 2 : kTargetCtasPerSm,
+  const int per_sm = std::max(1, std::min(pl.cache_kind == TC_FP8                ? 2
+                                          : (kivi && pl.NCW <= 4) ? kKiviCtasPerSm
+                                                                  : kTargetCtasPerSm,
                                           (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
   const int want_ctas = tuning ? tuning->num_ctas : 0;
   pl.overlap_prologue = tuning && (tuning->flags & PKV_TUNE_OVERLAP_PROLOGUE);

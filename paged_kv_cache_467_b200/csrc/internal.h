@@ -15,6 +15,7 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxConsumerWarps = 16;
 constexpr int kMaxCtas = 4096;          // upper bound of persistent CTAs per launch
 constexpr int kTargetCtasPerSm = 4;
+constexpr int kKiviCtasPerSm = 3;  // 2-bit cache: CTAs of up to 4 consumer warps
 constexpr size_t kSmemPerSm = 233472;  // 228 KB of shared memory per SM
 
 // Cache kinds of the tensor-core decode kernel.
@@ -105,10 +106,10 @@ struct KiviArgs {
   const void* new_value;
   void* residual_k;       // [num_seqs, 16, n_kv, 128] bf16
   void* residual_v;
-  void* key_cache;        // [num_blocks, 16, n_kv, 32] bytes
+  void* key_cache;        // [num_blocks, n_kv, 16, 32] bytes
   void* value_cache;
   float* k_scale;         // [num_blocks, n_kv, 128]
-  float* v_scale;         // [num_blocks, 16, n_kv]
+  float* v_scale;         // [num_blocks, n_kv, 16]
   const int32_t* block_tables;
   int max_blocks_per_seq;
   const int32_t* context_lens;

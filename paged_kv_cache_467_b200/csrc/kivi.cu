@@ -34,11 +34,13 @@ namespace {
 constexpr int kKiviD = 128;
 constexpr int kKiviThreads = 128;
 
+// Pools head-major inside a block, so a (block, KV head) tile is contiguous:
+// 512 bytes of codes per pool, 512 of K scales, 64 of V scales.
 struct KiviQuantTarget {
-  uint8_t* key_cache;    // [num_blocks, 16, n_kv, 32]
+  uint8_t* key_cache;    // [num_blocks, n_kv, 16, 32]
   uint8_t* value_cache;
   float* k_scale;        // [num_blocks, n_kv, 128]
-  float* v_scale;        // [num_blocks, 16, n_kv]
+  float* v_scale;        // [num_blocks, n_kv, 16]
   int n_kv;
 };
 
@@ -64,7 +66,7 @@ __device__ void kivi_quantize_rows(const __nv_bfloat16* src_k, const __nv_bfloat
     uint32_t bits = (uint32_t)(c & 3) << (2 * (i & 3));
     bits |= __shfl_xor_sync(0xffffffffu, bits, 1);
     bits |= __shfl_xor_sync(0xffffffffu, bits, 2);
-    if ((i & 3) == 0) t.key_cache[(((size_t)phys * kBlockSize + r) * t.n_kv + kv) * (kKiviD / 4) + (i >> 2)] = (uint8_t)bits;
+    if ((i & 3) == 0) t.key_cache[(((size_t)phys * t.n_kv + kv) * kBlockSize + r) * (kKiviD / 4) + (i >> 2)] = (uint8_t)bits;
   }
   // V: warp w takes tokens w, w+4, ...; lane l holds dims 4l .. 4l+3 (one code byte)
   for (int r = warp; r < kBlockSize; r += kKiviThreads / 32) {
@@ -79,7 +81,7 @@ __device__ void kivi_quantize_rows(const __nv_bfloat16* src_k, const __nv_bfloat
       c = max(-1, min(1, c));
       byte |= (uint32_t)(c & 3) << (2 * e);
     }
-    const size_t row = ((size_t)phys * kBlockSize + r) * t.n_kv + kv;
+    const size_t row = ((size_t)phys * t.n_kv + kv) * kBlockSize + r;
     t.value_cache[row * (kKiviD / 4) + lane] = (uint8_t)byte;
     if (lane == 0) t.v_scale[row] = vmax;
   }

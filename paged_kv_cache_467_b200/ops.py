@@ -290,8 +290,8 @@ def copy_blocks(key_cache, value_cache, block_mapping, k_scale=None, v_scale=Non
     code = cache_code(key_cache, cache_dtype)
     if code == PKV_INT4:
         d *= 2
-    elif code == PKV_KIVI2:
-        d *= 4
+    elif code == PKV_KIVI2:  # pools [nb, n_kv, 16, d / 4]
+        bs, n_kv, d = n_kv, bs, d * 4
     st = lib.pkv_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_mapping),
                              block_mapping.shape[0], n_kv, d, bs, nb, code, _ptr(device_error),
                              stream if stream is not None else _stream(key_cache.device))
@@ -305,8 +305,8 @@ def swap_blocks(src_key, src_value, dst_key, dst_value, block_mapping, src_k_sca
     code = cache_code(src_key, cache_dtype)
     if code == PKV_INT4:
         d *= 2
-    elif code == PKV_KIVI2:
-        d *= 4
+    elif code == PKV_KIVI2:  # pools [nb, n_kv, 16, d / 4]
+        bs, n_kv, d = n_kv, bs, d * 4
     dev = device if device is not None else (src_key.device if src_key.is_cuda else dst_key.device)
     st = lib.pkv_swap_blocks(_ptr(src_key), _ptr(src_value), _ptr(src_k_scale), _ptr(src_v_scale), snb,
                              _ptr(dst_key), _ptr(dst_value), _ptr(dst_k_scale), _ptr(dst_v_scale), dst_key.shape[0],
@@ -460,7 +460,7 @@ def kivi_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size) -> int:
 def kivi_quantize_blocks(key_rows, value_rows, dst_blocks, key_cache, value_cache, k_scale, v_scale,
                          device_error=None):
     """Quantise whole blocks ``key_rows``/``value_rows`` [n, 16, n_kv, d] (bf16) into the 2-bit pools
-    (uint8 [num_blocks, 16, n_kv, d / 4]) at physical blocks ``dst_blocks`` [n] (int32, -1 skips)."""
+    (uint8 [num_blocks, n_kv, 16, d / 4]) at physical blocks ``dst_blocks`` [n] (int32, -1 skips)."""
     n, block_size, n_kv, d = key_rows.shape
     st = lib.pkv_kivi_quantize_blocks(
         _ptr(key_rows), _ptr(value_rows), _ptr(dst_blocks), n, _ptr(key_cache), _ptr(value_cache), _ptr(k_scale),
@@ -474,9 +474,10 @@ def kivi_decode(out, query, residual_k, residual_v, key_cache, value_cache, k_sc
                 context_lens, max_context_len: int, key=None, value=None, sm_scale: float | None = None,
                 lse_out=None, workspace=None, device_error=None):
     """Decode over a 2-bit KIVI cache (full blocks in the pools, the partial last block in the BF16
-    residual [S, 16, n_kv, d]); ``key``/``value`` [S, n_kv, d] append token L-1 first."""
+    residual [S, 16, n_kv, d]; pools uint8 [num_blocks, n_kv, 16, d / 4], k_scale [num_blocks, n_kv, d],
+    v_scale [num_blocks, n_kv, 16]); ``key``/``value`` [S, n_kv, d] append token L-1 first."""
     S, n_q, d = query.shape
-    num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    num_blocks, n_kv, block_size = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:

@@ -29,6 +29,11 @@ def _ops():
     return ops
 
 
+def _codes(block_bytes):
+    """One device block [n_kv, 16, d/4] -> signed codes [16, n_kv, d] (the oracle's order)."""
+    return unpack_int2(block_bytes).transpose(1, 0, 2)
+
+
 def _bf16(x, dev="cuda"):
     return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).to(dev)
 
@@ -49,10 +54,10 @@ class Cache:
         ops = _ops()
         S, nb, nkv = w.num_seqs, w.num_blocks, w.n_kv
         g = torch.Generator(device="cuda").manual_seed(7)
-        self.kc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8, generator=g)
-        self.vc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8, generator=g)
+        self.kc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8, generator=g)
+        self.vc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8, generator=g)
         self.ks = torch.rand((nb, nkv, D), device="cuda", generator=g) * 3
-        self.vs = torch.rand((nb, 16, nkv), device="cuda", generator=g) * 3
+        self.vs = torch.rand((nb, nkv, 16), device="cuda", generator=g) * 3
         self.rk = torch.full((S, 16, nkv, D), float("nan"), device="cuda", dtype=torch.bfloat16)
         self.rv = torch.full((S, 16, nkv, D), float("nan"), device="cuda", dtype=torch.bfloat16)
         self.err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -64,10 +69,11 @@ class Cache:
                 blocks, _, _ = oracle.kivi_cache_state(K[: 16 * full], V[: 16 * full])
                 for b, (kcode, kscale, vcode, vscale) in enumerate(blocks):
                     phys = int(w.block_tables[s, b])
-                    self.kc[phys] = torch.from_numpy(pack_int2(kcode)).cuda()
-                    self.vc[phys] = torch.from_numpy(pack_int2(vcode)).cuda()
+                    # device layout: head-major inside the block
+                    self.kc[phys] = torch.from_numpy(pack_int2(kcode.transpose(1, 0, 2))).cuda()
+                    self.vc[phys] = torch.from_numpy(pack_int2(vcode.transpose(1, 0, 2))).cuda()
                     self.ks[phys] = torch.from_numpy(kscale).cuda()
-                    self.vs[phys] = torch.from_numpy(vscale).cuda()
+                    self.vs[phys] = torch.from_numpy(np.ascontiguousarray(vscale.T)).cuda()
             elif full:
                 kr = _bf16(K[: 16 * full].reshape(full, 16, nkv, D))
                 vr = _bf16(V[: 16 * full].reshape(full, 16, nkv, D))
@@ -124,10 +130,10 @@ def test_quantize_blocks_bit_exact():
     V[4, 0, 0, :8] = [4.0, 2.0, -2.0, 1.0, 0, 0, 0, 0]
     V[4, 0, 0, 8:] = 0.0
     dst = np.array([7, 0, 3, -1, 5, 8], np.int32)
-    kc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8)
-    vc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8)
+    kc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8)
+    vc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8)
     ks = torch.rand((nb, nkv, D), device="cuda")
-    vs = torch.rand((nb, 16, nkv), device="cuda")
+    vs = torch.rand((nb, nkv, 16), device="cuda")
     before = [t.clone() for t in (kc, vc, ks, vs)]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     ops.kivi_quantize_blocks(_bf16(K), _bf16(V), torch.from_numpy(dst).cuda(), kc, vc, ks, vs, device_error=err)
@@ -138,10 +144,10 @@ def test_quantize_blocks_bit_exact():
         if phys < 0:
             continue
         kcode, kscale, vcode, vscale = oracle.kivi_quantize_block(K[i], V[i])
-        assert np.array_equal(unpack_int2(kc[phys]), kcode), f"block {i}: K codes"
-        assert np.array_equal(unpack_int2(vc[phys]), vcode), f"block {i}: V codes"
+        assert np.array_equal(_codes(kc[phys]), kcode), f"block {i}: K codes"
+        assert np.array_equal(_codes(vc[phys]), vcode), f"block {i}: V codes"
         assert np.array_equal(ks[phys].view(np.int32), kscale.view(np.int32)), f"block {i}: K scales"
-        assert np.array_equal(vs[phys].view(np.int32), vscale.view(np.int32)), f"block {i}: V scales"
+        assert np.array_equal(vs[phys].T.view(np.int32), vscale.view(np.int32)), f"block {i}: V scales"
     untouched = [b for b in range(nb) if b not in set(dst.tolist())]
     for t, b0 in zip((kc, vc, ks, vs), before):
         assert np.array_equal(t[untouched], b0.cpu().numpy()[untouched])
@@ -150,8 +156,8 @@ def test_quantize_blocks_bit_exact():
 def test_quantize_blocks_flags_bad_destination():
     ops = _ops()
     rows = torch.zeros((2, 16, 1, D), device="cuda", dtype=torch.bfloat16)
-    kc = torch.zeros((4, 16, 1, D // 4), device="cuda", dtype=torch.uint8)
-    vc, ks, vs = torch.zeros_like(kc), torch.zeros((4, 1, D), device="cuda"), torch.zeros((4, 16, 1), device="cuda")
+    kc = torch.zeros((4, 1, 16, D // 4), device="cuda", dtype=torch.uint8)
+    vc, ks, vs = torch.zeros_like(kc), torch.zeros((4, 1, D), device="cuda"), torch.zeros((4, 1, 16), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     ops.kivi_quantize_blocks(rows, rows, torch.tensor([1, 4], dtype=torch.int32, device="cuda"), kc, vc, ks, vs,
                              device_error=err)
@@ -189,8 +195,8 @@ def test_decode_step_parity(n_q, n_kv):
         if L % 16 == 0:  # this step completed block L/16 - 1
             phys = int(w.block_tables[s, L // 16 - 1])
             kcode, kscale, vcode, vscale = oracle.kivi_quantize_block(K[L - 16 : L], V[L - 16 : L])
-            assert np.array_equal(unpack_int2(kc[phys]), kcode) and np.array_equal(unpack_int2(vc[phys]), vcode)
-            assert np.array_equal(ks[phys], kscale) and np.array_equal(vs[phys], vscale)
+            assert np.array_equal(_codes(kc[phys]), kcode) and np.array_equal(_codes(vc[phys]), vcode)
+            assert np.array_equal(ks[phys], kscale) and np.array_equal(vs[phys].T, vscale)
         else:
             assert np.array_equal(rk[s, (L - 1) % 16], K[L - 1])
 
@@ -224,10 +230,10 @@ def test_copy_and_swap_blocks():
     ops = _ops()
     nb, nkv = 8, 2
     g = torch.Generator(device="cuda").manual_seed(3)
-    kc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8, generator=g)
-    vc = torch.randint(0, 256, (nb, 16, nkv, D // 4), device="cuda", dtype=torch.uint8, generator=g)
+    kc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8, generator=g)
+    vc = torch.randint(0, 256, (nb, nkv, 16, D // 4), device="cuda", dtype=torch.uint8, generator=g)
     ks = torch.rand((nb, nkv, D), device="cuda", generator=g)
-    vs = torch.rand((nb, 16, nkv), device="cuda", generator=g)
+    vs = torch.rand((nb, nkv, 16), device="cuda", generator=g)
     ref = [t.cpu().clone() for t in (kc, vc, ks, vs)]
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     ops.copy_blocks(kc, vc, torch.tensor([[1, 5], [2, 6]], dtype=torch.int64, device="cuda"), ks, vs,
