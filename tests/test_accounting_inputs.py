@@ -95,3 +95,30 @@ def test_sequence_rows_cover_context():
         assert k.shape == (L, 2, 8) and v.shape == (L, 2, 8)
         assert len(w.history_slots(s)) == L - 1
     assert w.query().dtype == np.float32
+
+
+def test_kivi_bytes_and_bench_oracle_step():
+    """KIVI step bytes: 1600 B per full block and KV head (codes, K channel
+    scales, V token scales) plus the BF16 residual rows; the bench's oracle
+    step appends, quantises a completed block and decodes like the oracle's
+    own sequence decode."""
+    import numpy as np
+
+    import bench
+    import oracle
+    from paged_kv_cache_467_b200 import accounting, workloads
+
+    assert accounting.kivi_block_bytes(1, 128) == 1600
+    w = workloads.make_workload("kivi_cpu", seed=5, context_lens=[16, 21, 32, 3], n_q=4, n_kv=2, head_dim=128,
+                                cache_dtype="kivi2")
+    want = sum((L // 16) * 2 * 1600 + (L % 16) * 2 * 128 * 2 * 2 for L in (16, 21, 32, 3))
+    assert accounting.decode_kv_bytes(w) == want
+    rows = bench.prepare_oracle_rows(w, range(4))
+    assert bench.oracle_step_sample(w, range(4), rows) == want
+    q = w.query()
+    for s in range(4):
+        blocks, rk, rv, K, V, _ = rows[s]
+        L = int(w.context_lens[s])
+        assert len(blocks) == (L - 1) // 16 and rk.shape[0] == (L - 1) % 16
+        out, _ = oracle.kivi_decode_sequence(q[s], K[:L], V[:L], w.sm_scale)
+        assert np.isfinite(out).all()
