@@ -15,7 +15,7 @@ constexpr int kMaxStages = 8;
 constexpr int kMaxConsumerWarps = 16;
 constexpr int kMaxCtas = 4096;          // upper bound of persistent CTAs per launch
 constexpr int kTargetCtasPerSm = 4;
-constexpr int kKiviCtasPerSm = 3;  // 2-bit cache: CTAs of up to 4 consumer warps
+constexpr int kQuantCtasPerSm = 3;  // quantised caches: CTAs of up to 4 consumer warps
 constexpr size_t kSmemPerSm = 233472;  // 228 KB of shared memory per SM
 
 // Cache kinds of the tensor-core decode kernel.
