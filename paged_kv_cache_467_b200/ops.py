@@ -450,6 +450,23 @@ def paged_decode_step_window(out, query, key, value, key_cache, value_cache, blo
     return out
 
 
+def _check_kivi_tensors(S, n_kv, d, num_blocks, block_size, residual_k, residual_v, key_cache, value_cache,
+                        k_scale, v_scale):
+    """Shapes and dtypes the C ABI cannot see: the pools are head-major uint8 [num_blocks, n_kv, 16, d / 4]."""
+    want = {
+        "residual_k": (residual_k, torch.bfloat16, (S, block_size, n_kv, d)),
+        "residual_v": (residual_v, torch.bfloat16, (S, block_size, n_kv, d)),
+        "key_cache": (key_cache, torch.uint8, (num_blocks, n_kv, block_size, d // 4)),
+        "value_cache": (value_cache, torch.uint8, (num_blocks, n_kv, block_size, d // 4)),
+        "k_scale": (k_scale, torch.float32, (num_blocks, n_kv, d)),
+        "v_scale": (v_scale, torch.float32, (num_blocks, n_kv, block_size)),
+    }
+    for name, (t, dtype, shape) in want.items():
+        if t is None or t.dtype != dtype or tuple(t.shape) != shape:
+            got = None if t is None else (t.dtype, tuple(t.shape))
+            raise ValueError(f"kivi_decode: {name} must be {dtype} {shape}, got {got}")
+
+
 def kivi_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size) -> int:
     n = lib.pkv_kivi_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size)
     if n == ctypes.c_size_t(-1).value:
@@ -477,7 +494,10 @@ def kivi_decode(out, query, residual_k, residual_v, key_cache, value_cache, k_sc
     residual [S, 16, n_kv, d]; pools uint8 [num_blocks, n_kv, 16, d / 4], k_scale [num_blocks, n_kv, d],
     v_scale [num_blocks, n_kv, 16]); ``key``/``value`` [S, n_kv, d] append token L-1 first."""
     S, n_q, d = query.shape
-    num_blocks, n_kv, block_size = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
+    block_size, n_kv = residual_k.shape[1], residual_k.shape[2]  # residual [S, 16, n_kv, d]
+    num_blocks = key_cache.shape[0]
+    _check_kivi_tensors(S, n_kv, d, num_blocks, block_size, residual_k, residual_v, key_cache, value_cache, k_scale,
+                        v_scale)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(d)
     if workspace is None:

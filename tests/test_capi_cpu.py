@@ -182,3 +182,24 @@ def test_kivi_host_validation(lib):
     assert q(FAKE, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 64, 16, 8, 1, None, None) == 2
     assert q(FAKE, FAKE, FAKE, 3, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 0, None, None) == 2
     assert q(FAKE, FAKE, FAKE, -1, FAKE, FAKE, FAKE, FAKE, 2, 128, 16, 8, 1, None, None) == 1
+
+
+def test_kivi_binding_rejects_token_major_pools(lib):
+    """The binding checks the shapes the C ABI cannot see before any call."""
+    from paged_kv_cache_467_b200 import ops
+
+    S, nq, nkv, d, nb = 2, 8, 2, 128, 4
+    q = torch.zeros((S, nq, d), dtype=torch.bfloat16)
+    rk = torch.zeros((S, 16, nkv, d), dtype=torch.bfloat16)
+    ks = torch.zeros((nb, nkv, d))
+    vs = torch.zeros((nb, nkv, 16))
+    bt = torch.zeros((S, 1), dtype=torch.int32)
+    cl = torch.zeros(S, dtype=torch.int32)
+    head_major = torch.zeros((nb, nkv, 16, d // 4), dtype=torch.uint8)
+    token_major = torch.zeros((nb, 16, nkv, d // 4), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="key_cache"):
+        ops.kivi_decode(torch.empty_like(q), q, rk, rk, token_major, token_major, ks, vs, bt, cl, 0)
+    with pytest.raises(ValueError, match="residual_k"):
+        ops.kivi_decode(torch.empty_like(q), q, rk.float(), rk, head_major, head_major, ks, vs, bt, cl, 0)
+    with pytest.raises(ValueError, match="v_scale"):
+        ops.kivi_decode(torch.empty_like(q), q, rk, rk, head_major, head_major, ks, vs.transpose(1, 2), bt, cl, 0)
