@@ -14,7 +14,7 @@ examples, closed forms, invariants and independent library routines; see
 ``tests/test_oracle_*.py``.  No function here is "parity unpinned".
 """
 from .quant import (absmax_quantize, e4m3_decode, e4m3_encode, e4m3_value_table, e5m2_decode,  # noqa: F401
-                    e5m2_encode, e5m2_value_table, pack_int4, unpack_int4)
+                    e5m2_encode, e5m2_value_table, pack_int2, pack_int4, unpack_int2, unpack_int4)
 from .paged_attention import (  # noqa: F401
     attention_one_sequence,
     dequantize_rows,
