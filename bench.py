@@ -67,12 +67,39 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def strip_c_comments(text: str) -> str:
+    """C/C++ source without comments, trailing blanks and blank lines (string
+    and character literals kept as they are)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i : j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            while i < n and text[i] != "\n":
+                i += 1
+        elif text.startswith("/*", i):
+            end = text.find("*/", i + 2)
+            i = n if end < 0 else end + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (line.rstrip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_hash() -> str:
+    """Hash of the library's sources with comments removed: a profile taken on
+    these sources stays valid across comment edits, not across code edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_467_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + strip_c_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -1,4 +1,5 @@
-// Paged decode attention on the tensor-core path (BF16, INT8 and FP8 E4M3 caches).
+// Paged decode attention on the tensor-core path: BF16, INT8, INT4, FP8 E4M3,
+// FP8 E5M2 and 2-bit KIVI caches.
 //
 // What it computes: for every sequence s and query head h, softmax over the
 // s-th sequence's cached keys of sm_scale * <q_h, K_p> weighting the cached
@@ -11,19 +12,24 @@
 //  * Work unit = (sequence, group of HPC KV heads).  All units' 16-token blocks
 //    are laid end to end and every persistent CTA takes an equal contiguous
 //    share (split-K over context with no wave quantisation).  A unit cut by a
-//    share boundary is finished by whichever CTA writes its last piece: pieces
-//    carry (normalised o, log-sum-exp) and are merged in CTA order, so the
-//    result does not depend on timing.
+//    share boundary leaves one piece per CTA (normalised o, base-2 lse); the
+//    merge kernel, queued behind this one with programmatic serialisation,
+//    combines them in CTA order, so the result does not depend on timing.
 //  * One producer warp streams each block's K and V tiles of the CTA's KV heads
-//    into a ring of shared-memory stages with TMA (128-byte swizzle, tile
-//    [16 tokens x 128 bytes] per box), completing on mbarriers.  Block-table
-//    entries are fetched 32 at a time by the producer's lanes.
+//    into a ring of shared-memory stages, completing on mbarriers: TMA boxes of
+//    [16 tokens x 128 bytes] with the 128-byte swizzle (INT4: 64-byte rows,
+//    64-byte swizzle), or for the head-major 2-bit pools one bulk copy per pool
+//    plus a swizzled TMA box of the per-channel K scales.  Block-table entries
+//    are fetched 32 at a time by the producer's lanes.
 //  * Consumer warp (KV head, chunk of 8 query heads): S^T[16 tok x 8 heads] =
-//    K_blk * Q^T with m16n8k16 MMAs (K from ldmatrix, Q held in registers), an
-//    online base-2 softmax with warp shuffles, then O^T[d x 8] += V^T * P^T
-//    (V^T via ldmatrix.trans, P^T via movmatrix).  INT8 / FP8 codes are
-//    converted to exact f16 in registers; the per-token INT8 scales multiply the
-//    scores and the probabilities, the per-head FP8 scales fold into constants.
+//    K_blk * Q^T, an online base-2 softmax with warp shuffles, then
+//    O^T[d x 8] += V^T * P^T with P^T via movmatrix.  BF16 uses m16n8k16 MMAs
+//    fed by ldmatrix.  INT8 / INT4 scores run as m16n8k32 integer MMAs on the
+//    stored codes against the query quantised per unit into two 8-bit parts;
+//    E4M3 / E5M2 codes, and V codes of every quantised format, become exact f16
+//    in registers.  Per-token scales multiply the scores and the
+//    probabilities, per-head FP8 scales fold into constants, and the 2-bit
+//    cache's per-(block, channel) K scales fold into the f16 query operand.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
