@@ -251,7 +251,8 @@ struct TcTraits {
   static constexpr int kSteps = D / 16;  // k-steps of Q.K and m-tiles of P.V
 };
 
-// Write one finished (or merged) row pair: heads 2c, 2c+1 of this lane.
+// Head dimension held in accumulator row g (hi = 0) or g + 8 (hi = 1) of P.V
+// m-tile mt: the order in which each cache format's V fragments list the dims.
 template <int CACHE, int D>
 __device__ __forceinline__ int d_of(int mt, int hi, int g) {
   if constexpr (CACHE == TC_BF16) return mt * 16 + g + 8 * hi;
@@ -649,8 +650,8 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
 
   // Scores of one 16-token block held in stage memory st: S^T = K Q^T
   // [16 tokens x 8 heads] in log2 units, -inf past the sequence end.
-  // sv = (token g, head 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); vsc = int8 V
-  // scales of tokens g and g+8 (1 otherwise).
+  // sv = (token g, head 2c), (g, 2c+1), (g+8, 2c), (g+8, 2c+1); vsc = the
+  // per-token V scales (INT8, INT4, 2-bit) of tokens g and g+8 (1 otherwise).
   auto block_scores = [&](const uint8_t* st, uint32_t vm, float (&sv)[4], float (&vsc)[2]) {
     const uint32_t kt = smem_addr(st + head_local * Tr::kTile);
     const int t0 = g, t1 = g + 8;
@@ -1292,7 +1293,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // bytes] as (elements of one chunk, chunk index, token row), box = 1 chunk x 16
 // rows.  A chunk is 128 bytes (BF16 / INT8 / FP8 rows, 128-byte swizzle), or a
 // whole head row: 64 bytes of INT4 (64-byte swizzle) or 32 bytes of 2-bit
-// codes (no swizzle).
+// codes (no swizzle; the decode reads the head-major 2-bit pools with bulk
+// copies, so that map is only passed along).
 pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes_i,
                               int64_t rows) {
   auto fn = encode_fn();

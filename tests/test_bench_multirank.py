@@ -71,3 +71,14 @@ def test_single_rank_helpers():
 
     assert bench.max_over_ranks([3.0, 1.0], 1) == [3.0, 1.0]
     assert bench.whole_job_gbs(6e8, 1, 0.1) == 6000.0
+
+
+def test_source_hash_ignores_comments_only():
+    import bench
+
+    code = 'int a = 1;  // note\n/* block\n   comment */\nconst char* s = "// kept"; char q = \'"\';\n\n'
+    assert bench.strip_c_comments(code) == 'int a = 1;\nconst char* s = "// kept"; char q = \'"\';'
+    edited = code.replace("// note", "// another note").replace("block", "other block")
+    assert bench.strip_c_comments(edited) == bench.strip_c_comments(code)
+    assert bench.strip_c_comments(code.replace("a = 1", "a = 2")) != bench.strip_c_comments(code)
+    assert len(bench.kernel_source_hash()) == 16
