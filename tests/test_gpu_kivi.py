@@ -248,3 +248,34 @@ def test_copy_and_swap_blocks():
     for t, r, h in zip((kc, vc, ks, vs), ref, host):
         assert torch.equal(t.cpu(), r)
         assert torch.equal(h[2], r[0]) and torch.equal(h[0], r[7]) and not h[1].any()
+
+
+def test_decode_error_paths():
+    """A block-table entry outside the pool sets PKV_DEVERR_BLOCK_RANGE and a
+    length past the table sets PKV_DEVERR_CONTEXT_LEN; the other sequences keep
+    the oracle's result and nothing outside the buffers is touched."""
+    ops = _ops()
+    w = _wl([40, 64, 33], 8, 2, seed=31)
+    c = Cache(w, w.context_lens)
+    q = _bf16(w.query())
+    bt = torch.from_numpy(w.block_tables.copy()).cuda()
+    bt[1, 1] = w.num_blocks + 5  # sequence 1 reads a block outside the pool
+    out = torch.empty_like(q)
+    ops.kivi_decode(out, q, c.rk, c.rv, c.kc, c.vc, c.ks, c.vs, bt, torch.from_numpy(w.context_lens).cuda(),
+                    w.max_context_len, sm_scale=w.sm_scale, device_error=c.err)
+    torch.cuda.synchronize()
+    assert int(c.err.item()) & ops.DEVERR_BLOCK_RANGE
+    got = out.float().cpu().numpy()
+    qh = w.query()
+    for s in (0, 2):
+        K, V = w.sequence_kv(s)
+        L = int(w.context_lens[s])
+        want, _ = oracle.kivi_decode_sequence(qh[s], K[:L], V[:L], w.sm_scale)
+        assert np.abs(got[s] - want).max() <= TOL_OUT[0]
+    c.err.zero_()
+    cl = torch.from_numpy(w.context_lens.copy()).cuda()
+    cl[0] = w.block_tables.shape[1] * 16 + 7  # longer than its table
+    ops.kivi_decode(out, q, c.rk, c.rv, c.kc, c.vc, c.ks, c.vs, torch.from_numpy(w.block_tables).cuda(), cl,
+                    int(cl.max().item()), sm_scale=w.sm_scale, device_error=c.err)
+    torch.cuda.synchronize()
+    assert int(c.err.item()) & ops.DEVERR_CONTEXT_LEN
