@@ -5,9 +5,11 @@
 A step appends one token per sequence and runs decode attention over every
 sequence's paged cache, for one layer of the workload: one fused launch
 (pkv_paged_decode_step), or with --unfused the two calls pkv_kv_cache_write and
-pkv_paged_attention_decode.  Default workload: the Llama-3-8B-shaped decode
-step (batch 64, 32 query / 8 KV heads, head_dim 128, BF16 cache, block 16,
-context lengths uniform in [512, 4096], shuffled pool sized to fit exactly).
+pkv_paged_attention_decode.  Default workload: the largest single-GPU
+configuration, the long-context 70B-shaped decode step (batch 8, 64 query / 8
+KV heads, head_dim 128, BF16 cache, block 16, context lengths uniform in
+[32768, 131072], shuffled pool sized to fit exactly: about 2.7 GB of K/V read
+per step).  ``--config`` selects the others.
 
 Under torchrun every rank runs its own replica of the workload (sequences are
 independent: weak scaling, no collective on the data path); rank 0 prints one
@@ -40,12 +42,19 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--config", default="llama3_8b")
+    ap.add_argument("--config", default="long_70b")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--unfused", action="store_true", help="append in its own launch before the decode")
     ap.add_argument("--no-overlap", action="store_true", help="launch each step without overlapping its prologue")
     ap.add_argument("--op", default="decode_step", choices=["decode_step", "copy_blocks", "swap_blocks", "quest"],
                     help="what a step runs (the default is the decode step)")
+    ap.add_argument("--prefix-splits", type=int, default=0,
+                    help="shared-prefix config: splits of the prefix pass along the prefix (0 = automatic)")
+    ap.add_argument("--prefix-serial", action="store_true",
+                    help="shared-prefix config: run the decode of each sequence's own blocks after the prefix pass "
+                         "instead of beside it")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="run the configuration's first N sequences only (a smaller case for profiling)")
     ap.add_argument("--quest-budget", type=int, default=4096,
                     help="--op quest: tokens each KV head reads (a multiple of the 16-token page)")
     return ap.parse_args()
@@ -259,23 +268,36 @@ def blas_threads() -> int:
 
 
 def time_oracle(w, budget_s: float, max_seqs: int | None = None):
-    """Time oracle steps on a bounded sample of the workload's sequences."""
-    order = list(range(w.num_seqs))
-    seqs, t_total, b_total = [], 0.0, 0
-    host = {}
+    """Time oracle steps on a bounded sample of the workload's sequences.
+
+    Sequences are prepared one at a time (their host caches are dropped after
+    use, so host memory stays bounded).  Without ``max_seqs`` each sequence is
+    stepped once until ``budget_s`` of timed work; with it, at most
+    ``max_seqs`` sequences are prepared and each is stepped repeatedly for its
+    share of the budget.  Returns (KV bytes, seconds, sequences, steps)."""
+    seqs, t_total, b_total, steps = [], 0.0, 0, 0
     scales = w.fp8_head_scales() if w.cache_dtype.startswith("fp8") else None
-    for s in order:
+    for s in range(w.num_seqs):
         if max_seqs is not None and len(seqs) >= max_seqs:
             break
-        host.update(prepare_oracle_rows(w, [s], scales))
-        t0 = time.perf_counter()
-        b = oracle_step_sample(w, [s], host)
-        t_total += time.perf_counter() - t0
-        b_total += b
+        host = prepare_oracle_rows(w, [s], scales)
         seqs.append(s)
-        if t_total >= budget_s:
+        share = budget_s / max_seqs if max_seqs else 0.0
+        t_seq = 0.0
+        while True:
+            t0 = time.perf_counter()
+            b = oracle_step_sample(w, [s], host)
+            dt = time.perf_counter() - t0
+            t_seq += dt
+            b_total += b
+            steps += 1
+            if t_seq >= share:
+                break
+        t_total += t_seq
+        del host
+        if max_seqs is None and t_total >= budget_s:
             break
-    return b_total, t_total, seqs
+    return b_total, t_total, seqs, steps
 
 
 def run_reference(args, rank, world):
@@ -380,7 +402,10 @@ def run_b200(args, rank, world, local):
     if world > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
 
-    w = replica_workload(workloads.CONFIGS[args.config](), rank)
+    base = workloads.CONFIGS[args.config]()
+    if args.seqs:
+        base = workloads.first_sequences(base, args.seqs)
+    w = replica_workload(base, rank)
     S, nq, nkv, d, bs = w.num_seqs, w.n_q, w.n_kv, w.head_dim, w.block_size
     named = "int4" if w.cache_dtype == "int4" else None  # an int4 pool's torch dtype (uint8) does not name it
     gen = torch.Generator(device=dev).manual_seed(1234 + rank)
@@ -450,9 +475,13 @@ def run_b200(args, rank, world, local):
 
 
     prefix_blocks = w.shared_prefix_tokens // bs
+    prefix_tuning = None
     if prefix_blocks:
-        # the shared prefix is attended once for all sequences, then each sequence's own blocks
-        nws = max(nws, ops.shared_prefix_workspace_size(S, nq, nkv, d, bs, prefix_blocks))
+        # the shared prefix is attended once for all sequences, beside the decode of each sequence's own blocks
+        if args.prefix_splits or args.prefix_serial:
+            prefix_tuning = ops.DecodeTuning(0, 0, 0, ops.TUNE_PREFIX_SERIAL if args.prefix_serial else 0,
+                                             args.prefix_splits)
+        nws = max(nws, ops.shared_prefix_workspace_size(S, nq, nkv, d, bs, prefix_blocks, prefix_tuning))
         ws = torch.zeros(max(nws, 256), dtype=torch.uint8, device=dev)
 
     def fused(out, q, k_new, v_new, bt, cl, tun):
@@ -465,7 +494,7 @@ def run_b200(args, rank, world, local):
         elif prefix_blocks:
             ops.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, cl, w.max_context_len, prefix_blocks,
                                                      key=k_new, value=v_new, sm_scale=w.sm_scale, workspace=ws,
-                                                     device_error=err)
+                                                     device_error=err, tuning=prefix_tuning)
         else:
             ops.paged_decode_step(out, q, k_new, v_new, kc, vc, bt, cl, w.max_context_len, w.sm_scale, ks, vs,
                                   workspace=ws, device_error=err, tuning=tun, cache_dtype=named)
@@ -473,7 +502,8 @@ def run_b200(args, rank, world, local):
     def decode(out, q, bt, cl):
         if prefix_blocks:
             ops.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, cl, w.max_context_len, prefix_blocks,
-                                                     sm_scale=w.sm_scale, workspace=ws, device_error=err)
+                                                     sm_scale=w.sm_scale, workspace=ws, device_error=err,
+                                                     tuning=prefix_tuning)
         elif w.window:
             ops.paged_attention_decode_window(out, q, kc, vc, bt, cl, w.max_context_len, w.window, w.sinks,
                                               w.sm_scale, ks, vs, workspace=ws, device_error=err, cache_dtype=named)
@@ -601,7 +631,7 @@ def run_b200(args, rank, world, local):
                 "frac": achieved / peak,
                 "traffic": traffic,
                 "kernel": "kivi_residual_kernel + decode_tc_kernel<KIVI> + decode_merge_kernel (pkv_kivi_decode)"
-                if kivi else ("prefix_attn_kernel + " if prefix_blocks else "")
+                if kivi else ("prefix_tc_kernel (tcgen05) + " if prefix_blocks else "")
                 + ("decode_f32_kernel" if w.cache_dtype == "f32" else "decode_tc_kernel")
                 + ("" if args.unfused else " with fused append")
                 + ("" if w.cache_dtype == "f32" else " + decode_merge_kernel")
@@ -626,15 +656,18 @@ def run_b200(args, rank, world, local):
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
-            # the KIVI oracle quantises a sequence's blocks group by group before its
-            # timed step (seconds per sequence, untimed): a few sequences bound the run
-            b, t, seqs = time_oracle(w, budget_s=12.0, max_seqs=3 if kivi else None)
+            # the KIVI oracle quantises a sequence's blocks group by group before its timed
+            # step, and a long-context sequence takes seconds to prepare (both untimed): a few
+            # sequences, each stepped repeatedly, bound those runs
+            long_ctx = int(w.context_lens.max()) > 16384
+            b, t, seqs, nsteps = time_oracle(w, budget_s=12.0, max_seqs=3 if kivi else 2 if long_ctx else None)
             line["cpu_baseline"] = {
                 "value": b / t / 1e9,
                 "unit": "GB/s",
                 "cores": blas_threads(),
                 "kind": "oracle",
-                "sample": f"{len(seqs)} of {w.num_seqs} sequences (append + float64 decode), {t:.1f} s",
+                "sample": f"{len(seqs)} of {w.num_seqs} sequences, {nsteps} oracle steps (append + float64 "
+                          f"decode), {t:.1f} s",
             }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -63,6 +63,8 @@ typedef enum {
 #define PKV_DEVERR_BLOCK_RANGE 0x2  /* block table entry outside [0, num_blocks) */
 #define PKV_DEVERR_CONTEXT_LEN 0x4  /* context_len < 0, > max_context_len or > max_blocks_per_seq * block_size */
 #define PKV_DEVERR_TIMEOUT 0x8      /* a bounded wait inside a kernel gave up (~1 s) */
+#define PKV_DEVERR_PREFIX 0x10      /* shared-prefix decode: a block table does not begin with
+                                       row 0's prefix_blocks entries */
 
 /*
  * Append new tokens' K/V rows into their cache slots (reshape_and_cache).
@@ -214,20 +216,25 @@ pkv_status pkv_paged_decode_step_window(void* out, const void* query, const void
  * Strategies", Prefix Caching; "KV Cache Engineering for LLM Serving", section
  * 11).  The first prefix_blocks entries of every block table must name the same
  * blocks (the caller's contract, as for shared blocks in general; row 0's are
- * the ones read).  The prefix is attended once per KV head for the queries of
- * all sequences together (a dense tensor-core pass), and each sequence's own
- * positions [prefix_blocks * block_size, L) are attended starting from that
- * state, so the result equals pkv_paged_attention_decode's.
+ * the ones read, and a row that differs sets PKV_DEVERR_PREFIX).  The prefix is
+ * attended once per KV head for the queries of all sequences together (a dense
+ * pass on the fifth-generation tensor cores), each sequence's own positions
+ * [prefix_blocks * block_size, L) are attended by the paged decode, and the two
+ * softmax states are merged exactly, so the result equals
+ * pkv_paged_attention_decode's.
  *
  *   key, value        optional new rows [num_seqs, n_kv, head_dim] (act dtype):
  *                     appended as token L-1 first, as in pkv_paged_decode_step;
  *                     NULL for a plain decode
  *   prefix_blocks     >= 1; every context length must exceed prefix_blocks *
- *                     block_size (else PKV_DEVERR_CONTEXT_LEN and undefined output)
+ *                     block_size (else PKV_DEVERR_CONTEXT_LEN, and that
+ *                     sequence's output is undefined)
  *   workspace         pkv_shared_prefix_workspace_size bytes
- * BF16 cache and activations, head_dim 64 or 128.  Three launches on `stream`
- * (prefix pass, decode, merge), each queued behind the previous one with
- * programmatic serialisation.
+ * BF16 cache and activations, head_dim 64 or 128.  Three launches on `stream`:
+ * the prefix pass, the decode over each sequence's own blocks, which runs
+ * beside the prefix pass (it touches none of the prefix pass's data), and the
+ * merge.  The prefix pass waits for the kernel launched before the call; the
+ * decode starts only once every CTA of the prefix pass has done so.
  */
 size_t pkv_shared_prefix_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
                                         int prefix_blocks);
@@ -307,7 +314,15 @@ typedef struct {
   int num_ctas;
   int stages;
   int heads_per_cta;
-  int flags; /* PKV_TUNE_* bits */
+  int flags;         /* PKV_TUNE_* bits */
+  int prefix_splits; /* shared-prefix decode: splits of the prefix pass along the prefix (0 = automatic) */
+  int reserved;      /* must be 0 */
+  /* SM clock cycles a bounded wait of the decode kernels may spend before it
+   * gives up and sets PKV_DEVERR_TIMEOUT (0 = about one second).  A kernel that
+   * gives up still waits, with the full limit, for the copies it has issued, so
+   * nothing is in flight when it exits; its outputs are then undefined.  For
+   * tests of the timeout path. */
+  int64_t wait_limit_cycles;
 } pkv_decode_tuning;
 
 /* Launch the decode kernel so that it may start while the kernel launched just
@@ -318,6 +333,10 @@ typedef struct {
  * valid when context_lens and block_tables were not written by the kernel
  * launched immediately before this call. */
 #define PKV_TUNE_OVERLAP_PROLOGUE 0x1
+
+/* Shared-prefix decode: run the decode over each sequence's own blocks after
+ * the prefix pass instead of beside it. */
+#define PKV_TUNE_PREFIX_SERIAL 0x2
 
 /* Workspace bytes for pkv_paged_attention_decode_ex with the given tuning. */
 size_t pkv_paged_attention_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
@@ -340,6 +359,24 @@ pkv_status pkv_paged_attention_decode_ex(void* out, const void* query, const voi
                                          int64_t num_blocks, float sm_scale, pkv_dtype act_dtype, pkv_dtype cache_dtype,
                                          float* lse_out, void* workspace, size_t workspace_bytes, int32_t* device_error,
                                          const pkv_decode_tuning* tuning, void* stream);
+
+/* Shared-prefix decode with launch overrides (tuning may be NULL): num_ctas,
+ * stages and flags apply to the decode over each sequence's own blocks,
+ * prefix_splits to the prefix pass, PKV_TUNE_PREFIX_SERIAL orders the two
+ * passes.  Size the workspace with pkv_shared_prefix_workspace_size_ex and the
+ * same tuning. */
+size_t pkv_shared_prefix_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                           int prefix_blocks, const pkv_decode_tuning* tuning);
+pkv_status pkv_paged_attention_decode_shared_prefix_ex(void* out, const void* query, const void* key,
+                                                       const void* value, void* key_cache, void* value_cache,
+                                                       const int32_t* block_tables, int max_blocks_per_seq,
+                                                       const int32_t* context_lens, int max_context_len,
+                                                       int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                                       int64_t num_blocks, float sm_scale, int prefix_blocks,
+                                                       pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                                       void* workspace, size_t workspace_bytes,
+                                                       int32_t* device_error, const pkv_decode_tuning* tuning,
+                                                       void* stream);
 
 /* pkv_paged_attention_decode_pages with explicit launch shape (tuning may be
  * NULL; heads_per_cta must be 0 or 1: a page list belongs to one KV head).
@@ -375,7 +412,9 @@ pkv_status pkv_paged_attention_decode_pages_ex(void* out, const void* query, con
  *     bytes the shape needs.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress).  Make that first call before any stream capture
- *     on that device.
+ *     on that device.  The address is kept for the life of the process: after
+ *     cudaDeviceReset on a device it no longer names the array, so a process
+ *     that resets a device must not call this entry point on it again.
  *   - Every call on a device shares the one array.  Calls whose work can
  *     overlap on the GPU (different streams, no ordering between them) race on
  *     the array and give wrong results; keep such calls in one stream.

@@ -111,14 +111,21 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
     if (prefix_blocks > max_blocks_per_seq) return PKV_ERR_INVALID_ARG;
   }
 
+  if (tuning && (tuning->reserved != 0 || tuning->prefix_splits < 0 || tuning->wait_limit_cycles < 0))
+    return PKV_ERR_INVALID_ARG;
   TcArgs a{out, query, key_cache, value_cache, k_scale, v_scale, block_tables, max_blocks_per_seq, context_lens,
            max_context_len, num_blocks, sm_scale, lse_out, workspace, device_error, new_key, new_value, window,
            sinks, pages, k_pages};
   a.skip_blocks = prefix_blocks;
+  if (tuning) {
+    a.prefix_splits = tuning->prefix_splits;
+    a.prefix_serial = (tuning->flags & PKV_TUNE_PREFIX_SERIAL) != 0;
+    a.wait_limit = tuning->wait_limit_cycles;
+  }
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   if (cache_dtype == PKV_F32) return launch_decode_f32(s, a, strm);
   // a page list is per KV head: one KV head per CTA
-  pkv_decode_tuning one_head = tuning ? *tuning : pkv_decode_tuning{0, 0, 0, 0};
+  pkv_decode_tuning one_head = tuning ? *tuning : pkv_decode_tuning{0, 0, 0, 0, 0, 0, 0};
   if (pages) {
     one_head.heads_per_cta = 1;
     tuning = &one_head;
@@ -130,9 +137,9 @@ static pkv_status decode_impl(void* out, const void* query, const void* key_cach
   if (prefix_blocks > 0) {
     // the prefix pass keeps its partial states after the decode's scratch
     const size_t off = (plan.ws_total + 255) / 256 * 256;
-    need = off + prefix_workspace_bytes(num_seqs, n_q, n_kv, head_dim, prefix_blocks);
+    need = off + prefix_workspace_bytes(num_seqs, n_q, n_kv, head_dim, prefix_blocks, a.prefix_splits);
     if (workspace && workspace_bytes >= need) a.prefix_ws = static_cast<uint8_t*>(workspace) + off;
-    plan.overlap_prologue = true;  // the decode's prologue overlaps the prefix pass
+    plan.overlap_prologue = true;  // the decode is queued behind the prefix pass with programmatic serialisation
   }
   if (!workspace || workspace_bytes < need || !aligned16(workspace)) return PKV_ERR_WORKSPACE;
   return launch_tc(s, plan, a, strm);
@@ -364,14 +371,41 @@ pkv_status pkv_paged_attention_decode_pages_ex(void* out, const void* query, con
                      nullptr, nullptr, 0, 0, pages, k_pages);
 }
 
-size_t pkv_shared_prefix_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
-                                        int prefix_blocks) {
+size_t pkv_shared_prefix_workspace_size_ex(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                           int prefix_blocks, const pkv_decode_tuning* tuning) {
   const DecodeShape s{num_seqs, n_q, n_kv, head_dim, block_size, PKV_BF16, PKV_BF16};
   if (prefix_blocks < 1 || check_decode_shape(s) != PKV_OK) return (size_t)-1;
+  if (tuning && tuning->prefix_splits < 0) return (size_t)-1;
   if (num_seqs == 0) return 0;
   TcPlan plan;
-  if (plan_tc(s, nullptr, &plan) != PKV_OK) return (size_t)-1;
-  return (plan.ws_total + 255) / 256 * 256 + prefix_workspace_bytes(num_seqs, n_q, n_kv, head_dim, prefix_blocks);
+  if (plan_tc(s, tuning, &plan) != PKV_OK) return (size_t)-1;
+  return (plan.ws_total + 255) / 256 * 256 +
+         prefix_workspace_bytes(num_seqs, n_q, n_kv, head_dim, prefix_blocks, tuning ? tuning->prefix_splits : 0);
+}
+
+size_t pkv_shared_prefix_workspace_size(int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                        int prefix_blocks) {
+  return pkv_shared_prefix_workspace_size_ex(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks, nullptr);
+}
+
+pkv_status pkv_paged_attention_decode_shared_prefix_ex(void* out, const void* query, const void* key,
+                                                       const void* value, void* key_cache, void* value_cache,
+                                                       const int32_t* block_tables, int max_blocks_per_seq,
+                                                       const int32_t* context_lens, int max_context_len,
+                                                       int num_seqs, int n_q, int n_kv, int head_dim, int block_size,
+                                                       int64_t num_blocks, float sm_scale, int prefix_blocks,
+                                                       pkv_dtype act_dtype, pkv_dtype cache_dtype, float* lse_out,
+                                                       void* workspace, size_t workspace_bytes,
+                                                       int32_t* device_error, const pkv_decode_tuning* tuning,
+                                                       void* stream) {
+  if (prefix_blocks < 1) return PKV_ERR_INVALID_ARG;
+  if ((key == nullptr) != (value == nullptr)) return PKV_ERR_INVALID_ARG;
+  if (key && (!aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
+  if (max_context_len <= prefix_blocks * block_size && num_seqs > 0) return PKV_ERR_INVALID_ARG;
+  return decode_impl(out, query, key_cache, value_cache, nullptr, nullptr, block_tables, max_blocks_per_seq,
+                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
+                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, tuning, stream, key,
+                     value, 0, 0, nullptr, 0, prefix_blocks);
 }
 
 pkv_status pkv_paged_attention_decode_shared_prefix(void* out, const void* query, const void* key, const void* value,
@@ -382,14 +416,11 @@ pkv_status pkv_paged_attention_decode_shared_prefix(void* out, const void* query
                                                     int prefix_blocks, pkv_dtype act_dtype, pkv_dtype cache_dtype,
                                                     float* lse_out, void* workspace, size_t workspace_bytes,
                                                     int32_t* device_error, void* stream) {
-  if (prefix_blocks < 1) return PKV_ERR_INVALID_ARG;
-  if ((key == nullptr) != (value == nullptr)) return PKV_ERR_INVALID_ARG;
-  if (key && (!aligned16(key) || !aligned16(value))) return PKV_ERR_INVALID_ARG;
-  if (max_context_len <= prefix_blocks * block_size && num_seqs > 0) return PKV_ERR_INVALID_ARG;
-  return decode_impl(out, query, key_cache, value_cache, nullptr, nullptr, block_tables, max_blocks_per_seq,
-                     context_lens, max_context_len, num_seqs, n_q, n_kv, head_dim, block_size, num_blocks, sm_scale,
-                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes, device_error, nullptr, stream, key,
-                     value, 0, 0, nullptr, 0, prefix_blocks);
+  return pkv_paged_attention_decode_shared_prefix_ex(out, query, key, value, key_cache, value_cache, block_tables,
+                                                     max_blocks_per_seq, context_lens, max_context_len, num_seqs, n_q,
+                                                     n_kv, head_dim, block_size, num_blocks, sm_scale, prefix_blocks,
+                                                     act_dtype, cache_dtype, lse_out, workspace, workspace_bytes,
+                                                     device_error, nullptr, stream);
 }
 
 pkv_status pkv_paged_decode_step_ex(void* out, const void* query, const void* key, const void* value, void* key_cache,

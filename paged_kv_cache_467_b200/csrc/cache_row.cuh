@@ -112,7 +112,6 @@ __device__ __forceinline__ void write_row(const void* src_row, void* cache, floa
       if (lane == 0) scales[dst_row] = scale;  // dst_row = slot * n_kv + h
     } else {
       const float scale = __ldg(scales + h);
-#pragma unroll
       constexpr __nv_fp8_interpretation_t fmt = KIND == WK_E5M2 ? __NV_E5M2 : __NV_E4M3;
 #pragma unroll
       for (int e = 0; e < EPL; ++e)

@@ -72,9 +72,18 @@ struct TcParams {
   // past the count) to read instead of every block; one KV head per unit
   const int32_t* pages;
   int k_pages;
-  // shared-prefix decode: logical blocks < skip_blocks were attended by the
-  // prefix pass; the piece holding a unit's first block starts from its state
+  // shared-prefix decode: logical blocks < skip_blocks are attended by the
+  // prefix pass, whose pieces the merge adds; every unit then leaves a piece
+  // (merge_all), a unit finished inside one CTA in unit_o / unit_lse
   int skip_blocks;
+  int merge_all;
+  float* unit_o;    // [num_seqs * n_q][D], normalised
+  float* unit_lse;  // [num_seqs * n_q], base 2
+  // the prefix pass runs beside this kernel: wait for it (the previous
+  // kernel) only before exiting, not before the work
+  int late_wait;
+  long long wait_limit;  // SM cycles a ring wait may spend before giving up
+  // start state of each unit's first piece (the KIVI residual pass)
   const float* pre_o;    // [n_kv][rows][D], normalised
   const float* pre_lse;  // [n_kv][rows], base 2
   int pre_rows;
@@ -89,11 +98,7 @@ constexpr float kLn2 = 0.6931471805599453f;
 // Slack (log2 units) of the running softmax maximum before it is moved.
 constexpr float kLazyLog2 = 8.f;
 
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
+__device__ __forceinline__ float ex2(float x) { return ex2_approx(x); }
 
 // Attended length of sequence s, clamped to what the launch and table cover.
 __device__ __forceinline__ int seq_len(const TcParams& p, int s, bool report) {
@@ -266,9 +271,11 @@ __device__ __forceinline__ int d_of(int mt, int hi, int g) {
 // decode kernel with programmatic serialisation, combines them: one CTA per
 // unit, a thread per (query head, 4 dims), so every piece's loads of a thread
 // are independent and the whole merge costs about two L2 round trips instead
-// of a serial tail in the decode kernel.  Pieces are combined in CTA order:
-// M = max lse_k, w_k = 2^(lse_k - M), o = sum w_k o_k / sum w_k,
-// lse = M + log2(sum w_k).
+// of a serial tail in the decode kernel.  Pieces are combined in a fixed
+// order: M = max lse_k, w_k = 2^(lse_k - M), o = sum w_k o_k / sum w_k,
+// lse = M + log2(sum w_k).  Under a shared prefix every unit is merged
+// (decode_merge_all_kernel): its own piece(s) (CTA pieces, or the unit's whole
+// piece) and then the prefix pass's split pieces of the same query row.
 struct MergeParams {
   void* out;
   float* lse_out;
@@ -276,6 +283,13 @@ struct MergeParams {
   const float* part_lse;
   const int2* desc;
   int HG, QH, n_q, num_ctas, act_bf16;
+  // shared prefix (merge_all): whole-unit pieces and the prefix pass's pieces
+  int merge_all;
+  const float* unit_o;
+  const float* unit_lse;
+  const float* pre_o;    // [n_kv][pre_rows][pre_splits][D]
+  const float* pre_lse;  // [n_kv][pre_rows][pre_splits]
+  int pre_rows, pre_splits, G, HPC;
 };
 
 template <int D>
@@ -286,7 +300,9 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
   const int2 d = p.desc[u];
   const int c0 = d.x & 0x3FFFFFFF, n = d.y;
   const bool c0_slot1 = (d.x >> 30) & 1;
-  if (n < 2 || c0 + n > p.num_ctas) return;  // whole unit in one CTA (written there), or no pieces
+  // whole unit in one CTA (written there), or no pieces; a descriptor out of
+  // range (only after a timed-out decode) is skipped
+  if (n < 2 || n > p.num_ctas || c0 >= p.num_ctas || c0 + n > p.num_ctas) return;
   const int s = u / p.HG, hg = u - s * p.HG;
   constexpr int V = D / 4;
   for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
@@ -322,6 +338,78 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
           make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
     if (p.lse_out && v == 0) p.lse_out[row] = (M + log2f(wsum)) * kLn2;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) decode_merge_all_kernel(const MergeParams p) {
+  grid_launch_dependents();
+  grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
+  const int u = blockIdx.x;
+  const int2 d = p.desc[u];
+  const int c0 = d.x & 0x3FFFFFFF;
+  int n = d.y;
+  const bool c0_slot1 = (d.x >> 30) & 1;
+  // a descriptor out of range (only after a timed-out decode) contributes nothing
+  if (n < 0 || n > p.num_ctas || c0 >= p.num_ctas || c0 + n > p.num_ctas) n = 0;
+  const int s = u / p.HG, hg = u - s * p.HG;
+  const int npre = p.pre_splits;
+  const bool whole = n < 2;  // the unit's one piece (n == 1) or none (n == 0)
+  constexpr int V = D / 4;
+  for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
+    const int h = idx / V, v = idx - h * V;
+    const long long row = (long long)s * p.n_q + hg * p.QH + h;
+    // the unit's own pieces: CTA k's slot (k == 0 may be the CTA's second slot)
+    const float* own_lse = p.part_lse + ((size_t)c0 * 2 + (c0_slot1 ? 1 : 0)) * p.QH + h;
+    const float* own_o = p.part_o + (((size_t)c0 * 2 + (c0_slot1 ? 1 : 0)) * p.QH + h) * D;
+    const size_t own_step = (size_t)2 * p.QH;  // from CTA k's slot 0 to CTA k + 1's
+    const size_t own_back = c0_slot1 ? (size_t)p.QH : 0;  // CTA c0 + 1 and on: slot 0
+    // the prefix pass's splits of this query row, consecutive
+    const size_t pre_row = npre ? ((size_t)(hg * p.HPC + h / p.G) * p.pre_rows + (size_t)s * p.G + h % p.G) : 0;
+    const float* pre_lse = p.pre_lse + pre_row * npre;
+    const float* pre_o = p.pre_o + pre_row * npre * D;
+    float M = -INFINITY;
+    if (!whole) {
+      M = __ldcg(own_lse);
+#pragma unroll 4
+      for (int k = 1; k < n; ++k) M = fmaxf(M, __ldcg(own_lse + k * own_step - own_back));
+    } else if (n == 1) {
+      M = __ldcg(p.unit_lse + row);
+    }
+#pragma unroll 4
+    for (int k = 0; k < npre; ++k) M = fmaxf(M, __ldcg(pre_lse + k));
+    float wsum = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto add = [&](float lse, const float* o) {
+      const float w = ex2(lse - M);
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(o) + v);
+      wsum += w;
+      acc.x += w * x.x;
+      acc.y += w * x.y;
+      acc.z += w * x.z;
+      acc.w += w * x.w;
+    };
+    if (M > -INFINITY) {
+      if (!whole) {
+        add(__ldcg(own_lse), own_o);
+#pragma unroll 4
+        for (int k = 1; k < n; ++k) add(__ldcg(own_lse + k * own_step - own_back), own_o + (k * own_step - own_back) * D);
+      } else if (n == 1) {
+        add(__ldcg(p.unit_lse + row), p.unit_o + row * D);
+      }
+#pragma unroll 4
+      for (int k = 0; k < npre; ++k) add(__ldcg(pre_lse + k), pre_o + (size_t)k * D);
+    }
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    if (p.act_bf16) {
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + row * D + 4 * v);
+      o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    } else {
+      reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * D)[v] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    if (p.lse_out && v == 0) p.lse_out[row] = wsum > 0.f ? (M + log2f(wsum)) * kLn2 : -INFINITY;
   }
 }
 
@@ -402,11 +490,18 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
   // Everything above read only context_lens and block_tables.  Under a
   // programmatic launch the previous kernel may still be running: wait for it
   // before touching queries, new rows, the cache, the workspace or outputs.
-  grid_wait_prerequisites();
+  // Beside the shared-prefix pass (late_wait) that kernel is the prefix pass,
+  // which touches none of these (it let this grid start only after its own
+  // wait for the kernel before it): the producer waits for it before exiting,
+  // so that this grid completes after it and the merge sees its pieces.
+  if (!p.late_wait) grid_wait_prerequisites();
 
   // ------------------------------------------------------------ producer
   if (warp == p.NCW) {
-    if (a >= b) return;
+    if (a >= b) {
+      if (p.late_wait) grid_wait_prerequisites();
+      return;
+    }
     int it = 0;
     int pstage = 0;       // ring stage of block `it`
     uint32_t ppass = 0;   // parity of the ring pass of block `it`
@@ -431,10 +526,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
         int ok = 1;
         if (lane == 0) {
           const int stage = pstage;
-          if (it >= p.stages && !mbar_wait(&empty[stage], ppass ^ 1u)) {
+          if (it >= p.stages && !mbar_wait(&empty[stage], ppass ^ 1u, p.wait_limit)) {
             flag_error(p.err, DEVERR_TIMEOUT);
             ok = 0;
-          } else if (p.new_key && lastk && !appended && !(appended = mbar_wait(append_done, 0))) {
+          } else if (p.new_key && lastk && !appended && !(appended = mbar_wait(append_done, 0, p.wait_limit))) {
             // the block holding a new token is read only after the consumers wrote it
             flag_error(p.err, DEVERR_TIMEOUT);
             ok = 0;
@@ -484,10 +579,12 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
         }
       }
     }
-    // Never leave with copies in flight: wait for the last stages issued.
+    // Never leave with copies in flight: wait for the last stages issued
+    // (with the full limit, whatever the ring waits were given).
     if (lane == 0) {
       for (int k = max(0, it - p.stages); k < it; ++k) mbar_wait(&full[k % p.stages], (k / p.stages) & 1);
     }
+    if (p.late_wait) grid_wait_prerequisites();
     return;
   }
 
@@ -509,6 +606,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       const int u = u0 + __ffs(empty_units) - 1;
       empty_units &= empty_units - 1;
       if (warp == 0 && lane == 0) p.desc[u] = make_int2(0, 0);
+      if (p.merge_all) continue;  // the merge writes it (from the prefix pieces alone)
       const int s = u / p.HG, hg = u - s * p.HG;
       for (int n = 0; n < 8; ++n) {
         if (qc * 8 + n >= p.G) break;
@@ -605,9 +703,11 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
   float acc[KS][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-  // Query words of a unit as loaded (bf16 pairs) and the FP8 head scales.
+  // Query words of a unit as loaded (bf16 pairs), in the order of the MMA B
+  // fragments.  BF16: dims ks*16 + 2c, +1 and ks*16 + 2c + 8, +9.  FP8: k-step
+  // ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
+  // (the order in which the FP8 K fragments take the stored bytes).
   uint32_t qraw[KS][2];
-  float raw_k_scale = 1.f, raw_v_scale = 1.f;
   auto fetch_query = [&](int uu) {
     const int ss = uu / p.HG, hh = uu - ss * p.HG;
     const int kv = hh * p.HPC + head_local;
@@ -617,34 +717,14 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
 #pragma unroll
     for (int ks = 0; ks < KS; ++ks) {
       if constexpr (CACHE == TC_BF16) {
-        // MMA B fragment: dims ks*16 + 2c, +1 and ks*16 + 2c + 8, +9
         qraw[ks][0] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c) / 2) : 0u;
         qraw[ks][1] = q_ok ? __ldg(q32 + (ks * 16 + 2 * c + 8) / 2) : 0u;
-      } else if constexpr (CACHE == TC_INT4) {
-        // k-step ks = 2w + h pairs dims 32c + 8w + 2h + {0, 4} and {1, 5} (the
-        // nibble pairs of the INT4 word w of lane column c); one 16-byte load
-        // of dims 32c + 8w .. + 7 serves ks = 2w and 2w + 1
-        if (ks & 1) continue;
-        const uint4 w = q_ok ? __ldg(reinterpret_cast<const uint4*>(q32 + (32 * c + 4 * ks) / 2))
-                             : make_uint4(0u, 0u, 0u, 0u);
-        qraw[ks][0] = prmt(w.x, w.z, 0x5410);
-        qraw[ks][1] = prmt(w.x, w.z, 0x7632);
-        qraw[ks + 1][0] = prmt(w.y, w.w, 0x5410);
-        qraw[ks + 1][1] = prmt(w.y, w.w, 0x7632);
       } else {
-        // k-step ks = h * 4 + k covers, for lane column c, dims (2c + h) * 16 + 4k + {0..3}
         const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
         const uint2 w = q_ok ? __ldg(reinterpret_cast<const uint2*>(q32 + d0 / 2)) : make_uint2(0u, 0u);
         qraw[ks][0] = w.x;
         qraw[ks][1] = w.y;
       }
-    }
-    if constexpr (tc_fp8(CACHE)) {
-      // the f16 operands hold E4M3 values / 256 (e4m3x2_hi_to_f16x2_div256), or
-      // E5M2 values exactly (an E5M2 byte is the top byte of its f16)
-      constexpr float fold = CACHE == TC_FP8 ? 256.f : 1.f;
-      raw_k_scale = __ldg(p.k_scale + kv) * fold;
-      raw_v_scale = __ldg(p.v_scale + kv) * fold;
     }
   };
 
@@ -742,7 +822,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       sa[2] = ((float)ah[2] + (float)al[2] * (1.f / 254.f)) * qs0;
       sa[3] = ((float)ah[3] + (float)al[3] * (1.f / 254.f)) * qs1;
     } else {
-      // lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes each)
+      // FP8: lane (g, c) reads rows g and g+8, chunks 2c and 2c+1 (16 bytes
+      // each); k-step ks takes the byte pairs (0, 1) -> k = 2c, 2c+1 and (2, 3)
+      // -> k = 2c+8, 2c+9 of word ks & 3 of chunk 2c + (ks >> 2), as f16 values
       uint4 kr[2][2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -755,17 +837,17 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
         const uint32_t w0 = (&kr[0][h].x)[k], w1 = (&kr[1][h].x)[k];
         uint32_t af[4];
         if constexpr (CACHE == TC_E5M2) {
-          // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, as the f16 top bytes
+          // an E5M2 byte is the top byte of the f16 of the same value
           af[0] = prmt(w0, 0u, 0x1404);
           af[1] = prmt(w1, 0u, 0x1404);
           af[2] = prmt(w0, 0u, 0x3424);
           af[3] = prmt(w1, 0u, 0x3424);
         } else {
-          // bytes (0,1) -> k = 2c, 2c+1 and bytes (2,3) -> k = 2c+8, 2c+9, values / 256
-          af[0] = e4m3x2_hi_to_f16x2_div256(prmt(w0, 0u, 0x1404));
-          af[1] = e4m3x2_hi_to_f16x2_div256(prmt(w1, 0u, 0x1404));
-          af[2] = e4m3x2_hi_to_f16x2_div256(prmt(w0, 0u, 0x3424));
-          af[3] = e4m3x2_hi_to_f16x2_div256(prmt(w1, 0u, 0x3424));
+          // E4M3 pairs through the hardware conversion (exact values); a code
+          // that reads as NaN sits in a row that is not attended, whose score
+          // the select below replaces by -inf
+          e4m3x4_to_f16x2x2(w0, af[0], af[2]);
+          e4m3x4_to_f16x2x2(w1, af[1], af[3]);
         }
         if (ks & 1) mma_f16(sb, af, qf[ks][0], qf[ks][1]);
         else mma_f16(sa, af, qf[ks][0], qf[ks][1]);
@@ -890,7 +972,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
           af[1] = i8x2_to_f16x2(ta, 0x4342);
           af[2] = i8x2_to_f16x2(tb, 0x4140);
           af[3] = i8x2_to_f16x2(tb, 0x4342);
-        } else {
+        } else if constexpr (CACHE == TC_E5M2) {
           // byte A of the token-2c row into bits [15:8], of the token-2c+1 row into [31:24]
           const uint32_t A = 2 * (mt & 1);
           const uint32_t s0 = ((4 + A) << 12) | ((4 + A) << 8) | (A << 4) | A;
@@ -899,20 +981,29 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
           af[1] = prmt((&x0.x)[wi], (&y0.x)[wi], s1);
           af[2] = prmt((&x1.x)[wi], (&y1.x)[wi], s0);
           af[3] = prmt((&x1.x)[wi], (&y1.x)[wi], s1);
-          if constexpr (CACHE == TC_FP8) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) af[k] = e4m3x2_hi_to_f16x2_div256(af[k]);
-          } else {
-            // E5M2 bytes are the f16 top bytes: clear the duplicated low bytes, and
-            // the rows past the attended ones (their codes may be inf or NaN)
-            af[0] &= mlo5;
-            af[1] &= mlo5;
-            af[2] &= mhi5;
-            af[3] &= mhi5;
+          // E5M2 bytes are the f16 top bytes: clear the duplicated low bytes, and
+          // the rows past the attended ones (their codes may be inf or NaN)
+          af[0] &= mlo5;
+          af[1] &= mlo5;
+          af[2] &= mhi5;
+          af[3] &= mhi5;
+        } else {
+          // E4M3: bytes A and A+1 of the token-2c and token-2c+1 rows as two
+          // pairs [2c, 2c+1] through the hardware conversion; rows past the
+          // attended ones may hold NaN codes, so partial blocks are masked
+          const uint32_t A = 2 * (mt & 1);
+          const uint32_t sel = A | ((4 + A) << 4) | ((A + 1) << 8) | ((5 + A) << 12);
+          e4m3x4_to_f16x2x2(prmt((&x0.x)[wi], (&y0.x)[wi], sel), af[0], af[1]);
+          e4m3x4_to_f16x2x2(prmt((&x1.x)[wi], (&y1.x)[wi], sel), af[2], af[3]);
+          if (partial) {
+            af[0] &= mlo;
+            af[1] &= mlo;
+            af[2] &= mhi;
+            af[3] &= mhi;
           }
         }
-        // INT8 and E4M3 values decode finite whatever the bytes, and masked
-        // tokens carry P = 0, so they need no V mask
+        // INT8 values decode finite whatever the bytes, and masked tokens
+        // carry P = 0, so they need no V mask
         mma_f16(acc[mt], af, pb0, pb1);
       }
     }
@@ -938,7 +1029,7 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
         pk ^= 1u;
       }
       stage[k] = sk;
-      if (!mbar_wait(&full[sk], pk)) return false;
+      if (!mbar_wait(&full[sk], pk, p.wait_limit)) return false;
       st[k] = smem + (size_t)sk * p.stage_bytes;
       if constexpr (CACHE == TC_KIVI)
         valid[k] = 0xFFFFu;  // full blocks only
@@ -1022,7 +1113,10 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
           qf[ks][0] = qraw[ks][0];
           qf[ks][1] = qraw[ks][1];
         }
-      } else if constexpr (tc_fp8(CACHE)) {  // INT8 / INT4 quantise their queries below
+      } else if constexpr (tc_fp8(CACHE)) {
+        // the query as f16 pairs in the order of the FP8 K fragments; the codes
+        // become f16 of their exact values, so the per-head scales apply as they are
+        const int kv = hg * p.HPC + head_local;
         if (p.act_bf16) {
           fetch_query(u);
 #pragma unroll
@@ -1031,40 +1125,20 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
             qf[ks][1] = pack_f16(__uint_as_float(qraw[ks][1] << 16), __uint_as_float(qraw[ks][1] & 0xFFFF0000u));
           }
         } else {
-          // float32 queries: loaded and rounded to f16 here (not prefetched)
-          const int kv = hg * p.HPC + head_local;
           const bool q_ok = qc * 8 + g < p.G;
-          const size_t qoff = ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
-          const float* qrow = reinterpret_cast<const float*>(p.query) + qoff;
+          const float* qrow = reinterpret_cast<const float*>(p.query) + ((size_t)s * p.n_q + kv * p.G + qc * 8 + g) * D;
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
-            if constexpr (CACHE == TC_INT4) {
-              // dims 32c + 8w + 2h + {0, 4} and {1, 5} for ks = 2w + h (as fetch_query)
-              const int d0 = 32 * c + 8 * (ks >> 1) + 2 * (ks & 1);
-              float2 lo = make_float2(0.f, 0.f), hi = make_float2(0.f, 0.f);
-              if (q_ok) {
-                lo = __ldg(reinterpret_cast<const float2*>(qrow + d0));
-                hi = __ldg(reinterpret_cast<const float2*>(qrow + d0 + 4));
-              }
-              qf[ks][0] = pack_f16(lo.x, hi.x);
-              qf[ks][1] = pack_f16(lo.y, hi.y);
-            } else {
-              const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
-              float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (q_ok) w = __ldg(reinterpret_cast<const float4*>(qrow + d0));
-              qf[ks][0] = pack_f16(w.x, w.y);
-              qf[ks][1] = pack_f16(w.z, w.w);
-            }
-          }
-          if constexpr (tc_fp8(CACHE)) {
-            constexpr float fold = CACHE == TC_FP8 ? 256.f : 1.f;
-            raw_k_scale = __ldg(p.k_scale + kv) * fold;
-            raw_v_scale = __ldg(p.v_scale + kv) * fold;
+            const int d0 = (2 * c + (ks >> 2)) * 16 + 4 * (ks & 3);
+            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (q_ok) w = __ldg(reinterpret_cast<const float4*>(qrow + d0));
+            qf[ks][0] = pack_f16(w.x, w.y);
+            qf[ks][1] = pack_f16(w.z, w.w);
           }
         }
+        head_k_scale = __ldg(p.k_scale + kv);
+        head_v_scale = __ldg(p.v_scale + kv);
       }
-      head_k_scale = raw_k_scale;
-      head_v_scale = raw_v_scale;
       if constexpr (tc_row_scaled(CACHE)) {
         // this lane's 32 dims 32c .. 32c+31 of query head g, quantised per head:
         // t = q * 127 / max|q|, h = rint(t), l = rint((t - h) * 254), both in
@@ -1227,7 +1301,22 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       const float lse0 = m0 + log2f(lt0), lse1 = m1 + log2f(lt1);
       const bool contained = P[u] >= a && P[u + 1] <= b;
       const long long row0 = (long long)s * p.n_q + hg * QH + qbase_local + 2 * c;  // head 2c of this lane
-      if (contained) {
+      if (contained && p.merge_all) {
+        // the whole unit's piece, for the merge with the shared prefix's pieces
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int dd = d_of<CACHE, D>(mt, hi, g);
+            if (head0_ok) __stcg(p.unit_o + row0 * D + dd, acc[mt][2 * hi] * inv0);
+            if (head1_ok) __stcg(p.unit_o + (row0 + 1) * D + dd, acc[mt][2 * hi + 1] * inv1);
+          }
+        }
+        if (g == 0) {
+          if (head0_ok) __stcg(p.unit_lse + row0, lse0);
+          if (head1_ok) __stcg(p.unit_lse + row0 + 1, lse1);
+        }
+      } else if (contained) {
 #pragma unroll
         for (int mt = 0; mt < KS; ++mt) {
 #pragma unroll
@@ -1333,7 +1422,7 @@ static pkv_status make_kivi_scale_map(CUtensorMap* map, const float* k_scale, in
 
 template <int CACHE, int D, int MAXW, int MINB = 1>
 static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
-                                 const TcParams& prm, cudaStream_t stream) {
+                                 const TcParams& prm, const PrefixPieces& pre, cudaStream_t stream) {
   auto kern = decode_tc_kernel<CACHE, D, MAXW, MINB>;
   static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
   if ((int)plan.smem_bytes > configured_bytes) {
@@ -1368,6 +1457,15 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mp.n_q = prm.n_q;
   mp.num_ctas = plan.num_ctas;
   mp.act_bf16 = prm.act_bf16;
+  mp.merge_all = prm.merge_all;
+  mp.unit_o = prm.unit_o;
+  mp.unit_lse = prm.unit_lse;
+  mp.pre_o = pre.o;
+  mp.pre_lse = pre.lse;
+  mp.pre_rows = pre.rows;
+  mp.pre_splits = pre.splits;
+  mp.G = plan.G;
+  mp.HPC = plan.HPC;
   cudaLaunchConfig_t mcfg = {};
   mcfg.gridDim = dim3(plan.units);
   mcfg.blockDim = dim3((unsigned)std::min(256, (mp.QH * (D / 4) + 31) / 32 * 32));
@@ -1378,7 +1476,8 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mattr[0].val.programmaticStreamSerializationAllowed = 1;
   mcfg.attrs = mattr;
   mcfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&mcfg, decode_merge_kernel<D>, mp);
+  e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, decode_merge_all_kernel<D>, mp)
+                    : cudaLaunchKernelEx(&mcfg, decode_merge_kernel<D>, mp);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_merge_kernel launch");
   return PKV_OK;
@@ -1391,12 +1490,12 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
 // flight: 15 warps per SM instead of 12 (INT4 -13 %, INT8 and E4M3 -5 %).
 template <int CACHE, int D>
 static pkv_status launch_one(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
-                             const TcParams& prm, cudaStream_t stream) {
-  if constexpr (CACHE != TC_BF16) {
-    if (plan.NCW <= 4) return launch_variant<CACHE, D, 4, kQuantCtasPerSm>(plan, km, vm, sm, prm, stream);
+                             const TcParams& prm, const PrefixPieces& pre, cudaStream_t stream) {
+  if constexpr (tc_narrow(CACHE)) {
+    if (plan.NCW <= 4) return launch_variant<CACHE, D, 4, kQuantCtasPerSm>(plan, km, vm, sm, prm, pre, stream);
   }
-  if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, sm, prm, stream);
-  return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, sm, prm, stream);
+  if (plan.NCW <= 8) return launch_variant<CACHE, D, 8>(plan, km, vm, sm, prm, pre, stream);
+  return launch_variant<CACHE, D, kMaxConsumerWarps>(plan, km, vm, sm, prm, pre, stream);
 }
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream) {
@@ -1416,12 +1515,14 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   } else {
     sm = km;  // unused
   }
-  PrefixState pre = a.prefix;
-  if (a.skip_blocks > 0 && a.prefix_ws) {
-    // shared prefix first; the decode over the sequences' own blocks then
-    // starts from its state (queued with programmatic serialisation)
-    st = launch_prefix(s, km, vm, a.query, a.block_tables, a.num_blocks, a.skip_blocks, a.sm_scale, a.prefix_ws,
-                       a.device_error, &pre, stream);
+  const long long wait_limit = a.wait_limit > 0 ? a.wait_limit : kWaitLimitCycles;
+  PrefixPieces pieces;
+  const bool shared_prefix = a.skip_blocks > 0 && a.prefix_ws;
+  if (shared_prefix) {
+    // The shared prefix's pass first; the decode over each sequence's own
+    // blocks, queued with programmatic serialisation, runs beside it (or after
+    // it, prefix_serial), and the merge combines both sides' pieces.
+    st = launch_prefix(s, km, vm, a, wait_limit, &pieces, stream);
     if (st != PKV_OK) return st;
   }
 
@@ -1454,9 +1555,14 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.pages = a.pages;
   prm.k_pages = a.k_pages;
   prm.skip_blocks = a.skip_blocks;
-  prm.pre_o = pre.o;
-  prm.pre_lse = pre.lse;
-  prm.pre_rows = pre.rows;
+  prm.merge_all = shared_prefix ? 1 : 0;
+  prm.unit_o = pieces.unit_o;
+  prm.unit_lse = pieces.unit_lse;
+  prm.late_wait = shared_prefix && !a.prefix_serial ? 1 : 0;
+  prm.wait_limit = wait_limit;
+  prm.pre_o = a.prefix.o;
+  prm.pre_lse = a.prefix.lse;
+  prm.pre_rows = a.prefix.rows;
   prm.whole_blocks = kivi ? 1 : 0;
   prm.G = plan.G;
   prm.QC = plan.QC;
@@ -1471,14 +1577,14 @@ pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, 
   prm.tx_bytes = plan.tx_bytes;
 
   if (plan.cache_kind == TC_BF16) {
-    if (s.head_dim == 64) return launch_one<TC_BF16, 64>(plan, km, vm, sm, prm, stream);
-    return launch_one<TC_BF16, 128>(plan, km, vm, sm, prm, stream);
+    if (s.head_dim == 64) return launch_one<TC_BF16, 64>(plan, km, vm, sm, prm, pieces, stream);
+    return launch_one<TC_BF16, 128>(plan, km, vm, sm, prm, pieces, stream);
   }
-  if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, sm, prm, stream);
-  if (plan.cache_kind == TC_INT4) return launch_one<TC_INT4, 128>(plan, km, vm, sm, prm, stream);
-  if (plan.cache_kind == TC_E5M2) return launch_one<TC_E5M2, 128>(plan, km, vm, sm, prm, stream);
-  if (plan.cache_kind == TC_KIVI) return launch_one<TC_KIVI, 128>(plan, km, vm, sm, prm, stream);
-  return launch_one<TC_FP8, 128>(plan, km, vm, sm, prm, stream);
+  if (plan.cache_kind == TC_INT8) return launch_one<TC_INT8, 128>(plan, km, vm, sm, prm, pieces, stream);
+  if (plan.cache_kind == TC_INT4) return launch_one<TC_INT4, 128>(plan, km, vm, sm, prm, pieces, stream);
+  if (plan.cache_kind == TC_E5M2) return launch_one<TC_E5M2, 128>(plan, km, vm, sm, prm, pieces, stream);
+  if (plan.cache_kind == TC_KIVI) return launch_one<TC_KIVI, 128>(plan, km, vm, sm, prm, pieces, stream);
+  return launch_one<TC_FP8, 128>(plan, km, vm, sm, prm, pieces, stream);
 }
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -1509,7 +1615,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     // four CTAs per SM measured best for bf16; the quantised caches, whose
     // dequantisation is heavy on the ALUs, do best with four consumer warps per
     // CTA and three CTAs per SM (narrow launch bound, more warps in flight).
-    const int warps = pl.cache_kind != TC_BF16 ? 4 : 2;
+    const int warps = tc_narrow(pl.cache_kind) ? 4 : 2;
     pl.HPC = 1;
     for (int h = std::min(s.n_kv, warps); h >= 1; --h) {
       if (s.n_kv % h == 0 && h * pl.QC <= warps) {
@@ -1538,7 +1644,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
     // whole shared memory (~190 KB) of K/V in flight; fewer CTAs per SM only
     // when even 2 stages do not fit.
     stages = 2;
-    const int target_per_sm = (pl.cache_kind != TC_BF16 && pl.NCW <= 4) ? kQuantCtasPerSm : kTargetCtasPerSm;
+    const int target_per_sm = (tc_narrow(pl.cache_kind) && pl.NCW <= 4) ? kQuantCtasPerSm : kTargetCtasPerSm;
     for (int per = target_per_sm; per >= 1; --per) {
       const size_t budget = (size_t)kSmemPerSm / per - 1024;
       if (budget < fixed) continue;
@@ -1554,7 +1660,7 @@ pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan
   pl.smem_bytes = (size_t)stages * pl.stage_bytes + fixed;
   if (pl.smem_bytes > (size_t)optin) return want_stages > 0 ? PKV_ERR_INVALID_ARG : PKV_ERR_UNSUPPORTED;
   // CTAs resident per SM from shared memory alone (1 KB reserved per CTA).
-  const int per_sm = std::max(1, std::min((pl.cache_kind != TC_BF16 && pl.NCW <= 4) ? kQuantCtasPerSm
+  const int per_sm = std::max(1, std::min((tc_narrow(pl.cache_kind) && pl.NCW <= 4) ? kQuantCtasPerSm
                                                                                     : kTargetCtasPerSm,
                                           (int)(kSmemPerSm / (pl.smem_bytes + 1024))));
   const int want_ctas = tuning ? tuning->num_ctas : 0;

@@ -25,6 +25,10 @@ __host__ __device__ constexpr bool tc_row_scaled(int c) { return c == TC_INT8 ||
 // V scaled per (token, head): the row-scaled formats and the 2-bit KIVI cache,
 // whose K scales are per (block, head, channel)
 __host__ __device__ constexpr bool tc_v_row_scaled(int c) { return tc_row_scaled(c) || c == TC_KIVI; }
+// Caches whose decode is bound by the work of unpacking codes (every format but
+// BF16): 3 CTAs of up to 4 consumer warps per SM under a narrow register
+// bound, for more warps in flight.  BF16 takes 4 CTAs of 2 warps.
+__host__ __device__ constexpr bool tc_narrow(int c) { return c != TC_BF16; }
 
 struct DecodeShape {
   int num_seqs, n_q, n_kv, head_dim, block_size;
@@ -48,16 +52,29 @@ struct TcPlan {
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
 
-// Shared-prefix pass (prefix.cu): per (KV head, query row = s * G + head in
-// group) the normalised output over the prefix and its base-2 lse (the
-// prefix's splits already combined), which the decode kernel over each
-// sequence's own blocks starts from.
-constexpr int kMaxPrefixSplits = 64;
+// Start state of a decode unit (kivi.cu's residual pass): per (KV head,
+// query row = s * G + head in group) the normalised output and its base-2 lse,
+// which the decode over the quantised blocks starts from.
 struct PrefixState {
   const float* o = nullptr;    // [n_kv][rows][head_dim]
   const float* lse = nullptr;  // [n_kv][rows]
-  int splits = 0;              // splits of the prefix pass (combined into o / lse)
+  int splits = 0;
   int rows = 0;
+};
+
+// Shared-prefix pass (prefix.cu): per (KV head, query row = s * G + head in
+// group, split of the prefix) the normalised output over the split's tokens
+// and its base-2 lse.  The merge launch combines these pieces with the pieces
+// of each sequence's own blocks; a decode unit that one CTA finished whole
+// leaves its piece in unit_o / unit_lse.
+constexpr int kMaxPrefixSplits = 64;
+struct PrefixPieces {
+  const float* o = nullptr;    // [n_kv][rows][splits][head_dim]
+  const float* lse = nullptr;  // [n_kv][rows][splits]
+  int splits = 0;
+  int rows = 0;
+  float* unit_o = nullptr;     // [num_seqs * n_q][head_dim]
+  float* unit_lse = nullptr;   // [num_seqs * n_q]
 };
 
 struct TcArgs {
@@ -91,6 +108,9 @@ struct TcArgs {
   int skip_blocks = 0;
   PrefixState prefix;
   void* prefix_ws = nullptr;  // scratch of the prefix pass (prefix_workspace_bytes)
+  int prefix_splits = 0;      // splits of the prefix pass (0 = automatic)
+  bool prefix_serial = false; // the decode waits for the prefix pass instead of running beside it
+  long long wait_limit = 0;   // SM cycles a bounded wait of the decode kernels spends (0 = default)
 };
 
 pkv_status launch_tc(const DecodeShape& s, const TcPlan& plan, const TcArgs& a, cudaStream_t stream);
@@ -125,11 +145,10 @@ pkv_status launch_kivi_quantize_blocks(const void* key_rows, const void* value_r
                                        int64_t n, void* key_cache, void* value_cache, float* k_scale, float* v_scale,
                                        int n_kv, int64_t num_blocks, int32_t* device_error, cudaStream_t stream);
 
-size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks);
+size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks, int want_splits);
 pkv_status make_pool_map(CUtensorMap* map, const void* base, int elem, int chunk_bytes, int row_bytes, int64_t rows);
-pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const void* query,
-                         const int32_t* block_tables, int64_t num_blocks, int prefix_blocks, float sm_scale,
-                         void* prefix_ws, int32_t* device_error, PrefixState* state, cudaStream_t stream);
+pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const TcArgs& a,
+                         long long wait_limit, PrefixPieces* pieces, cudaStream_t stream);
 
 pkv_status launch_decode_f32(const DecodeShape& s, const TcArgs& a, cudaStream_t stream);
 

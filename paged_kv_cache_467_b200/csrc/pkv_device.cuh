@@ -16,6 +16,7 @@ enum : int {
   DEVERR_BLOCK_RANGE = 0x2,
   DEVERR_CONTEXT_LEN = 0x4,
   DEVERR_TIMEOUT = 0x8,
+  DEVERR_PREFIX = 0x10,
 };
 
 // A bounded wait gives up after this many SM clock cycles (about 1 s at 2 GHz).
@@ -60,12 +61,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; false if the wait ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false if the wait ran
+// out (after `limit` SM clock cycles).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }
@@ -174,6 +176,25 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D(16x8, f32) += A(16x32) * B(32x8), FP8 operands: A E4M3 (a_e5m2 = false)
+// or E5M2 codes, B E4M3.
+template <bool A_E5M2>
+__device__ __forceinline__ void mma_fp8(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  if constexpr (A_E5M2) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e5m2.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  } else {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+  }
+}
+
 // Four int8 values packed into a word, element 0 in the low byte.
 __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
   return (uint32_t)(a & 0xFF) | ((uint32_t)(b & 0xFF) << 8) | ((uint32_t)(c & 0xFF) << 16) | ((uint32_t)d << 24);
@@ -211,6 +232,19 @@ __device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t biased_word, uint32_t
   __half2 v = *reinterpret_cast<const __half2*>(&h);
   v = __hsub2(v, __half2half2(__ushort_as_half(0x6480)));  // 0x6480 = 1152.0
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The two E4M3 pairs of w (bytes 0-1 and bytes 2-3) -> two f16x2 words holding
+// the codes' values exactly (the hardware conversion; NaN codes give NaN).
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n"
+      "  .reg .b16 l, h;\n"
+      "  mov.b32 {l, h}, %2;\n"
+      "  cvt.rn.f16x2.e4m3x2 %0, l;\n"
+      "  cvt.rn.f16x2.e4m3x2 %1, h;\n"
+      "}\n"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 // Two E4M3 bytes held in bits [15:8] and [31:24] of t (other bits ignored) ->
@@ -259,6 +293,13 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
+}
+
+// 2^x on the special-function unit (flush-to-zero, approximate).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ float warp_max(float v) {

@@ -1,21 +1,30 @@
-// Shared-prefix pass of decode attention.  When every sequence of a batch
-// starts with the same physical blocks (a common system prompt: "Chapter 18 -
-// KV-Cache Optimization Strategies", Prefix Caching; "KV Cache Engineering for
-// LLM Serving", section 11), the attention over those blocks is computed once
-// per KV head for the queries of all sequences together: the scores are a
-// dense [S*G x 16] x [16 x d] product per block instead of S separate
-// [G x 16] ones, and the prefix is read once per query tile instead of once
-// per sequence.  The pass is split along the prefix; each split leaves a
-// normalised partial output and its base-2 log-sum-exp per query row, a small
-// second launch combines the splits (softmax states merge exactly:
-// M = max lse_i, o = sum 2^(lse_i - M) o_i / sum 2^(lse_i - M)), and the
-// decode kernel over each sequence's own blocks starts from that state.
+// Shared-prefix pass of decode attention on the fifth-generation tensor cores.
 //
-// CTA = 4 warps x 16 query rows of one KV head, one split of the prefix.  Q
-// fragments stay in registers; K and V blocks come through a ring of TMA
-// stages (the decode kernel's pool view: 16 rows x 128-byte chunks, 128-byte
-// swizzle); S = Q K^T and O += P V on m16n8k16 BF16 MMAs, P reused from the
-// score accumulators.
+// When every sequence of a batch starts with the same physical blocks (a
+// common system prompt: "Chapter 18 - KV-Cache Optimization Strategies",
+// Prefix Caching; "KV Cache Engineering for LLM Serving", section 11), the
+// attention over those blocks is a dense product: per KV head, the
+// R = num_seqs * G query rows against the prefix's tokens.  This pass computes
+// it once per KV head for all rows together, so each K/V tile of the prefix is
+// read by ceil(R / 128) CTAs instead of by every sequence.
+//
+// CTA = one KV head, 128 query rows (the MMA's M), one split of the prefix.
+//  * Q tile [128 x D] bf16 in shared memory, K-major with the 128-byte swizzle.
+//  * K and V of 64 tokens (four 16-token blocks) per chunk come by TMA through
+//    a two-stage ring, in the pool's own row layout: K is the K-major B
+//    operand of S = Q K^T, V the MN-major B operand of O += P V.
+//  * S [128 x 64] and O [128 x D] accumulate in tensor memory (fp32).  One
+//    thread issues the tcgen05.mma instructions and commits them to mbarriers.
+//  * Each of the 128 threads owns one query row (one TMEM lane): it reads its
+//    64 scores with tcgen05.ld, keeps the row's running max and sum (online
+//    softmax in base 2, the max moved only past 2^8 of slack, rescaling its O
+//    row in tensor memory then), and writes its bf16 probabilities into the P
+//    tile, the K-major A operand of P V.
+//  * The split's result per row, normalised o and base-2 lse, is one piece of
+//    the final merge, next to the pieces of the sequence's own blocks.
+// The CTAs that hold KV head 0 also check the prefix contract: every
+// sequence's first prefix_blocks table entries equal row 0's, and every
+// context is longer than the prefix.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -24,347 +33,403 @@
 
 #include "internal.h"
 #include "pkv_device.cuh"
+#include "tcgen05.cuh"
 
 namespace pkv {
 
-constexpr int kPrefixWarps = 4;
-constexpr int kPrefixStages = 4;
+constexpr int kPfxRows = 128;   // query rows per CTA (MMA M, TMEM lanes)
+constexpr int kPfxTok = 64;     // tokens per chunk (N of Q K^T, K of P V)
+constexpr int kPfxBlocks = kPfxTok / kBlockSize;
+constexpr int kPfxStages = 2;
+constexpr int kPfxThreads = 128;
+constexpr uint32_t kPfxTmemCols = 256;  // S at columns [0, 64), O at [128, 128 + D)
+constexpr uint32_t kPfxOCol = 128;
+
+template <int D>
+struct PfxLayout {
+  static constexpr int kDBlk = D / 64;                    // 128-byte column blocks of a bf16 row
+  static constexpr uint32_t kQ = kPfxRows * D * 2;        // [dblk][128 rows][128 B]
+  static constexpr uint32_t kKV = kPfxTok * D * 2;        // [dblk][64 tokens][128 B]
+  static constexpr uint32_t kStage = 2 * kKV;             // K then V
+  static constexpr uint32_t kP = kPfxRows * kPfxTok * 2;  // [128 rows][128 B]
+  static constexpr uint32_t kOffStage = kQ;
+  static constexpr uint32_t kOffP = kOffStage + kPfxStages * kStage;
+  static constexpr uint32_t kOffBar = kOffP + kP;
+  static constexpr uint32_t kBytes = kOffBar + 128;
+  static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
+};
 
 struct PrefixParams {
-  const __nv_bfloat16* query;  // [num_seqs, n_q, D]
-  const int32_t* block_tables;  // the prefix is the first prefix_blocks entries of row 0
+  const __nv_bfloat16* query;    // [num_seqs, n_q, D]
+  const int32_t* block_tables;   // the prefix is the first prefix_blocks entries of row 0
+  const int32_t* context_lens;
   int* err;
   float* part_o;    // [n_kv][rows][splits][D]
   float* part_lse;  // [n_kv][rows][splits], base 2
   long long num_blocks;
-  int rows, n_q, n_kv, G, prefix_blocks, splits, per_split;
+  long long wait_limit;
+  int rows, num_seqs, n_q, n_kv, G, prefix_blocks, max_blocks_per_seq;
+  int splits, chunks_per_split;
   float scale_log2;
 };
 
-__device__ __forceinline__ float ex2f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
+// Every sequence shares row 0's first prefix_blocks entries and is longer than
+// the prefix; violations set PKV_DEVERR_PREFIX / PKV_DEVERR_CONTEXT_LEN.  The
+// CTAs of KV head 0 share the check: this CTA's tile of sequences over its
+// split's blocks.
+__device__ void check_prefix_contract(const PrefixParams& p, int tile, int b0, int nblk) {
+  const int s_first = tile * kPfxRows / p.G;
+  const int s_last = min(p.num_seqs - 1, (tile * kPfxRows + kPfxRows - 1) / p.G);
+  const int nseq = s_last - s_first + 1;
+  bool bad_prefix = false, bad_len = false;
+  for (int idx = threadIdx.x; idx < nseq * nblk; idx += blockDim.x) {
+    const int s = s_first + idx / nblk, b = b0 + idx % nblk;
+    if (s > 0 && __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + b) != __ldg(p.block_tables + b))
+      bad_prefix = true;
+  }
+  if (b0 == 0) {
+    for (int s = s_first + (int)threadIdx.x; s <= s_last; s += blockDim.x)
+      if (__ldg(p.context_lens + s) <= p.prefix_blocks * kBlockSize) bad_len = true;
+  }
+  if (bad_prefix) flag_error(p.err, DEVERR_PREFIX);
+  if (bad_len) flag_error(p.err, DEVERR_CONTEXT_LEN);
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPrefixWarps * 32) prefix_attn_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                                          const __grid_constant__ CUtensorMap vmap,
-                                                                          const PrefixParams p) {
-  constexpr int kChunks = D * 2 / 128;
-  constexpr int kTile = kChunks * 2048;  // one head's 16-row tile of K (or V)
-  constexpr int KS = D / 16;
+__global__ void __launch_bounds__(kPfxThreads, 1)
+    prefix_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                     const PrefixParams p) {
+  using Ly = PfxLayout<D>;
+  constexpr int KS = D / 16;  // k-steps of Q K^T
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t full[kPrefixStages];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const int kv = blockIdx.y, split = blockIdx.z;
-  const int b0 = split * p.per_split, b1 = min(b0 + p.per_split, p.prefix_blocks);
-  const int nblk = max(0, b1 - b0);
+  uint8_t* q_tile = smem;
+  uint8_t* p_tile = smem + Ly::kOffP;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kOffBar);  // [kPfxStages] K/V chunk landed
+  uint64_t* empty = full + kPfxStages;                                // [kPfxStages] P V of the chunk done
+  uint64_t* bar_s = empty + kPfxStages;                               // S of the next chunk ready
+  uint64_t* bar_done = bar_s + 1;                                     // every MMA of the CTA done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
 
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tile = blockIdx.x, kv = blockIdx.y, split = blockIdx.z;
+  const int b0 = split * p.chunks_per_split * kPfxBlocks;
+  const int b1 = min(b0 + p.chunks_per_split * kPfxBlocks, p.prefix_blocks);
+  const int nblk = max(0, b1 - b0);
+  const int nchunks = (nblk + kPfxBlocks - 1) / kPfxBlocks;
+
+  // The previous kernel on the stream may still run: wait for it before
+  // reading anything, then let the next kernel be scheduled.
+  grid_wait_prerequisites();
   grid_launch_dependents();
+
   if (tid == 0) {
-    for (int k = 0; k < kPrefixStages; ++k) mbar_init(&full[k], 1);
+    for (int k = 0; k < kPfxStages; ++k) {
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_done, 1);
     fence_barrier_init();
     prefetch_tensormap(&kmap);
     prefetch_tensormap(&vmap);
   }
-  __syncthreads();
-  grid_wait_prerequisites();
-
-  auto issue = [&](int j) {  // block b0 + j into stage j % kPrefixStages
-    const int stage = j % kPrefixStages;
-    int phys = __ldg(p.block_tables + b0 + j);
-    if (phys < 0 || (long long)phys >= p.num_blocks) {
-      flag_error(p.err, DEVERR_BLOCK_RANGE);
-      phys = -1;  // row -16: the TMA zero-fills the box
-    }
-    uint8_t* st = smem + (size_t)stage * 2 * kTile;
-    mbar_arrive_expect_tx(&full[stage], 2 * kTile);
-#pragma unroll
-    for (int ch = 0; ch < kChunks; ++ch) {
-      tma_load_3d(st + ch * 2048, &kmap, 0, kv * kChunks + ch, phys * kBlockSize, &full[stage]);
-      tma_load_3d(st + kTile + ch * 2048, &vmap, 0, kv * kChunks + ch, phys * kBlockSize, &full[stage]);
-    }
-  };
-  if (tid == 0)
-    for (int j = 0; j < min(nblk, kPrefixStages); ++j) issue(j);
-
-  // ---- this warp's 16 query rows as A fragments (rows past the batch are 0)
-  const int row0 = blockIdx.x * (kPrefixWarps * 16) + warp * 16;
-  uint32_t qa[KS][4];
-  {
-    const int ra = row0 + g, rb = row0 + g + 8;
-    const bool oka = ra < p.rows, okb = rb < p.rows;
-    const uint32_t* qa_row = reinterpret_cast<const uint32_t*>(
-        p.query + ((size_t)(oka ? ra / p.G : 0) * p.n_q + kv * p.G + (oka ? ra % p.G : 0)) * D);
-    const uint32_t* qb_row = reinterpret_cast<const uint32_t*>(
-        p.query + ((size_t)(okb ? rb / p.G : 0) * p.n_q + kv * p.G + (okb ? rb % p.G : 0)) * D);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      qa[ks][0] = oka ? __ldg(qa_row + ks * 8 + c) : 0u;
-      qa[ks][1] = okb ? __ldg(qb_row + ks * 8 + c) : 0u;
-      qa[ks][2] = oka ? __ldg(qa_row + ks * 8 + 4 + c) : 0u;
-      qa[ks][3] = okb ? __ldg(qb_row + ks * 8 + 4 + c) : 0u;
-    }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kPfxTmemCols);
+    tmem_relinquish();
   }
+  if (kv == 0) check_prefix_contract(p, tile, b0, nblk);
 
-  float o[D / 8][4];
+  // ---- K/V chunk c (blocks b0 + 4c ..) into stage c % 2; blocks past the
+  // split, and table entries outside the pool, read as zeros (TMA fill)
+  auto issue_chunk = [&](int c) {
+    const int stage = c % kPfxStages;
+    uint8_t* kst = smem + Ly::kOffStage + stage * Ly::kStage;
+    uint8_t* vst = kst + Ly::kKV;
+    mbar_arrive_expect_tx(&full[stage], Ly::kStage);
 #pragma unroll
-  for (int dt = 0; dt < D / 8; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;  // rows g and g + 8
-
-  // ldmatrix row addresses: K (non-transposed) and V (transposed), tokens 0..15
-  const int mi = lane >> 3, r8 = lane & 7;
-  const int k_tok = r8 + (mi >> 1) * 8, k_half = mi & 1;  // matrices (tok 0-7 | 8-15) x (d 0-7 | 8-15)
-  const int v_tok = r8 + (mi & 1) * 8, v_dt = mi >> 1;    // matrices (tok 0-7 | 8-15) x (d-tile dt | dt + 1)
-
-  bool ok = true;
-  int j = 0;
-  for (; j < nblk; ++j) {
-    const int stage = j % kPrefixStages;
-    ok = mbar_wait(&full[stage], (j / kPrefixStages) & 1);
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    const uint32_t kt = smem_addr(smem + (size_t)stage * 2 * kTile);
-    const uint32_t vt = kt + kTile;
-
-    // ---- S = Q K^T: [16 rows x 16 tokens] as two n8 tiles
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < kPfxBlocks; ++i) {
+      const int b = b0 + c * kPfxBlocks + i;
+      int phys = -1;
+      if (b < b1) {
+        phys = __ldg(p.block_tables + b);
+        if (phys < 0 || (long long)phys >= p.num_blocks) {
+          flag_error(p.err, DEVERR_BLOCK_RANGE);
+          phys = -1;
+        }
+      }
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int piece = (ks & 3) * 2 + k_half;
-      uint32_t b[4];
-      ldmatrix_x4(b, kt + (ks >> 2) * 2048 + k_tok * 128 + ((piece ^ (k_tok & 7)) << 4));
-      mma_bf16(s0, qa[ks], b[0], b[1]);
-      mma_bf16(s1, qa[ks], b[2], b[3]);
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      s0[e] *= p.scale_log2;
-      s1[e] *= p.scale_log2;
-    }
-    // ---- online softmax over the block, rows g (s*[0], s*[1]) and g + 8 (s*[2], s*[3])
-    float mx_a = fmaxf(fmaxf(s0[0], s0[1]), fmaxf(s1[0], s1[1]));
-    float mx_b = fmaxf(fmaxf(s0[2], s0[3]), fmaxf(s1[2], s1[3]));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    // lazy rescale: the reference max moves (and the accumulators are
-    // rescaled) only when a score exceeds it by more than 2^8, so P <= 2^8
-    if (__any_sync(0xffffffffu, mx_a > m_a + 8.f || mx_b > m_b + 8.f)) {
-      const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-      const float al_a = ex2f(m_a - mn_a), al_b = ex2f(m_b - mn_b);
-      m_a = mn_a;
-      m_b = mn_b;
-      l_a *= al_a;
-      l_b *= al_b;
-#pragma unroll
-      for (int dt = 0; dt < D / 8; ++dt) {
-        o[dt][0] *= al_a;
-        o[dt][1] *= al_a;
-        o[dt][2] *= al_b;
-        o[dt][3] *= al_b;
+      for (int db = 0; db < Ly::kDBlk; ++db) {
+        const uint32_t off = db * (kPfxTok * 128) + i * (kBlockSize * 128);
+        tma_load_3d(kst + off, &kmap, 0, kv * Ly::kDBlk + db, phys * kBlockSize, &full[stage]);
+        tma_load_3d(vst + off, &vmap, 0, kv * Ly::kDBlk + db, phys * kBlockSize, &full[stage]);
       }
     }
-    float pa[4] = {ex2f(s0[0] - m_a), ex2f(s0[1] - m_a), ex2f(s1[0] - m_a), ex2f(s1[1] - m_a)};
-    float pb[4] = {ex2f(s0[2] - m_b), ex2f(s0[3] - m_b), ex2f(s1[2] - m_b), ex2f(s1[3] - m_b)};
-    l_a += (pa[0] + pa[1] + pa[2] + pa[3]);
-    l_b += (pb[0] + pb[1] + pb[2] + pb[3]);
-    // P as the A operand: (row g, tokens 2c, 2c+1), (row g+8, ...), (row g, 2c+8, 2c+9), (row g+8, ...)
-    uint32_t pf[4] = {pack_bf16(pa[0], pa[1]), pack_bf16(pb[0], pb[1]), pack_bf16(pa[2], pa[3]),
-                      pack_bf16(pb[2], pb[3])};
-    // ---- O += P V: d-tiles of 8, two per transposed ldmatrix
-#pragma unroll
-    for (int dt = 0; dt < D / 8; dt += 2) {
-      const int d_tile = dt + v_dt;  // the 8 dims (16 bytes) of this lane's matrix
-      uint32_t b[4];
-      ldmatrix_x4_trans(b, vt + (d_tile >> 3) * 2048 + v_tok * 128 + (((d_tile & 7) ^ (v_tok & 7)) << 4));
-      mma_bf16(o[dt], pf, b[0], b[1]);
-      mma_bf16(o[dt + 1], pf, b[2], b[3]);
-    }
-    __syncthreads();  // every warp is done with this stage
-    if (tid == 0 && j + kPrefixStages < nblk) issue(j + kPrefixStages);
+  };
+  __syncthreads();  // barriers initialised
+  int issued = 0;
+  if (tid == 0) {
+    for (; issued < min(nchunks, kPfxStages); ++issued) issue_chunk(issued);
   }
-  if (!ok) {
+
+  // ---- this thread's query row into the K-major swizzled Q tile: 16-byte
+  // piece j of row r at column block j / 8, position (j % 8) ^ (r % 8)
+  const int row = tile * kPfxRows + tid;
+  const bool row_ok = row < p.rows;
+  {
+    const int s = row_ok ? row / p.G : 0, h = row_ok ? row % p.G : 0;
+    const uint4* src = reinterpret_cast<const uint4*>(p.query + ((size_t)s * p.n_q + kv * p.G + h) * D);
+#pragma unroll
+    for (int j = 0; j < D / 8; ++j) {
+      const uint4 v = row_ok ? __ldg(src + j) : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t off = (j >> 3) * (kPfxRows * 128) + tid * 128 + (((j & 7) ^ (tid & 7)) << 4);
+      *reinterpret_cast<uint4*>(q_tile + off) = v;
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_s = tmem, t_o = tmem + kPfxOCol;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
+
+  constexpr uint32_t idesc_qk = umma_idesc_bf16(kPfxRows, kPfxTok, false, false);
+  constexpr uint32_t idesc_pv = umma_idesc_bf16(kPfxRows, D, false, true);
+  const uint32_t q_addr = smem_addr(q_tile), p_addr = smem_addr(p_tile);
+  auto issue_qk = [&](int c) {
+    const uint32_t k_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * (kPfxRows * 128) + (ks & 3) * 32, 16, 1024);
+      const uint64_t b = umma_desc_sw128(k_addr + (ks >> 2) * (kPfxTok * 128) + (ks & 3) * 32, 16, 1024);
+      umma_bf16(t_s, a, b, idesc_qk, ks > 0);
+    }
+    umma_commit(bar_s);
+  };
+  auto issue_pv = [&](int c) {
+    const uint32_t v_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage + Ly::kKV);
+#pragma unroll
+    for (int kt = 0; kt < kPfxTok / 16; ++kt) {
+      const uint64_t a = umma_desc_sw128(p_addr + kt * 32, 16, 1024);
+      const uint64_t b = umma_desc_sw128(v_addr + kt * 2048, kPfxTok * 128, 1024);
+      umma_bf16(t_o, a, b, idesc_pv, (c > 0 || kt > 0) ? 1u : 0u);
+    }
+    umma_commit(&empty[c % kPfxStages]);
+  };
+
+  bool ok = true;
+  int waited = 0;  // chunks whose K/V landing thread 0 has waited for
+  if (tid == 0 && nchunks > 0) {
+    ok = mbar_wait(&full[0], 0, p.wait_limit);
+    if (ok) {
+      waited = 1;
+      issue_qk(0);
+    }
+  }
+
+  float m = -INFINITY, l = 0.f;  // this row's running max (log2 units) and sum
+  int c = 0;
+  for (; c < nchunks; ++c) {
+    ok = mbar_wait(bar_s, c & 1, p.wait_limit) && ok;
+    tc_fence_after_sync();
+    // ---- this row's 64 scores (raw Q K^T); tokens past the split do not count
+    uint32_t sr[2][32];
+    tmem_ld32(t_s + lane_base, sr[0]);
+    tmem_ld32(t_s + lane_base + 32, sr[1]);
+    tmem_wait_ld();
+    const int valid = min(kPfxTok, (nblk - c * kPfxBlocks) * kBlockSize);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kPfxTok; ++j) {
+      if (j >= valid) sr[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+      mx = fmaxf(mx, __uint_as_float(sr[j >> 5][j & 31]));
+    }
+    mx *= p.scale_log2;
+    // lazy running max: moved only when a score passes it by more than 2^8
+    // (the previous P V is complete: its commit precedes this chunk's S)
+    const bool need = c > 0 && mx > m + 8.f;
+    if (__any_sync(0xffffffffu, need)) {
+      const float alpha = need ? ex2_approx(m - mx) : 1.f;
+#pragma unroll
+      for (int cb = 0; cb < D / 32; ++cb) {
+        uint32_t orow[32];
+        tmem_ld32(t_o + lane_base + cb * 32, orow);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * alpha);
+        tmem_st32(t_o + lane_base + cb * 32, orow);
+      }
+      tmem_wait_st();
+      if (need) {
+        l *= alpha;
+        m = mx;
+      }
+    }
+    if (c == 0) m = mx;
+    // ---- probabilities in bf16 into the P tile (row tid, K-major, 128-byte swizzle)
+    float lsum = 0.f;
+#pragma unroll
+    for (int j8 = 0; j8 < kPfxTok / 8; ++j8) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = j8 * 8 + 2 * e;
+        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[j >> 5][j & 31]), p.scale_log2, -m));
+        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31]), p.scale_log2, -m));
+        lsum += p0 + p1;
+        w[e] = pack_bf16(p0, p1);
+      }
+      *reinterpret_cast<uint4*>(p_tile + tid * 128 + ((j8 ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    l += lsum;
+    fence_proxy_async_smem();
+    tc_fence_before_sync();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
     if (tid == 0) {
-      flag_error(p.err, DEVERR_TIMEOUT);
-      // blocks j .. j + stages - 1 were issued and not consumed: let them land
-      // before the CTA exits (each wait bounded)
-      for (int i = j; i < min(nblk, j + kPrefixStages); ++i)
-        mbar_wait(&full[i % kPrefixStages], (i / kPrefixStages) & 1);
+      tc_fence_after_sync();
+      issue_pv(c);
+      if (c + 1 < nchunks) {
+        ok = mbar_wait(&full[(c + 1) % kPfxStages], ((c + 1) / kPfxStages) & 1, p.wait_limit);
+        if (ok) {
+          waited = c + 2;
+          issue_qk(c + 1);
+        }
+      }
+      if (ok && issued < nchunks) {
+        // the stage of chunk c is free once its P V completed
+        ok = mbar_wait(&empty[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
+        if (ok) issue_chunk(issued++);
+      }
     }
-    return;
   }
 
-  // ---- normalise and store this split's partial state
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-  const int ra = row0 + g, rb = row0 + g + 8;
-  const float ia = l_a > 0.f ? 1.f / l_a : 0.f, ib = l_b > 0.f ? 1.f / l_b : 0.f;
-  const size_t base = (size_t)kv * p.rows;
+  // ---- every MMA done (also on the error path: nothing in flight at exit)
+  if (tid == 0) {
+    umma_commit(bar_done);
+    if (!mbar_wait(bar_done, 0)) ok = false;
+    // chunks issued but never waited for (error path): let them land
+    for (int k = waited; k < issued; ++k) mbar_wait(&full[k % kPfxStages], (k / kPfxStages) & 1);
+  }
+  ok = __syncthreads_and(ok && c == nchunks);
+  tc_fence_after_sync();
+  if (!ok) {
+    if (tid == 0) flag_error(p.err, DEVERR_TIMEOUT);
+  } else {
+    // ---- normalised partial o and base-2 lse of this row and split (every
+    // lane takes part in the warp-wide loads; rows past the batch store nothing)
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float4* dst = reinterpret_cast<float4*>(p.part_o + (((size_t)kv * p.rows + (row_ok ? row : 0)) * p.splits + split) * D);
 #pragma unroll
-  for (int dt = 0; dt < D / 8; ++dt) {
-    const int d = dt * 8 + 2 * c;
-    if (ra < p.rows)
-      *reinterpret_cast<float2*>(p.part_o + ((base + ra) * p.splits + split) * D + d) =
-          make_float2(o[dt][0] * ia, o[dt][1] * ia);
-    if (rb < p.rows)
-      *reinterpret_cast<float2*>(p.part_o + ((base + rb) * p.splits + split) * D + d) =
-          make_float2(o[dt][2] * ib, o[dt][3] * ib);
+    for (int cb = 0; cb < D / 32; ++cb) {
+      uint32_t orow[32];
+      tmem_ld32(t_o + lane_base + cb * 32, orow);
+      tmem_wait_ld();
+      if (row_ok) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          dst[cb * 8 + j] = make_float4(__uint_as_float(orow[4 * j]) * inv, __uint_as_float(orow[4 * j + 1]) * inv,
+                                        __uint_as_float(orow[4 * j + 2]) * inv, __uint_as_float(orow[4 * j + 3]) * inv);
+      }
+    }
+    if (row_ok) p.part_lse[((size_t)kv * p.rows + row) * p.splits + split] = nchunks > 0 ? m + log2f(l) : -INFINITY;
   }
-  if (c == 0) {
-    if (ra < p.rows) p.part_lse[(base + ra) * p.splits + split] = nblk > 0 ? m_a + log2f(l_a) : -INFINITY;
-    if (rb < p.rows) p.part_lse[(base + rb) * p.splits + split] = nblk > 0 ? m_b + log2f(l_b) : -INFINITY;
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kPfxTmemCols);
   }
 }
 
-// Splits of the prefix so that about four CTAs run on every SM (the pass is
-// latency-bound: more resident warps hide more of each block's MMA and
-// softmax chain), each split at least 4 blocks long.
-static void prefix_grid(int rows, int n_kv, int prefix_blocks, int* splits, int* per_split) {
-  const int tiles = (rows + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
-  const int want = std::max(1, (4 * std::max(1, device_sm_count())) / std::max(1, tiles * n_kv));
-  int sp = std::max(1, std::min(want, prefix_blocks / 4));
-  sp = std::min(sp, kMaxPrefixSplits);
-  *per_split = (prefix_blocks + sp - 1) / sp;
-  *splits = (prefix_blocks + *per_split - 1) / *per_split;
-}
-
-// The splits' states combined per (KV head, query row): one CTA of 256 threads
-// per 8 rows, a thread per (row, 4 dims), the splits' loads independent.
-struct CombineParams {
-  const float* part_o;
-  const float* part_lse;
-  float* o;    // [n_kv * rows][D]
-  float* lse;  // [n_kv * rows]
-  int total_rows, splits;
-};
-
-template <int D>
-__global__ void __launch_bounds__(256) prefix_combine_kernel(const CombineParams p) {
-  grid_launch_dependents();
-  grid_wait_prerequisites();
-  constexpr int V = D / 4;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const int r = idx / V, v = idx - r * V;
-  if (r >= p.total_rows) return;
-  const float* lse = p.part_lse + (size_t)r * p.splits;
-  float M = -INFINITY;
-#pragma unroll 8
-  for (int k = 0; k < p.splits; ++k) M = fmaxf(M, __ldcg(lse + k));
-  float wsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-  for (int k = 0; k < p.splits; ++k) {
-    const float w = ex2f(__ldcg(lse + k) - M);
-    const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + ((size_t)r * p.splits + k) * D) + v);
-    wsum += w;
-    acc.x += w * o.x;
-    acc.y += w * o.y;
-    acc.z += w * o.z;
-    acc.w += w * o.w;
-  }
-  const float inv = 1.f / wsum;
-  reinterpret_cast<float4*>(p.o + (size_t)r * D)[v] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (v == 0) p.lse[r] = M + log2f(wsum);
+// Splits of the prefix: about one CTA per SM over the (row tile, KV head)
+// pairs, each split a whole number of 64-token chunks.
+static void prefix_grid(int rows, int n_kv, int prefix_blocks, int want_splits, int* splits, int* chunks_per_split) {
+  const int tiles = (rows + kPfxRows - 1) / kPfxRows;
+  const int chunks = (prefix_blocks + kPfxBlocks - 1) / kPfxBlocks;
+  int sp = want_splits > 0 ? want_splits : std::max(1, std::max(1, device_sm_count()) / std::max(1, tiles * n_kv));
+  sp = std::max(1, std::min({sp, chunks, kMaxPrefixSplits}));
+  *chunks_per_split = (chunks + sp - 1) / sp;
+  *splits = (chunks + *chunks_per_split - 1) / *chunks_per_split;
 }
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks) {
+size_t prefix_workspace_bytes(int num_seqs, int n_q, int n_kv, int head_dim, int prefix_blocks, int want_splits) {
   const int rows = num_seqs * (n_q / n_kv);
-  int splits = 1, per = 1;
-  prefix_grid(rows, n_kv, prefix_blocks, &splits, &per);
+  int splits = 1, cps = 1;
+  prefix_grid(rows, n_kv, prefix_blocks, want_splits, &splits, &cps);
   const size_t part_o = (size_t)n_kv * rows * splits * head_dim * 4;
   const size_t part_l = (size_t)n_kv * rows * splits * 4;
-  const size_t o = (size_t)n_kv * rows * head_dim * 4;
-  const size_t l = (size_t)n_kv * rows * 4;
-  return align256(part_o) + align256(part_l) + align256(o) + align256(l);
+  const size_t unit_o = (size_t)num_seqs * n_q * head_dim * 4;
+  const size_t unit_l = (size_t)num_seqs * n_q * 4;
+  return align256(part_o) + align256(part_l) + align256(unit_o) + align256(unit_l);
 }
 
-pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const void* query,
-                         const int32_t* block_tables, int64_t num_blocks, int prefix_blocks, float sm_scale,
-                         void* prefix_ws, int32_t* device_error, PrefixState* state, cudaStream_t stream) {
+// One instantiation per head_dim, each granted its own shared-memory size once.
+template <int D>
+static pkv_status run_prefix_kernel(dim3 grid, const CUtensorMap& km, const CUtensorMap& vm, const PrefixParams& p,
+                                    cudaStream_t stream) {
+  constexpr uint32_t smem = PfxLayout<D>::kSmem;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(prefix_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix)");
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kPfxThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, prefix_tc_kernel<D>, km, vm, p);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "prefix_tc_kernel launch");
+  return PKV_OK;
+}
+
+pkv_status launch_prefix(const DecodeShape& s, const CUtensorMap& km, const CUtensorMap& vm, const TcArgs& a,
+                         long long wait_limit, PrefixPieces* pieces, cudaStream_t stream) {
   PrefixParams p;
-  p.query = static_cast<const __nv_bfloat16*>(query);
-  p.block_tables = block_tables;
-  p.err = device_error;
+  p.query = static_cast<const __nv_bfloat16*>(a.query);
+  p.block_tables = a.block_tables;
+  p.context_lens = a.context_lens;
+  p.err = a.device_error;
+  p.num_seqs = s.num_seqs;
   p.n_q = s.n_q;
   p.n_kv = s.n_kv;
   p.G = s.n_q / s.n_kv;
   p.rows = s.num_seqs * p.G;
-  p.prefix_blocks = prefix_blocks;
-  p.num_blocks = num_blocks;
-  p.scale_log2 = (float)((double)sm_scale * 1.4426950408889634);
-  prefix_grid(p.rows, s.n_kv, prefix_blocks, &p.splits, &p.per_split);
-  uint8_t* ws = static_cast<uint8_t*>(prefix_ws);
+  p.prefix_blocks = a.skip_blocks;
+  p.max_blocks_per_seq = a.max_blocks_per_seq;
+  p.num_blocks = a.num_blocks;
+  p.wait_limit = wait_limit;
+  p.scale_log2 = (float)((double)a.sm_scale * 1.4426950408889634);
+  prefix_grid(p.rows, s.n_kv, a.skip_blocks, a.prefix_splits, &p.splits, &p.chunks_per_split);
+  uint8_t* ws = static_cast<uint8_t*>(a.prefix_ws);
   const size_t part_o = align256((size_t)s.n_kv * p.rows * p.splits * s.head_dim * 4);
   const size_t part_l = align256((size_t)s.n_kv * p.rows * p.splits * 4);
-  const size_t comb_o = align256((size_t)s.n_kv * p.rows * s.head_dim * 4);
+  const size_t unit_o = align256((size_t)s.num_seqs * s.n_q * s.head_dim * 4);
   p.part_o = reinterpret_cast<float*>(ws);
   p.part_lse = reinterpret_cast<float*>(ws + part_o);
-  CombineParams cp;
-  cp.part_o = p.part_o;
-  cp.part_lse = p.part_lse;
-  cp.o = reinterpret_cast<float*>(ws + part_o + part_l);
-  cp.lse = reinterpret_cast<float*>(ws + part_o + part_l + comb_o);
-  cp.total_rows = s.n_kv * p.rows;
-  cp.splits = p.splits;
-  state->o = cp.o;
-  state->lse = cp.lse;
-  state->splits = 1;
-  state->rows = p.rows;
+  pieces->o = p.part_o;
+  pieces->lse = p.part_lse;
+  pieces->splits = p.splits;
+  pieces->rows = p.rows;
+  pieces->unit_o = reinterpret_cast<float*>(ws + part_o + part_l);
+  pieces->unit_lse = reinterpret_cast<float*>(ws + part_o + part_l + unit_o);
 
-  const int tiles = (p.rows + kPrefixWarps * 16 - 1) / (kPrefixWarps * 16);
-  const int tile_bytes = s.head_dim * 2 * 16;
-  const size_t smem = (size_t)kPrefixStages * 2 * tile_bytes + 1024;
-  auto run = [&](auto kern) -> pkv_status {
-    static int configured = 0;
-    if ((int)smem > configured) {
-      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix)");
-      configured = (int)smem;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(tiles, s.n_kv, p.splits);
-    cfg.blockDim = dim3(kPrefixWarps * 32);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, km, vm, p);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "prefix_attn_kernel launch");
-    return PKV_OK;
-  };
-  auto combine = [&](auto kern) -> pkv_status {
-    const long long threads = (long long)cp.total_rows * (s.head_dim / 4);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
-    cfg.blockDim = dim3(256);
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, cp);
-    if (e == cudaSuccess) e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "prefix_combine_kernel launch");
-    return PKV_OK;
-  };
-  pkv_status st = PKV_ERR_UNSUPPORTED;
-  if (s.head_dim == 128) {
-    st = run(prefix_attn_kernel<128>);
-    if (st == PKV_OK) st = combine(prefix_combine_kernel<128>);
-  } else if (s.head_dim == 64) {
-    st = run(prefix_attn_kernel<64>);
-    if (st == PKV_OK) st = combine(prefix_combine_kernel<64>);
-  }
-  return st;
+  const int tiles = (p.rows + kPfxRows - 1) / kPfxRows;
+  const dim3 grid(tiles, s.n_kv, p.splits);
+  if (s.head_dim == 128) return run_prefix_kernel<128>(grid, km, vm, p, stream);
+  if (s.head_dim == 64) return run_prefix_kernel<64>(grid, km, vm, p, stream);
+  return PKV_ERR_UNSUPPORTED;
 }
 
 }  // namespace pkv

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libpkv.so")
 
 PKV_F32, PKV_BF16, PKV_INT8, PKV_FP8_E4M3, PKV_FP8_E5M2, PKV_INT4, PKV_KIVI2 = 0, 1, 2, 3, 4, 5, 6
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or dtype", 3: "workspace missing or too small", 4: "CUDA error"}
-DEVERR_SLOT_RANGE, DEVERR_BLOCK_RANGE, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT = 0x1, 0x2, 0x4, 0x8
+DEVERR_SLOT_RANGE, DEVERR_BLOCK_RANGE, DEVERR_CONTEXT_LEN, DEVERR_TIMEOUT, DEVERR_PREFIX = 0x1, 0x2, 0x4, 0x8, 0x10
 
 _CACHE_DTYPES = {
     "f32": PKV_F32,
@@ -42,11 +42,15 @@ class PkvError(RuntimeError):
 
 
 class DecodeTuning(ctypes.Structure):
+    """pkv_decode_tuning: launch overrides (0 = automatic); see include/pkv.h."""
+
     _fields_ = [("num_ctas", ctypes.c_int), ("stages", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
-                ("flags", ctypes.c_int)]
+                ("flags", ctypes.c_int), ("prefix_splits", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("wait_limit_cycles", ctypes.c_int64)]
 
 
 TUNE_OVERLAP_PROLOGUE = 0x1
+TUNE_PREFIX_SERIAL = 0x2
 
 
 def _load() -> ctypes.CDLL:
@@ -93,9 +97,14 @@ def _load() -> ctypes.CDLL:
     lib.pkv_paged_decode_step_window.restype = i32
     lib.pkv_shared_prefix_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.pkv_shared_prefix_workspace_size.restype = sz
+    lib.pkv_shared_prefix_workspace_size_ex.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(DecodeTuning)]
+    lib.pkv_shared_prefix_workspace_size_ex.restype = sz
     lib.pkv_paged_attention_decode_shared_prefix.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32, i32,
                                                              i32, i32, i64, f32, i32, i32, i32, vp, vp, sz, vp, vp]
     lib.pkv_paged_attention_decode_shared_prefix.restype = i32
+    lib.pkv_paged_attention_decode_shared_prefix_ex.argtypes = (
+        lib.pkv_paged_attention_decode_shared_prefix.argtypes[:-1] + [ctypes.POINTER(DecodeTuning), vp])
+    lib.pkv_paged_attention_decode_shared_prefix_ex.restype = i32
     lib.pkv_kivi_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     lib.pkv_kivi_workspace_size.restype = sz
     lib.pkv_kivi_quantize_blocks.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp]
@@ -131,6 +140,11 @@ def _ptr(t) -> int | None:
 
 def _stream(device=None) -> int:
     return torch.cuda.current_stream(device).cuda_stream
+
+
+def _default_scale(sm_scale, head_dim: int) -> float:
+    """The softmax scale to pass: the caller's, else 1 / sqrt(head_dim)."""
+    return 1.0 / math.sqrt(head_dim) if sm_scale is None else sm_scale
 
 
 def act_code(t: torch.Tensor) -> int:
@@ -218,8 +232,7 @@ def paged_attention_decode(
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     ccode = cache_code(key_cache, cache_dtype)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, tuning)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
@@ -244,8 +257,7 @@ def paged_decode_step(out, query, key, value, key_cache, value_cache, block_tabl
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     ccode = cache_code(key_cache, cache_dtype)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, tuning)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
@@ -270,8 +282,7 @@ def paged_attention_decode_static(out, query, key_cache, value_cache, block_tabl
     """pkv_paged_attention_decode_static: decode with the library's own scratch (no workspace argument)."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     st = lib.pkv_paged_attention_decode_static(
         _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
@@ -323,8 +334,7 @@ def paged_attention_decode_window(out, query, key_cache, value_cache, block_tabl
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     ccode = cache_code(key_cache, cache_dtype)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
@@ -374,8 +384,7 @@ def paged_attention_decode_pages(out, query, key_cache, value_cache, block_table
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     ccode = cache_code(key_cache, cache_dtype)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         t1 = None if tuning is None else DecodeTuning(tuning.num_ctas, tuning.stages, 1, tuning.flags)
         nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode, t1)
@@ -395,8 +404,12 @@ def paged_attention_decode_pages(out, query, key_cache, value_cache, block_table
     return out
 
 
-def shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks) -> int:
-    n = lib.pkv_shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks)
+def shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks, tuning=None) -> int:
+    if tuning is None:
+        n = lib.pkv_shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks)
+    else:
+        n = lib.pkv_shared_prefix_workspace_size_ex(num_seqs, n_q, n_kv, head_dim, block_size, prefix_blocks,
+                                                    ctypes.byref(tuning))
     if n == ctypes.c_size_t(-1).value:
         raise PkvError(2, "pkv_shared_prefix_workspace_size")
     return int(n)
@@ -405,23 +418,27 @@ def shared_prefix_workspace_size(num_seqs, n_q, n_kv, head_dim, block_size, pref
 def paged_attention_decode_shared_prefix(out, query, key_cache, value_cache, block_tables, context_lens,
                                          max_context_len: int, prefix_blocks: int, key=None, value=None,
                                          sm_scale: float | None = None, lse_out=None, workspace=None,
-                                         device_error=None):
+                                         device_error=None, tuning: DecodeTuning | None = None):
     """Decode with the first ``prefix_blocks`` blocks shared by every sequence: one dense pass over the
-    prefix for all queries, then each sequence's own blocks; ``key``/``value`` append token L-1 first."""
+    prefix for all queries beside the decode of each sequence's own blocks, then their merge;
+    ``key``/``value`` append token L-1 first."""
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
-        nbytes = shared_prefix_workspace_size(S, n_q, n_kv, d, block_size, prefix_blocks)
+        nbytes = shared_prefix_workspace_size(S, n_q, n_kv, d, block_size, prefix_blocks, tuning)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    st = lib.pkv_paged_attention_decode_shared_prefix(
+    args = [
         _ptr(out), _ptr(query), _ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
         block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, n_q, n_kv, d, block_size, num_blocks,
         float(sm_scale), int(prefix_blocks), act_code(query), cache_code(key_cache), _ptr(lse_out), _ptr(workspace),
-        ws_bytes, _ptr(device_error), _stream(query.device),
-    )
+        ws_bytes, _ptr(device_error),
+    ]
+    if tuning is None:
+        st = lib.pkv_paged_attention_decode_shared_prefix(*args, _stream(query.device))
+    else:
+        st = lib.pkv_paged_attention_decode_shared_prefix_ex(*args, ctypes.byref(tuning), _stream(query.device))
     _check(st, "pkv_paged_attention_decode_shared_prefix")
     return out
 
@@ -434,8 +451,7 @@ def paged_decode_step_window(out, query, key, value, key_cache, value_cache, blo
     S, n_q, d = query.shape
     num_blocks, block_size, n_kv = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     ccode = cache_code(key_cache, cache_dtype)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         nbytes = paged_attention_workspace_size(S, n_q, n_kv, d, block_size, ccode)
         workspace = workspace_for(nbytes, query.device) if nbytes else None
@@ -498,8 +514,7 @@ def kivi_decode(out, query, residual_k, residual_v, key_cache, value_cache, k_sc
     num_blocks = key_cache.shape[0]
     _check_kivi_tensors(S, n_kv, d, num_blocks, block_size, residual_k, residual_v, key_cache, value_cache, k_scale,
                         v_scale)
-    if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(d)
+    sm_scale = _default_scale(sm_scale, d)
     if workspace is None:
         nbytes = kivi_workspace_size(S, n_q, n_kv, d, block_size)
         workspace = workspace_for(nbytes, query.device) if nbytes else None

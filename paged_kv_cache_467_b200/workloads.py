@@ -395,6 +395,19 @@ def sliding_window(seed: int = 1) -> DecodeWorkload:
     return w
 
 
+def first_sequences(w: DecodeWorkload, n: int) -> DecodeWorkload:
+    """The same workload cut to its first n sequences (a smaller case of the
+    same shapes, lengths and pool recipe, for profiling)."""
+    if n >= w.num_seqs:
+        return w
+    out = make_workload(
+        f"{w.name}_first{n}", seed=w.seed, context_lens=w.context_lens[:n], n_q=w.n_q, n_kv=w.n_kv,
+        head_dim=w.head_dim, block_size=w.block_size, act_dtype=w.act_dtype, cache_dtype=w.cache_dtype,
+        sm_scale=w.sm_scale, shared_prefix_tokens=w.shared_prefix_tokens,
+        outlier_fraction=0.01 if w.k_outlier_channels is not None else 0.0, window=w.window, sinks=w.sinks)
+    return out
+
+
 CONFIGS = {
     "tiny": tiny,
     "llama3_8b": llama3_8b,

@@ -1,6 +1,8 @@
-"""GPU parity of the shared-prefix decode (a dense pass over the blocks every
-sequence shares, then each sequence's own blocks) against the oracle's plain
-decode ("Chapter 18 - KV-Cache Optimization Strategies", Prefix Caching)."""
+"""GPU parity of the shared-prefix decode (a dense tensor-core pass over the
+blocks every sequence shares, beside the paged decode of each sequence's own
+blocks, then the merge of both) against the oracle's plain decode ("Chapter 18
+- KV-Cache Optimization Strategies", Prefix Caching), and the device checks of
+the prefix contract."""
 import numpy as np
 import pytest
 import torch
@@ -26,17 +28,18 @@ def _ops():
     return ops
 
 
-def run_shared(w, st, append=False):
+def run_shared(w, st, append=False, tuning=None, prefix_blocks=None):
     ops = _ops()
     out = torch.full((w.num_seqs, w.n_q, w.head_dim), float("nan"), dtype=torch.bfloat16, device="cuda")
     lse = torch.full((w.num_seqs, w.n_q), float("nan"), dtype=torch.float32, device="cuda")
     k = v = None
     if append:
         k, v = new_rows(w)
+    pb = w.shared_prefix_tokens // 16 if prefix_blocks is None else prefix_blocks
     ops.paged_attention_decode_shared_prefix(out, st.query, st.key_cache, st.value_cache, st.block_tables,
-                                             st.context_lens, w.max_context_len, w.shared_prefix_tokens // 16,
-                                             key=k, value=v, sm_scale=w.sm_scale, lse_out=lse,
-                                             device_error=st.device_error)
+                                             st.context_lens, w.max_context_len, pb, key=k, value=v,
+                                             sm_scale=w.sm_scale, lse_out=lse, device_error=st.device_error,
+                                             tuning=tuning)
     torch.cuda.synchronize()
     return out.float().cpu().numpy().astype(np.float64), lse.cpu().numpy().astype(np.float64)
 
@@ -96,3 +99,60 @@ def test_prefix_config_sampled():
     check(w, st, out, lse, seqs=range(0, 128, 11))
     again, lse2 = run_shared(w, st)
     assert np.array_equal(out, again) and np.array_equal(lse, lse2)  # deterministic
+
+
+def test_prefix_pass_beside_and_after_the_decode_agree():
+    """The prefix pass running beside the decode, or before it, and any number
+    of splits along the prefix: the same pieces, merged in the same order."""
+    ops = _ops()
+    w = workloads.make_workload("p", seed=83, context_lens=[1100 + 61 * i for i in range(40)], n_q=32, n_kv=8,
+                                head_dim=128, extra_blocks=3, shared_prefix_tokens=1024)
+    st = fill_gpu(w)
+    results = {}
+    for splits in (0, 1, 3, 16):
+        for serial in (False, True):
+            tun = ops.DecodeTuning(0, 0, 0, ops.TUNE_PREFIX_SERIAL if serial else 0, splits)
+            out, lse = run_shared(w, st, tuning=tun)
+            assert int(st.device_error.item()) == 0
+            check(w, st, out, lse, seqs=range(0, 40, 7))
+            results[(splits, serial)] = (out, lse)
+        # the order of the two passes does not change a bit
+        assert np.array_equal(results[(splits, False)][0], results[(splits, True)][0])
+        assert np.array_equal(results[(splits, False)][1], results[(splits, True)][1])
+
+
+def test_sequence_shorter_than_prefix_is_flagged():
+    """A context that does not reach past the shared prefix sets the context-length
+    bit; the other sequences are unaffected."""
+    ops = _ops()
+    w = workloads.make_workload("p", seed=84, context_lens=[200, 150, 90, 300], n_q=32, n_kv=8, head_dim=128,
+                                extra_blocks=3, shared_prefix_tokens=64)
+    st = fill_gpu(w)
+    lens = st.context_lens.clone()
+    lens[2] = 50  # inside the 64-token prefix
+    st.context_lens = lens
+    out, lse = run_shared(w, st)
+    assert int(st.device_error.item()) & ops.DEVERR_CONTEXT_LEN
+    assert not int(st.device_error.item()) & ops.DEVERR_PREFIX
+    check(w, st, out, lse, seqs=[0, 1, 3])
+
+
+def test_table_that_leaves_the_prefix_is_flagged():
+    """A block table whose first entries are not row 0's sets PKV_DEVERR_PREFIX.
+    Here the diverging block is a byte copy of the shared one, so every output
+    still matches the oracle."""
+    ops = _ops()
+    w = workloads.make_workload("p", seed=85, context_lens=[200, 150, 90, 300], n_q=32, n_kv=8, head_dim=128,
+                                extra_blocks=3, shared_prefix_tokens=64)
+    st = fill_gpu(w)
+    used = set(int(b) for b in w.block_tables.reshape(-1) if b >= 0)
+    spare = next(b for b in range(w.num_blocks) if b not in used)
+    src = int(w.block_tables[2, 1])
+    pairs = torch.tensor([[src, spare]], dtype=torch.int64, device="cuda")
+    ops.copy_blocks(st.key_cache, st.value_cache, pairs)
+    tables = st.block_tables.clone()
+    tables[2, 1] = spare
+    st.block_tables = tables
+    out, lse = run_shared(w, st)
+    assert int(st.device_error.item()) == ops.DEVERR_PREFIX
+    check(w, st, out, lse)

@@ -3,16 +3,16 @@
 Such a caller (for example a plug-in whose host runtime owns all device memory,
 or a loop that must not call cudaMalloc) gets its scratch from a fixed array
 inside libpkv.  These tests call that entry point through the C ABI and check
-it against pkv_paged_attention_decode, which takes a caller-owned workspace, on
-two calls in a row: the second call finds the array as the first one left it.
-The file is named to be collected last.
+it against the oracle and against pkv_paged_attention_decode, which takes a
+caller-owned workspace, on two calls in a row: the second call finds the array
+as the first one left it.  The file is named to be collected last.
 """
 import numpy as np
 import pytest
 import torch
 
 from paged_kv_cache_467_b200 import workloads
-from gpu_harness import TOL, fill_gpu, run_decode
+from gpu_harness import TOL, assert_close, fill_gpu, oracle_sequence, run_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -57,6 +57,10 @@ def test_static_scratch_matches_workspace_entry_point_two_calls_in_a_row():
         _compare(got, want, w.cache_dtype)
         np.testing.assert_allclose(got_lse, want_lse, rtol=0, atol=2e-3)
         assert int(st.device_error.item()) == 0
+        for s in range(w.num_seqs):  # and against the oracle directly
+            o, l, _ = oracle_sequence(w, s)
+            assert_close(got[s], o, w.cache_dtype, f"{w.name} seq {s}")
+            np.testing.assert_allclose(got_lse[s], l, rtol=0, atol=2e-3)
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
