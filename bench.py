@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--prefix-serial", action="store_true",
                     help="shared-prefix config: run the decode of each sequence's own blocks after the prefix pass "
                          "instead of beside it")
+    ap.add_argument("--plain-decode", action="store_true",
+                    help="shared-prefix configuration: run the plain decode step, every sequence reading the "
+                         "shared blocks itself (through L2), instead of the shared-prefix pass")
     ap.add_argument("--seqs", type=int, default=0,
                     help="run the configuration's first N sequences only (a smaller case for profiling)")
     ap.add_argument("--quest-budget", type=int, default=4096,
@@ -101,27 +104,38 @@ def strip_c_comments(text: str) -> str:
     return "\n".join(line for line in lines if line)
 
 
-def kernel_source_hash() -> str:
-    """Hash of the library's sources with comments removed: a profile taken on
-    these sources stays valid across comment edits, not across code edits."""
+# Sources each kernel family is built from: a profile of a kernel stays valid
+# while these files keep their code (comments aside).
+KERNEL_SOURCES = {
+    "decode": ("decode_tc.cu", "pkv_device.cuh", "cache_row.cuh", "internal.h"),
+    "prefix": ("prefix.cu", "tcgen05.cuh", "pkv_device.cuh", "internal.h"),
+    "kivi": ("kivi.cu", "decode_tc.cu", "pkv_device.cuh", "cache_row.cuh", "internal.h"),
+}
+
+
+def kernel_source_hash(files=None) -> str:
+    """Hash of the library's sources (all of them, or the named files of csrc/)
+    with comments removed: a profile taken on these sources stays valid across
+    comment edits, not across code edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "paged_kv_cache_467_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             h.update(name.encode() + strip_c_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(config: str):
-    """DRAM bytes per decode launch from the committed ncu summary, or None when
-    the summary is missing or was taken on different kernel sources."""
+def profiled_traffic(config: str, family: str = "decode"):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the summary is missing or was taken on different
+    sources of that kernel."""
     path = os.path.join(ROOT, "profiles", f"decode_{config}_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(KERNEL_SOURCES[family]):
         return None
     return float(m_bytes.group(1))
 
@@ -474,7 +488,7 @@ def run_b200(args, rank, world, local):
     kv_bytes = accounting.decode_kv_bytes(w)
 
 
-    prefix_blocks = w.shared_prefix_tokens // bs
+    prefix_blocks = 0 if args.plain_decode else w.shared_prefix_tokens // bs
     prefix_tuning = None
     if prefix_blocks:
         # the shared prefix is attended once for all sequences, beside the decode of each sequence's own blocks
@@ -606,7 +620,7 @@ def run_b200(args, rank, world, local):
         peak, peak_kind = measured_peaks()
         value = whole_job_gbs(kv_bytes, world, ms)
         achieved = kv_bytes / (att_ms * 1e-3) / 1e9
-        traffic = profiled_traffic(args.config)
+        traffic = profiled_traffic(args.config, "kivi" if kivi else "decode")
         line = {
             "metric": METRIC,
             "value": value,

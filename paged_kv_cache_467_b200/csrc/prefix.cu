@@ -8,20 +8,25 @@
 // it once per KV head for all rows together, so each K/V tile of the prefix is
 // read by ceil(R / 128) CTAs instead of by every sequence.
 //
-// CTA = one KV head, 128 query rows (the MMA's M), one split of the prefix.
-//  * Q tile [128 x D] bf16 in shared memory, K-major with the 128-byte swizzle.
-//  * K and V of 64 tokens (four 16-token blocks) per chunk come by TMA through
-//    a two-stage ring, in the pool's own row layout: K is the K-major B
-//    operand of S = Q K^T, V the MN-major B operand of O += P V.
-//  * S [128 x 64] and O [128 x D] accumulate in tensor memory (fp32).  One
-//    thread issues the tcgen05.mma instructions and commits them to mbarriers.
-//  * Each of the 128 threads owns one query row (one TMEM lane): it reads its
-//    64 scores with tcgen05.ld, keeps the row's running max and sum (online
-//    softmax in base 2, the max moved only past 2^8 of slack, rescaling its O
-//    row in tensor memory then), and writes its bf16 probabilities into the P
-//    tile, the K-major A operand of P V.
-//  * The split's result per row, normalised o and base-2 lse, is one piece of
-//    the final merge, next to the pieces of the sequence's own blocks.
+// CTA = one KV head, 128 query rows (the MMA's M), one split of the prefix,
+// six warps with fixed roles:
+//  * a TMA warp streams K and V of 64 tokens (four 16-token blocks) per chunk
+//    through a three-stage ring, in the pool's own row layout (K is the K-major
+//    B operand of S = Q K^T, V the MN-major B operand of O += P V); its lanes
+//    read the split's block-table entries once, up front, and it starts while
+//    the softmax warps still load the queries;
+//  * an MMA warp issues the tcgen05.mma instructions from one thread: S of a
+//    chunk into one of two tensor-memory buffers while the softmax warps still
+//    read the other, and P V of the chunk before into the O accumulator
+//    [128 x D] (fp32, tensor memory), each committed to mbarriers;
+//  * four softmax warps own one query row (one TMEM lane) per thread: a row's
+//    64 scores come in by tcgen05.ld, its running max and sum are kept in
+//    base 2 (the max moved only past 2^8 of slack, its O row then rescaled in
+//    tensor memory), and its bf16 probabilities go to one of two P tiles
+//    (the K-major A operand of P V).
+//  * Q [128 x D] bf16 sits in shared memory, K-major with the 128-byte swizzle.
+// The split's result per row, normalised o and base-2 lse, is one piece of the
+// final merge, next to the pieces of the sequence's own blocks.
 // The CTAs that hold KV head 0 also check the prefix contract: every
 // sequence's first prefix_blocks table entries equal row 0's, and every
 // context is longer than the prefix.
@@ -40,9 +45,11 @@ namespace pkv {
 constexpr int kPfxRows = 128;   // query rows per CTA (MMA M, TMEM lanes)
 constexpr int kPfxTok = 64;     // tokens per chunk (N of Q K^T, K of P V)
 constexpr int kPfxBlocks = kPfxTok / kBlockSize;
-constexpr int kPfxStages = 2;
-constexpr int kPfxThreads = 128;
-constexpr uint32_t kPfxTmemCols = 256;  // S at columns [0, 64), O at [128, 128 + D)
+constexpr int kPfxStages = 3;
+constexpr int kPfxSoftmaxThreads = 128;  // warps 0-3: one query row each
+constexpr int kPfxMmaWarp = 4, kPfxTmaWarp = 5;
+constexpr int kPfxThreads = 192;
+constexpr uint32_t kPfxTmemCols = 256;  // S buffers at columns [0, 64) and [64, 128), O at [128, 128 + D)
 constexpr uint32_t kPfxOCol = 128;
 
 template <int D>
@@ -51,11 +58,11 @@ struct PfxLayout {
   static constexpr uint32_t kQ = kPfxRows * D * 2;        // [dblk][128 rows][128 B]
   static constexpr uint32_t kKV = kPfxTok * D * 2;        // [dblk][64 tokens][128 B]
   static constexpr uint32_t kStage = 2 * kKV;             // K then V
-  static constexpr uint32_t kP = kPfxRows * kPfxTok * 2;  // [128 rows][128 B]
+  static constexpr uint32_t kP = kPfxRows * kPfxTok * 2;  // one P tile [128 rows][128 B]
   static constexpr uint32_t kOffStage = kQ;
-  static constexpr uint32_t kOffP = kOffStage + kPfxStages * kStage;
-  static constexpr uint32_t kOffBar = kOffP + kP;
-  static constexpr uint32_t kBytes = kOffBar + 128;
+  static constexpr uint32_t kOffP = kOffStage + kPfxStages * kStage;  // two P tiles
+  static constexpr uint32_t kOffBar = kOffP + 2 * kP;
+  static constexpr uint32_t kBytes = kOffBar + 256;
   static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
 };
 
@@ -104,14 +111,18 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_tile = smem;
-  uint8_t* p_tile = smem + Ly::kOffP;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kOffBar);  // [kPfxStages] K/V chunk landed
-  uint64_t* empty = full + kPfxStages;                                // [kPfxStages] P V of the chunk done
-  uint64_t* bar_s = empty + kPfxStages;                               // S of the next chunk ready
-  uint64_t* bar_done = bar_s + 1;                                     // every MMA of the CTA done
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kOffBar);  // [stages] K/V chunk landed
+  uint64_t* empty = full + kPfxStages;                                // [stages] P V of the chunk done
+  uint64_t* s_full = empty + kPfxStages;                              // [2] S buffer written
+  uint64_t* s_free = s_full + 2;                                      // [2] S buffer read out
+  uint64_t* p_full = s_free + 2;                                      // [2] P tile written (O rescaled)
+  uint64_t* p_free = p_full + 2;                                      // [2] P V done with the P tile
+  uint64_t* o_done = p_free + 2;                                      // one phase per P V
+  uint64_t* bar_done = o_done + 1;                                    // every MMA of the CTA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, kv = blockIdx.y, split = blockIdx.z;
   const int b0 = split * p.chunks_per_split * kPfxBlocks;
   const int b1 = min(b0 + p.chunks_per_split * kPfxBlocks, p.prefix_blocks);
@@ -128,55 +139,32 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
       mbar_init(&full[k], 1);
       mbar_init(&empty[k], 1);
     }
-    mbar_init(bar_s, 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&s_full[k], 1);
+      mbar_init(&s_free[k], kPfxSoftmaxThreads);
+      mbar_init(&p_full[k], kPfxSoftmaxThreads);
+      mbar_init(&p_free[k], 1);
+    }
+    mbar_init(o_done, 1);
     mbar_init(bar_done, 1);
+    *abort_flag = 0;
     fence_barrier_init();
-    prefetch_tensormap(&kmap);
-    prefetch_tensormap(&vmap);
   }
-  if (warp == 0) {
+  if (warp == kPfxMmaWarp) {
     tmem_alloc(tmem_slot, kPfxTmemCols);
     tmem_relinquish();
   }
-  if (kv == 0) check_prefix_contract(p, tile, b0, nblk);
+  tc_fence_before_sync();
+  __syncthreads();  // barriers initialised, TMEM allocated
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_o = tmem + kPfxOCol;
 
-  // ---- K/V chunk c (blocks b0 + 4c ..) into stage c % 2; blocks past the
-  // split, and table entries outside the pool, read as zeros (TMA fill)
-  auto issue_chunk = [&](int c) {
-    const int stage = c % kPfxStages;
-    uint8_t* kst = smem + Ly::kOffStage + stage * Ly::kStage;
-    uint8_t* vst = kst + Ly::kKV;
-    mbar_arrive_expect_tx(&full[stage], Ly::kStage);
-#pragma unroll
-    for (int i = 0; i < kPfxBlocks; ++i) {
-      const int b = b0 + c * kPfxBlocks + i;
-      int phys = -1;
-      if (b < b1) {
-        phys = __ldg(p.block_tables + b);
-        if (phys < 0 || (long long)phys >= p.num_blocks) {
-          flag_error(p.err, DEVERR_BLOCK_RANGE);
-          phys = -1;
-        }
-      }
-#pragma unroll
-      for (int db = 0; db < Ly::kDBlk; ++db) {
-        const uint32_t off = db * (kPfxTok * 128) + i * (kBlockSize * 128);
-        tma_load_3d(kst + off, &kmap, 0, kv * Ly::kDBlk + db, phys * kBlockSize, &full[stage]);
-        tma_load_3d(vst + off, &vmap, 0, kv * Ly::kDBlk + db, phys * kBlockSize, &full[stage]);
-      }
-    }
-  };
-  __syncthreads();  // barriers initialised
-  int issued = 0;
-  if (tid == 0) {
-    for (; issued < min(nchunks, kPfxStages); ++issued) issue_chunk(issued);
-  }
-
-  // ---- this thread's query row into the K-major swizzled Q tile: 16-byte
-  // piece j of row r at column block j / 8, position (j % 8) ^ (r % 8)
+  // ---- softmax warps: this thread's query row into the K-major swizzled Q
+  // tile (16-byte piece j of row r at column block j / 8, position (j % 8) ^ (r % 8))
   const int row = tile * kPfxRows + tid;
-  const bool row_ok = row < p.rows;
-  {
+  const bool row_ok = tid < kPfxSoftmaxThreads && row < p.rows;
+  if (tid < kPfxSoftmaxThreads) {
     const int s = row_ok ? row / p.G : 0, h = row_ok ? row % p.G : 0;
     const uint4* src = reinterpret_cast<const uint4*>(p.query + ((size_t)s * p.n_q + kv * p.G + h) * D);
 #pragma unroll
@@ -185,159 +173,247 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
       const uint32_t off = (j >> 3) * (kPfxRows * 128) + tid * 128 + (((j & 7) ^ (tid & 7)) << 4);
       *reinterpret_cast<uint4*>(q_tile + off) = v;
     }
+    fence_proxy_async_smem();
   }
-  fence_proxy_async_smem();
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t t_s = tmem, t_o = tmem + kPfxOCol;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
+  // the Q tile is complete once the softmax warps and the MMA warp meet here
+  // (the TMA warp does not wait for it)
+  if (warp != kPfxTmaWarp) named_barrier(1, kPfxSoftmaxThreads + 32);
 
-  constexpr uint32_t idesc_qk = umma_idesc_bf16(kPfxRows, kPfxTok, false, false);
-  constexpr uint32_t idesc_pv = umma_idesc_bf16(kPfxRows, D, false, true);
-  const uint32_t q_addr = smem_addr(q_tile), p_addr = smem_addr(p_tile);
-  auto issue_qk = [&](int c) {
-    const uint32_t k_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage);
+  if (warp == kPfxTmaWarp) {
+    // ---------------------------------------------------------- TMA warp
+    // lane i holds the physical block of the split's blocks b0 + i, b0 + 32 + i, ...
+    constexpr int kMaxHeld = 4;  // up to 128 blocks per split held in registers
+    int held[kMaxHeld];
 #pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * (kPfxRows * 128) + (ks & 3) * 32, 16, 1024);
-      const uint64_t b = umma_desc_sw128(k_addr + (ks >> 2) * (kPfxTok * 128) + (ks & 3) * 32, 16, 1024);
-      umma_bf16(t_s, a, b, idesc_qk, ks > 0);
+    for (int r = 0; r < kMaxHeld; ++r) {
+      const int b = b0 + r * 32 + lane;
+      held[r] = -1;
+      if (b < b1) {
+        held[r] = __ldg(p.block_tables + b);
+        if (held[r] < 0 || (long long)held[r] >= p.num_blocks) {
+          flag_error(p.err, DEVERR_BLOCK_RANGE);
+          held[r] = -1;
+        }
+      }
     }
-    umma_commit(bar_s);
-  };
-  auto issue_pv = [&](int c) {
-    const uint32_t v_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage + Ly::kKV);
+    int issued = 0;
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+    }
+    for (; issued < nchunks; ++issued) {
+      // the chunk's four physical blocks (-1: past the split or outside the pool)
+      int phys4[kPfxBlocks];
 #pragma unroll
-    for (int kt = 0; kt < kPfxTok / 16; ++kt) {
-      const uint64_t a = umma_desc_sw128(p_addr + kt * 32, 16, 1024);
-      const uint64_t b = umma_desc_sw128(v_addr + kt * 2048, kPfxTok * 128, 1024);
-      umma_bf16(t_o, a, b, idesc_pv, (c > 0 || kt > 0) ? 1u : 0u);
-    }
-    umma_commit(&empty[c % kPfxStages]);
-  };
-
-  bool ok = true;
-  int waited = 0;  // chunks whose K/V landing thread 0 has waited for
-  if (tid == 0 && nchunks > 0) {
-    ok = mbar_wait(&full[0], 0, p.wait_limit);
-    if (ok) {
-      waited = 1;
-      issue_qk(0);
-    }
-  }
-
-  float m = -INFINITY, l = 0.f;  // this row's running max (log2 units) and sum
-  int c = 0;
-  for (; c < nchunks; ++c) {
-    ok = mbar_wait(bar_s, c & 1, p.wait_limit) && ok;
-    tc_fence_after_sync();
-    // ---- this row's 64 scores (raw Q K^T); tokens past the split do not count
-    uint32_t sr[2][32];
-    tmem_ld32(t_s + lane_base, sr[0]);
-    tmem_ld32(t_s + lane_base + 32, sr[1]);
-    tmem_wait_ld();
-    const int valid = min(kPfxTok, (nblk - c * kPfxBlocks) * kBlockSize);
-    float mx = -INFINITY;
+      for (int i = 0; i < kPfxBlocks; ++i) {
+        const int j = issued * kPfxBlocks + i;  // block index inside the split
+        int v = -1;
 #pragma unroll
-    for (int j = 0; j < kPfxTok; ++j) {
-      if (j >= valid) sr[j >> 5][j & 31] = __float_as_uint(-INFINITY);
-      mx = fmaxf(mx, __uint_as_float(sr[j >> 5][j & 31]));
+        for (int r = 0; r < kMaxHeld; ++r) v = (j >> 5) == r ? held[r] : v;
+        phys4[i] = __shfl_sync(0xffffffffu, v, j & 31);
+        if (j >= kMaxHeld * 32 && b0 + j < b1) {  // a split longer than the lanes hold: read it here
+          phys4[i] = __ldg(p.block_tables + b0 + j);
+          if (phys4[i] < 0 || (long long)phys4[i] >= p.num_blocks) {
+            if (lane == 0) flag_error(p.err, DEVERR_BLOCK_RANGE);
+            phys4[i] = -1;
+          }
+        }
+      }
+      if (lane == 0) {
+        const int k = issued, stage = k % kPfxStages;
+        // the stage's previous chunk (k - stages) must have gone through P V
+        if (k >= kPfxStages && !mbar_wait(&empty[stage], ((k / kPfxStages) - 1) & 1, p.wait_limit))
+          atomicExch(abort_flag, 1);
+        uint8_t* kst = smem + Ly::kOffStage + stage * Ly::kStage;
+        uint8_t* vst = kst + Ly::kKV;
+        if (!*abort_flag) {
+          mbar_arrive_expect_tx(&full[stage], Ly::kStage);
+#pragma unroll
+          for (int i = 0; i < kPfxBlocks; ++i) {
+            // blocks past the split, and table entries outside the pool, read as zeros (TMA fill)
+#pragma unroll
+            for (int db = 0; db < Ly::kDBlk; ++db) {
+              const uint32_t off = db * (kPfxTok * 128) + i * (kBlockSize * 128);
+              tma_load_3d(kst + off, &kmap, 0, kv * Ly::kDBlk + db, phys4[i] * kBlockSize, &full[stage]);
+              tma_load_3d(vst + off, &vmap, 0, kv * Ly::kDBlk + db, phys4[i] * kBlockSize, &full[stage]);
+            }
+          }
+        }
+      }
+      if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
     }
-    mx *= p.scale_log2;
-    // lazy running max: moved only when a score passes it by more than 2^8
-    // (the previous P V is complete: its commit precedes this chunk's S)
-    const bool need = c > 0 && mx > m + 8.f;
-    if (__any_sync(0xffffffffu, need)) {
-      const float alpha = need ? ex2_approx(m - mx) : 1.f;
+    // never leave with copies in flight: the last stages issued have landed
+    if (lane == 0) {
+      for (int k = max(0, issued - kPfxStages); k < issued; ++k)
+        mbar_wait(&full[k % kPfxStages], (k / kPfxStages) & 1);
+    }
+  } else if (warp == kPfxMmaWarp) {
+    // ---------------------------------------------------------- MMA warp
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(kPfxRows, kPfxTok, false, false);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(kPfxRows, D, false, true);
+      const uint32_t q_addr = smem_addr(q_tile);
+      auto issue_pv = [&](int c) {  // O += P(c) V(c), then free the stage and the P tile
+        const uint32_t v_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage + Ly::kKV);
+        const uint32_t pt = smem_addr(smem + Ly::kOffP + (c & 1) * Ly::kP);
+#pragma unroll
+        for (int kt = 0; kt < kPfxTok / 16; ++kt) {
+          const uint64_t a = umma_desc_sw128(pt + kt * 32, 16, 1024);
+          const uint64_t b = umma_desc_sw128(v_addr + kt * 2048, kPfxTok * 128, 1024);
+          umma_bf16(t_o, a, b, idesc_pv, (c > 0 || kt > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[c % kPfxStages]);
+        umma_commit(&p_free[c & 1]);
+        umma_commit(o_done);
+      };
+      bool ok = true;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        ok = mbar_wait(&full[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
+        if (ok && c >= 2) ok = mbar_wait(&s_free[c & 1], ((c - 2) >> 1) & 1, p.wait_limit);
+        if (!ok) break;
+        tc_fence_after_sync();
+        // S(c) = Q K(c)^T into S buffer c % 2
+        const uint32_t k_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * (kPfxRows * 128) + (ks & 3) * 32, 16, 1024);
+          const uint64_t b = umma_desc_sw128(k_addr + (ks >> 2) * (kPfxTok * 128) + (ks & 3) * 32, 16, 1024);
+          umma_bf16(tmem + (c & 1) * kPfxTok, a, b, idesc_qk, ks > 0);
+        }
+        umma_commit(&s_full[c & 1]);
+        // P V of the chunk before, once its probabilities are written
+        if (c >= 1) {
+          ok = mbar_wait(&p_full[(c - 1) & 1], ((c - 1) >> 1) & 1, p.wait_limit);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv(c - 1);
+        }
+      }
+      if (ok && nchunks > 0) {
+        ok = mbar_wait(&p_full[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1, p.wait_limit);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_pv(nchunks - 1);
+        }
+      }
+      if (!ok) atomicExch(abort_flag, 1);
+      // every MMA issued has completed before the CTA moves on
+      umma_commit(bar_done);
+      mbar_wait(bar_done, 0);
+    }
+  } else {
+    // ---------------------------------------------------------- softmax warps
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lanes
+    float m = -INFINITY, l = 0.f;                             // running max (log2 units) and sum
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      if (!mbar_wait(&s_full[c & 1], (c >> 1) & 1, p.wait_limit)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      // ---- this row's 64 scores (raw Q K^T); tokens past the split do not count
+      uint32_t sr[2][32];
+      tmem_ld32(tmem + (c & 1) * kPfxTok + lane_base, sr[0]);
+      tmem_ld32(tmem + (c & 1) * kPfxTok + lane_base + 32, sr[1]);
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      mbar_arrive(&s_free[c & 1]);
+      const int valid = min(kPfxTok, (nblk - c * kPfxBlocks) * kBlockSize);
+      if (valid < kPfxTok) {
+#pragma unroll
+        for (int j = 0; j < kPfxTok; ++j)
+          if (j >= valid) sr[j >> 5][j & 31] = __float_as_uint(-INFINITY);
+      }
+      // row max over eight independent chains
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(sr[0][e]);
+#pragma unroll
+      for (int j = 8; j < kPfxTok; ++j) mx8[j & 7] = fmaxf(mx8[j & 7], __uint_as_float(sr[j >> 5][j & 31]));
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      mx *= p.scale_log2;
+      // lazy running max: moved only when a score passes it by more than 2^8;
+      // the O row is rescaled once the P V before has completed
+      const bool need = c > 0 && mx > m + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        if (!mbar_wait(o_done, (c - 1) & 1, p.wait_limit)) ok = false;
+        tc_fence_after_sync();
+        const float alpha = need ? ex2_approx(m - mx) : 1.f;
+#pragma unroll
+        for (int cb = 0; cb < D / 32; ++cb) {
+          uint32_t orow[32];
+          tmem_ld32(t_o + lane_base + cb * 32, orow);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * alpha);
+          tmem_st32(t_o + lane_base + cb * 32, orow);
+        }
+        tmem_wait_st();
+        if (need) {
+          l *= alpha;
+          m = mx;
+        }
+      }
+      if (c == 0) m = mx;
+      // ---- probabilities in bf16 into P tile c % 2 (row tid, K-major, 128-byte swizzle),
+      // once the P V two chunks back is done with it
+      if (c >= 2 && !mbar_wait(&p_free[c & 1], ((c - 2) >> 1) & 1, p.wait_limit)) ok = false;
+      uint8_t* pt = smem + Ly::kOffP + (c & 1) * Ly::kP;
+      float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // row sum over four independent chains
+#pragma unroll
+      for (int j8 = 0; j8 < kPfxTok / 8; ++j8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = j8 * 8 + 2 * e;
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[j >> 5][j & 31]), p.scale_log2, -m));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31]), p.scale_log2, -m));
+          ls4[e] += p0 + p1;
+          w[e] = pack_bf16(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(pt + tid * 128 + ((j8 ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+      fence_proxy_async_smem();
+      tc_fence_before_sync();
+      mbar_arrive(&p_full[c & 1]);
+      if (!ok) break;
+    }
+    // ---- the last P V done: normalised partial o and base-2 lse of this row
+    // and split (every lane takes part in the warp-wide loads; rows past the
+    // batch store nothing)
+    if (ok && nchunks > 0 && !mbar_wait(o_done, (nchunks - 1) & 1, p.wait_limit)) ok = false;
+    if (!__all_sync(0xffffffffu, ok)) {
+      atomicExch(abort_flag, 1);
+    } else {
+      tc_fence_after_sync();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float4* dst =
+          reinterpret_cast<float4*>(p.part_o + (((size_t)kv * p.rows + (row_ok ? row : 0)) * p.splits + split) * D);
 #pragma unroll
       for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t orow[32];
         tmem_ld32(t_o + lane_base + cb * 32, orow);
         tmem_wait_ld();
+        if (row_ok) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) orow[j] = __float_as_uint(__uint_as_float(orow[j]) * alpha);
-        tmem_st32(t_o + lane_base + cb * 32, orow);
-      }
-      tmem_wait_st();
-      if (need) {
-        l *= alpha;
-        m = mx;
-      }
-    }
-    if (c == 0) m = mx;
-    // ---- probabilities in bf16 into the P tile (row tid, K-major, 128-byte swizzle)
-    float lsum = 0.f;
-#pragma unroll
-    for (int j8 = 0; j8 < kPfxTok / 8; ++j8) {
-      uint32_t w[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = j8 * 8 + 2 * e;
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[j >> 5][j & 31]), p.scale_log2, -m));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[(j + 1) >> 5][(j + 1) & 31]), p.scale_log2, -m));
-        lsum += p0 + p1;
-        w[e] = pack_bf16(p0, p1);
-      }
-      *reinterpret_cast<uint4*>(p_tile + tid * 128 + ((j8 ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    l += lsum;
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    if (tid == 0) {
-      tc_fence_after_sync();
-      issue_pv(c);
-      if (c + 1 < nchunks) {
-        ok = mbar_wait(&full[(c + 1) % kPfxStages], ((c + 1) / kPfxStages) & 1, p.wait_limit);
-        if (ok) {
-          waited = c + 2;
-          issue_qk(c + 1);
+          for (int j = 0; j < 8; ++j)
+            dst[cb * 8 + j] = make_float4(__uint_as_float(orow[4 * j]) * inv, __uint_as_float(orow[4 * j + 1]) * inv,
+                                          __uint_as_float(orow[4 * j + 2]) * inv,
+                                          __uint_as_float(orow[4 * j + 3]) * inv);
         }
       }
-      if (ok && issued < nchunks) {
-        // the stage of chunk c is free once its P V completed
-        ok = mbar_wait(&empty[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
-        if (ok) issue_chunk(issued++);
-      }
+      if (row_ok) p.part_lse[((size_t)kv * p.rows + row) * p.splits + split] = nchunks > 0 ? m + log2f(l) : -INFINITY;
     }
   }
 
-  // ---- every MMA done (also on the error path: nothing in flight at exit)
-  if (tid == 0) {
-    umma_commit(bar_done);
-    if (!mbar_wait(bar_done, 0)) ok = false;
-    // chunks issued but never waited for (error path): let them land
-    for (int k = waited; k < issued; ++k) mbar_wait(&full[k % kPfxStages], (k / kPfxStages) & 1);
-  }
-  ok = __syncthreads_and(ok && c == nchunks);
-  tc_fence_after_sync();
-  if (!ok) {
-    if (tid == 0) flag_error(p.err, DEVERR_TIMEOUT);
-  } else {
-    // ---- normalised partial o and base-2 lse of this row and split (every
-    // lane takes part in the warp-wide loads; rows past the batch store nothing)
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    float4* dst = reinterpret_cast<float4*>(p.part_o + (((size_t)kv * p.rows + (row_ok ? row : 0)) * p.splits + split) * D);
-#pragma unroll
-    for (int cb = 0; cb < D / 32; ++cb) {
-      uint32_t orow[32];
-      tmem_ld32(t_o + lane_base + cb * 32, orow);
-      tmem_wait_ld();
-      if (row_ok) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-          dst[cb * 8 + j] = make_float4(__uint_as_float(orow[4 * j]) * inv, __uint_as_float(orow[4 * j + 1]) * inv,
-                                        __uint_as_float(orow[4 * j + 2]) * inv, __uint_as_float(orow[4 * j + 3]) * inv);
-      }
-    }
-    if (row_ok) p.part_lse[((size_t)kv * p.rows + row) * p.splits + split] = nchunks > 0 ? m + log2f(l) : -INFINITY;
-  }
+  if (kv == 0) check_prefix_contract(p, tile, b0, nblk);
   tc_fence_before_sync();
-  __syncthreads();
-  if (warp == 0) {
+  __syncthreads();  // nothing in flight, every TMEM read done
+  if (tid == 0 && *abort_flag) flag_error(p.err, DEVERR_TIMEOUT);
+  if (warp == kPfxMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kPfxTmemCols);
   }
