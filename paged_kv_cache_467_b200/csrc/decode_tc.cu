@@ -265,6 +265,17 @@ __device__ __forceinline__ int d_of(int mt, int hi, int g) {
   else return g * 16 + 2 * mt + hi;
 }
 
+// Factor between an accumulator entry (m-tile mt, row g (hi = 0) or g + 8
+// (hi = 1) of P.V) and the value it stands for: INT4 high nibbles and 2-bit
+// codes are unpacked where they sit in their byte, so those entries hold 16
+// (INT4, rows g + 8) or 4^(mt % 4) (2-bit, m-tile mt) times the sum.
+template <int CACHE>
+__device__ __forceinline__ float v_unscale(int mt, int hi) {
+  if constexpr (CACHE == TC_INT4) return hi ? 1.f / 16.f : 1.f;
+  else if constexpr (CACHE == TC_KIVI) return 1.f / (float)(1 << (2 * (mt & 3)));
+  else return 1.f;
+}
+
 // ---------------------------------------------------------------- merge
 // A unit split over several CTAs leaves one normalised partial output and its
 // base-2 log-sum-exp per CTA ("piece").  A second launch, queued behind the
@@ -787,14 +798,15 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       }
       // k-step ks: word m = ks >> 2 of the row, byte pair (t, t + 2) with
       // t = (ks >> 1) & 1, codes s0 = 2 (ks & 1) and s0 + 1 of each byte:
-      // dims 32c + 16m + 4t + s and 32c + 16m + 8 + 4t + s
+      // dims 32c + 16m + 4t + s and 32c + 16m + 8 + 4t + s.  The codes are
+      // unpacked where they sit (times 4^s0, 4^(s0+1)); the query parts carry
+      // 4^-s0 and 4^-(s0+1) (kivi_query_factor).
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         const int m = ks >> 2, t = (ks >> 1) & 1, s0 = 2 * (ks & 1);
-        const uint32_t w0 = m ? r0.y : r0.x, w1 = m ? r1.y : r1.x;
-        const int sh = 2 * s0 + 8 * t;
-        const uint32_t af[4] = {i2x2_to_f16x2(w0 >> sh), i2x2_to_f16x2(w1 >> sh), i2x2_to_f16x2(w0 >> (sh + 2)),
-                                i2x2_to_f16x2(w1 >> (sh + 2))};
+        const uint32_t w0 = (m ? r0.y : r0.x) >> (8 * t), w1 = (m ? r1.y : r1.x) >> (8 * t);
+        const uint32_t af[4] = {i2x2_at_to_f16x2(w0, s0), i2x2_at_to_f16x2(w1, s0), i2x2_at_to_f16x2(w0, s0 + 1),
+                                i2x2_at_to_f16x2(w1, s0 + 1)};
         const uint32_t b0 = hmul2_u32(qf[ks][0], pack_f16(f[4 * m + t][s0], f[4 * m + t + 2][s0]));
         const uint32_t b1 = hmul2_u32(qf[ks][1], pack_f16(f[4 * m + t][s0 + 1], f[4 * m + t + 2][s0 + 1]));
         if (ks & 1) mma_f16(sb, af, b0, b1);
@@ -923,11 +935,14 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       for (int J = 0; J < 2; ++J) {
         const uint32_t sel = J ? 0x7632u : 0x5410u;
         const uint32_t z0 = prmt(x0, y0, sel), z1 = prmt(x1, y1, sel);
+        const uint32_t h0 = z0 >> 8, h1 = z1 >> 8;
 #pragma unroll
         for (int s2 = 0; s2 < 4; ++s2) {
-          // codes are finite and masked tokens carry P = 0: no V mask needed
-          const uint32_t af[4] = {i2x2_to_f16x2(z0 >> (2 * s2)), i2x2_to_f16x2(z0 >> (2 * s2 + 8)),
-                                  i2x2_to_f16x2(z1 >> (2 * s2)), i2x2_to_f16x2(z1 >> (2 * s2 + 8))};
+          // codes are finite and masked tokens carry P = 0: no V mask needed.
+          // Unpacked where they sit, m-tile 4J + s2 holds 4^s2 times the
+          // values (v_unscale takes the factor out at the end)
+          const uint32_t af[4] = {i2x2_at_to_f16x2(z0, s2), i2x2_at_to_f16x2(h0, s2), i2x2_at_to_f16x2(z1, s2),
+                                  i2x2_at_to_f16x2(h1, s2)};
           mma_f16(acc[4 * J + s2], af, pb0, pb1);
         }
       }
@@ -940,17 +955,19 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       const uint2 x0 = row8(2 * c), y0 = row8(2 * c + 1), x1 = row8(2 * c + 8), y1 = row8(2 * c + 9);
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
-        // dims 16g + 2mt (+1): byte mt of the 8, low (high) nibble; tokens side by side
+        // dims 16g + 2mt (+1): byte mt of the 8, low (high) nibble; tokens side by
+        // side.  The high nibbles are unpacked where they sit, as 16 times the
+        // codes (v_unscale takes the factor out of rows g + 8 at the end)
         const int wi = mt >> 2, b = mt & 3;
         const uint32_t sel = b | (b << 4) | ((4 + b) << 8) | ((4 + b) << 12);
-        const uint32_t z0 = prmt((&x0.x)[wi], (&y0.x)[wi], sel) ^ 0x88888888u;
-        const uint32_t z1 = prmt((&x1.x)[wi], (&y1.x)[wi], sel) ^ 0x88888888u;
+        const uint32_t z0 = prmt((&x0.x)[wi], (&y0.x)[wi], sel);
+        const uint32_t z1 = prmt((&x1.x)[wi], (&y1.x)[wi], sel);
         uint32_t af[4];
         // codes are finite and masked tokens carry P = 0: no V mask needed
-        af[0] = i4x2_to_f16x2(z0);
-        af[1] = i4x2_to_f16x2(z0 >> 4);
-        af[2] = i4x2_to_f16x2(z1);
-        af[3] = i4x2_to_f16x2(z1 >> 4);
+        af[0] = i4x2_at_to_f16x2<false>(z0);
+        af[1] = i4x2_at_to_f16x2<true>(z0);
+        af[2] = i4x2_at_to_f16x2<false>(z1);
+        af[3] = i4x2_at_to_f16x2<true>(z1);
         mma_f16(acc[mt], af, pb0, pb1);
       }
     } else {
@@ -1239,9 +1256,12 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
         }
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
+          // the K codes of k-step ks come as 4^s0 and 4^(s0+1) times their values
+          // (s0 = 2 (ks & 1)): the query parts take 4^-s0 and 4^-(s0+1)
           const int e = 16 * (ks >> 2) + 4 * ((ks >> 1) & 1) + 2 * (ks & 1);
-          qf[ks][0] = pack_f16(x[e], x[e + 8]);
-          qf[ks][1] = pack_f16(x[e + 1], x[e + 9]);
+          const float f0 = (ks & 1) ? 1.f / 16.f : 1.f, f1 = (ks & 1) ? 1.f / 64.f : 0.25f;
+          qf[ks][0] = pack_f16(x[e] * f0, x[e + 8] * f0);
+          qf[ks][1] = pack_f16(x[e + 1] * f1, x[e + 9] * f1);
         }
       }
 #pragma unroll
@@ -1260,8 +1280,9 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
 #pragma unroll
           for (int hi = 0; hi < 2; ++hi) {
             const int dd = d_of<CACHE, D>(mt, hi, g);
-            if (head0_ok) acc[mt][2 * hi] = __ldcg(o0 + dd);
-            if (head1_ok) acc[mt][2 * hi + 1] = __ldcg(o0 + D + dd);
+            const float f = 1.f / v_unscale<CACHE>(mt, hi);
+            if (head0_ok) acc[mt][2 * hi] = __ldcg(o0 + dd) * f;
+            if (head1_ok) acc[mt][2 * hi + 1] = __ldcg(o0 + D + dd) * f;
           }
         }
         if (head0_ok) m0 = __ldcg(p.pre_lse + r0);
@@ -1295,6 +1316,17 @@ __global__ void __launch_bounds__((MAXW + 1) * 32, MINB)
       for (int o = 4; o < 32; o <<= 1) {
         lt0 += __shfl_xor_sync(0xffffffffu, lt0, o);
         lt1 += __shfl_xor_sync(0xffffffffu, lt1, o);
+      }
+      if constexpr (CACHE == TC_INT4 || CACHE == TC_KIVI) {
+        // the factors of the codes unpacked in place (the range ends here)
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            acc[mt][2 * hi] *= v_unscale<CACHE>(mt, hi);
+            acc[mt][2 * hi + 1] *= v_unscale<CACHE>(mt, hi);
+          }
+        }
       }
       const float post = tc_fp8(CACHE) ? head_v_scale : 1.f;
       const float inv0 = post / lt0, inv1 = post / lt1;

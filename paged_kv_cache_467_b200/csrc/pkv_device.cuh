@@ -278,6 +278,39 @@ __device__ __forceinline__ uint32_t i2x2_to_f16x2(uint32_t t) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The two 2-bit two's-complement codes at bits [2s, 2s+1] and [16+2s, 17+2s]
+// of t (other bits ignored) -> f16x2 of the codes times 4^s, exactly: XOR with
+// 2 << 2s turns a code c in place into (c + 2) << 2s, which ORed into the
+// mantissa of 1024.0 reads as 1024 + (c + 2) 4^s; subtracting 1024 + 2 * 4^s
+// leaves c * 4^s.  One LOP3 and one HSUB2, no shift (s is a constant once the
+// caller's loop is unrolled).
+__device__ __forceinline__ uint32_t i2x2_at_to_f16x2(uint32_t t, int s) {
+  const uint32_t mask = 0x00030003u << (2 * s);
+  const uint32_t flip = 0x64006400u | (0x00020002u << (2 * s));
+  const unsigned short base = (unsigned short)(0x6400 + (2 << (2 * s)));  // f16 of 1024 + 2 * 4^s
+  const uint32_t h = (t & mask) ^ flip;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __half2half2(__ushort_as_half(base)));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// The two two's-complement 4-bit codes in the low (HI = false) or high
+// (HI = true) nibbles of bytes 0 and 2 of t -> f16x2 of the codes (low) or of
+// 16 times the codes (high), exactly: XOR with 8 << shift makes the nibble
+// n = code + 8 in place, which ORed into the mantissa of 1024.0 reads as
+// 1024 + n (or 1024 + 16 n); subtracting 1032 (or 1152) leaves the code (or
+// 16 times it).  One LOP3 and one HSUB2, no shift.
+template <bool HI>
+__device__ __forceinline__ uint32_t i4x2_at_to_f16x2(uint32_t t) {
+  constexpr uint32_t mask = HI ? 0x00F000F0u : 0x000F000Fu;
+  constexpr uint32_t flip = HI ? 0x64806480u : 0x64086408u;
+  constexpr unsigned short base = HI ? 0x6480 : 0x6408;  // f16 of 1152 = 1024 + 16 * 8, of 1032 = 1024 + 8
+  const uint32_t h = (t & mask) ^ flip;
+  __half2 v = *reinterpret_cast<const __half2*>(&h);
+  v = __hsub2(v, __half2half2(__ushort_as_half(base)));
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&a), *reinterpret_cast<const __half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
