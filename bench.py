@@ -110,6 +110,8 @@ KERNEL_SOURCES = {
     "decode": ("decode_tc.cu", "pkv_device.cuh", "cache_row.cuh", "internal.h"),
     "prefix": ("prefix.cu", "tcgen05.cuh", "pkv_device.cuh", "internal.h"),
     "kivi": ("kivi.cu", "decode_tc.cu", "pkv_device.cuh", "cache_row.cuh", "internal.h"),
+    # the shared-prefix step: the prefix pass and the decode of each sequence's own blocks
+    "prefix_step": ("decode_tc.cu", "prefix.cu", "tcgen05.cuh", "pkv_device.cuh", "cache_row.cuh", "internal.h"),
 }
 
 
@@ -620,7 +622,9 @@ def run_b200(args, rank, world, local):
         peak, peak_kind = measured_peaks()
         value = whole_job_gbs(kv_bytes, world, ms)
         achieved = kv_bytes / (att_ms * 1e-3) / 1e9
-        traffic = profiled_traffic(args.config, "kivi" if kivi else "decode")
+        traffic = None
+        if not args.seqs and not args.plain_decode and not args.unfused:
+            traffic = profiled_traffic(args.config, "kivi" if kivi else "prefix_step" if prefix_blocks else "decode")
         line = {
             "metric": METRIC,
             "value": value,
