@@ -280,13 +280,16 @@ __device__ __forceinline__ float v_unscale(int mt, int hi) {
 // A unit split over several CTAs leaves one normalised partial output and its
 // base-2 log-sum-exp per CTA ("piece").  A second launch, queued behind the
 // decode kernel with programmatic serialisation, combines them: one CTA per
-// unit, a thread per (query head, 4 dims), so every piece's loads of a thread
-// are independent and the whole merge costs about two L2 round trips instead
-// of a serial tail in the decode kernel.  Pieces are combined in a fixed
-// order: M = max lse_k, w_k = 2^(lse_k - M), o = sum w_k o_k / sum w_k,
-// lse = M + log2(sum w_k).  Under a shared prefix every unit is merged
-// (decode_merge_all_kernel): its own piece(s) (CTA pieces, or the unit's whole
-// piece) and then the prefix pass's split pieces of the same query row.
+// unit, a thread per (query head, 4 dims).  A thread loads the lse and its 4
+// dims of up to kMergeBatch pieces at once, so a merge of that many pieces
+// costs one L2 round trip, and combines them in a fixed order with a running
+// maximum: M' = max(M, lse_k), the sums so far scaled by 2^(M - M'), then
+// w_k = 2^(lse_k - M'); o = sum w_k o_k / sum w_k, lse = M + log2(sum w_k).
+// Under a shared prefix every unit is merged (decode_merge_all_kernel): its
+// own piece(s) (CTA pieces, or the unit's whole piece) and then the prefix
+// pass's split pieces of the same query row.
+constexpr int kMergeBatch = 8;
+
 struct MergeParams {
   void* out;
   float* lse_out;
@@ -298,13 +301,111 @@ struct MergeParams {
   int merge_all;
   const float* unit_o;
   const float* unit_lse;
-  const float* pre_o;    // [n_kv][pre_rows][pre_splits][D]
-  const float* pre_lse;  // [n_kv][pre_rows][pre_splits]
+  const float* pre_o;    // [n_kv][pre_splits][pre_rows][D]
+  const float* pre_lse;  // [n_kv][pre_splits][pre_rows]
   int pre_rows, pre_splits, G, HPC;
 };
 
+// Running combination of pieces (lse base 2, o normalised) in the order given.
+struct MergeAcc {
+  float M = -INFINITY, wsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  // piece(k, lse_ptr, o_ptr) names piece k's lse and this thread's 4 dims
+  template <typename PieceFn>
+  __device__ __forceinline__ void add_pieces(int n, PieceFn piece) {
+    if (n > kMergeBatch) {
+      // many pieces: the maximum over all lse first, then one pass of weights
+      // (two round trips whatever n is)
+      float mb = M;
+#pragma unroll 8
+      for (int k = 0; k < n; ++k) {
+        const float* lp;
+        const float4* op;
+        piece(k, lp, op);
+        mb = fmaxf(mb, __ldcg(lp));
+      }
+      if (mb == -INFINITY) return;
+      const float sc = ex2(M - mb);
+      wsum *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+#pragma unroll 8
+      for (int k = 0; k < n; ++k) {
+        const float* lp;
+        const float4* op;
+        piece(k, lp, op);
+        const float lv = __ldcg(lp);
+        const float4 ov = __ldcg(op);
+        if (lv > -INFINITY) {
+          const float w = ex2(lv - mb);
+          wsum += w;
+          acc.x += w * ov.x;
+          acc.y += w * ov.y;
+          acc.z += w * ov.z;
+          acc.w += w * ov.w;
+        }
+      }
+      M = mb;
+      return;
+    }
+    for (int k0 = 0; k0 < n; k0 += kMergeBatch) {
+      float lv[kMergeBatch];
+      float4 ov[kMergeBatch];
+#pragma unroll
+      for (int i = 0; i < kMergeBatch; ++i) {
+        lv[i] = -INFINITY;
+        ov[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k0 + i < n) {
+          const float* lp;
+          const float4* op;
+          piece(k0 + i, lp, op);
+          lv[i] = __ldcg(lp);
+          ov[i] = __ldcg(op);
+        }
+      }
+      float mb = M;
+#pragma unroll
+      for (int i = 0; i < kMergeBatch; ++i) mb = fmaxf(mb, lv[i]);
+      if (mb == -INFINITY) continue;  // no piece with any weight yet
+      const float sc = ex2(M - mb);   // 0 while M is -inf
+      wsum *= sc;
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+#pragma unroll
+      for (int i = 0; i < kMergeBatch; ++i) {
+        if (lv[i] > -INFINITY) {
+          const float w = ex2(lv[i] - mb);
+          wsum += w;
+          acc.x += w * ov[i].x;
+          acc.y += w * ov[i].y;
+          acc.z += w * ov[i].z;
+          acc.w += w * ov[i].w;
+        }
+      }
+      M = mb;
+    }
+  }
+  // out row (bf16 or f32) and lse (natural log; -inf and zeros if nothing had weight)
+  __device__ __forceinline__ void store(const MergeParams& p, long long row, int v, int D) const {
+    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+    if (p.act_bf16) {
+      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + row * D + 4 * v);
+      o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    } else {
+      reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * D)[v] =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+    if (p.lse_out && v == 0) p.lse_out[row] = wsum > 0.f ? (M + log2f(wsum)) * kLn2 : -INFINITY;
+  }
+};
+
 template <int D>
-__global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(512, 2) decode_merge_kernel(const MergeParams p) {
   grid_launch_dependents();
   grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
   const int u = blockIdx.x;
@@ -318,42 +419,19 @@ __global__ void __launch_bounds__(256) decode_merge_kernel(const MergeParams p) 
   constexpr int V = D / 4;
   for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
     const int h = idx / V, v = idx - h * V;
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int k = 0; k < n; ++k) {
-      const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-      M = fmaxf(M, __ldcg(p.part_lse + ((size_t)(c0 + k) * 2 + slot) * p.QH + h));
-    }
-    float wsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int k = 0; k < n; ++k) {
-      const int slot = (k == 0 && c0_slot1) ? 1 : 0;
-      const size_t piece = ((size_t)(c0 + k) * 2 + slot) * p.QH + h;
-      const float w = ex2(__ldcg(p.part_lse + piece) - M);
-      const float4 o = __ldcg(reinterpret_cast<const float4*>(p.part_o + piece * D) + v);
-      wsum += w;
-      acc.x += w * o.x;
-      acc.y += w * o.y;
-      acc.z += w * o.z;
-      acc.w += w * o.w;
-    }
-    const float inv = 1.f / wsum;
-    const long long row = (long long)s * p.n_q + hg * p.QH + h;
-    if (p.act_bf16) {
-      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + row * D + 4 * v);
-      o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    } else {
-      reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * D)[v] =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
-    if (p.lse_out && v == 0) p.lse_out[row] = (M + log2f(wsum)) * kLn2;
+    MergeAcc m;
+    // CTA c0 + k's piece: slot 1 for k == 0 when the unit starts inside CTA c0's range
+    m.add_pieces(n, [&](int k, const float*& lp, const float4*& op) {
+      const size_t piece = ((size_t)(c0 + k) * 2 + ((k == 0 && c0_slot1) ? 1 : 0)) * p.QH + h;
+      lp = p.part_lse + piece;
+      op = reinterpret_cast<const float4*>(p.part_o + piece * D) + v;
+    });
+    m.store(p, (long long)s * p.n_q + hg * p.QH + h, v, D);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) decode_merge_all_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(512, 2) decode_merge_all_kernel(const MergeParams p) {
   grid_launch_dependents();
   grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
   const int u = blockIdx.x;
@@ -365,62 +443,36 @@ __global__ void __launch_bounds__(256) decode_merge_all_kernel(const MergeParams
   if (n < 0 || n > p.num_ctas || c0 >= p.num_ctas || c0 + n > p.num_ctas) n = 0;
   const int s = u / p.HG, hg = u - s * p.HG;
   const int npre = p.pre_splits;
-  const bool whole = n < 2;  // the unit's one piece (n == 1) or none (n == 0)
+  const int own = n;  // the unit's own pieces: n CTA pieces, its one whole piece (n == 1), or none
   constexpr int V = D / 4;
   for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
     const int h = idx / V, v = idx - h * V;
     const long long row = (long long)s * p.n_q + hg * p.QH + h;
-    // the unit's own pieces: CTA k's slot (k == 0 may be the CTA's second slot)
-    const float* own_lse = p.part_lse + ((size_t)c0 * 2 + (c0_slot1 ? 1 : 0)) * p.QH + h;
-    const float* own_o = p.part_o + (((size_t)c0 * 2 + (c0_slot1 ? 1 : 0)) * p.QH + h) * D;
-    const size_t own_step = (size_t)2 * p.QH;  // from CTA k's slot 0 to CTA k + 1's
-    const size_t own_back = c0_slot1 ? (size_t)p.QH : 0;  // CTA c0 + 1 and on: slot 0
-    // the prefix pass's splits of this query row, consecutive
-    const size_t pre_row = npre ? ((size_t)(hg * p.HPC + h / p.G) * p.pre_rows + (size_t)s * p.G + h % p.G) : 0;
-    const float* pre_lse = p.pre_lse + pre_row * npre;
-    const float* pre_o = p.pre_o + pre_row * npre * D;
-    float M = -INFINITY;
-    if (!whole) {
-      M = __ldcg(own_lse);
-#pragma unroll 4
-      for (int k = 1; k < n; ++k) M = fmaxf(M, __ldcg(own_lse + k * own_step - own_back));
-    } else if (n == 1) {
-      M = __ldcg(p.unit_lse + row);
-    }
-#pragma unroll 4
-    for (int k = 0; k < npre; ++k) M = fmaxf(M, __ldcg(pre_lse + k));
-    float wsum = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    auto add = [&](float lse, const float* o) {
-      const float w = ex2(lse - M);
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(o) + v);
-      wsum += w;
-      acc.x += w * x.x;
-      acc.y += w * x.y;
-      acc.z += w * x.z;
-      acc.w += w * x.w;
-    };
-    if (M > -INFINITY) {
-      if (!whole) {
-        add(__ldcg(own_lse), own_o);
-#pragma unroll 4
-        for (int k = 1; k < n; ++k) add(__ldcg(own_lse + k * own_step - own_back), own_o + (k * own_step - own_back) * D);
-      } else if (n == 1) {
-        add(__ldcg(p.unit_lse + row), p.unit_o + row * D);
+    // own piece k: the whole unit's (own == 1, written by one CTA), or CTA
+    // c0 + k's slot (slot 1 of CTA c0 when the unit starts inside its range,
+    // slot 0 after that: 2 QH lse apart)
+    const size_t own0 = own == 1 ? 0 : ((size_t)c0 * 2 + (c0_slot1 ? 1 : 0)) * p.QH + h;
+    const float* own_l = own == 1 ? p.unit_lse + row : p.part_lse + own0;
+    const float* own_o = own == 1 ? p.unit_o + row * D : p.part_o + own0 * D;
+    const long long own_back = c0_slot1 ? p.QH : 0;
+    // the prefix pass's splits of this query row, pre_rows apart
+    const int kvh = hg * p.HPC + h / p.G;
+    const size_t pre_row = (size_t)kvh * npre * p.pre_rows + (size_t)s * p.G + h % p.G;
+    const float* pre_l = p.pre_lse + pre_row;
+    const float* pre_o = p.pre_o + pre_row * D;
+    MergeAcc m;
+    m.add_pieces(own + npre, [&](int k, const float*& lp, const float4*& op) {
+      if (k < own) {
+        const long long off = k == 0 ? 0 : (long long)k * 2 * p.QH - own_back;
+        lp = own_l + off;
+        op = reinterpret_cast<const float4*>(own_o + off * D) + v;
+      } else {
+        const size_t off = (size_t)(k - own) * p.pre_rows;
+        lp = pre_l + off;
+        op = reinterpret_cast<const float4*>(pre_o + off * D) + v;
       }
-#pragma unroll 4
-      for (int k = 0; k < npre; ++k) add(__ldcg(pre_lse + k), pre_o + (size_t)k * D);
-    }
-    const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    if (p.act_bf16) {
-      __nv_bfloat162* o = reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(p.out) + row * D + 4 * v);
-      o[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      o[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    } else {
-      reinterpret_cast<float4*>(static_cast<float*>(p.out) + row * D)[v] =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    }
-    if (p.lse_out && v == 0) p.lse_out[row] = wsum > 0.f ? (M + log2f(wsum)) * kLn2 : -INFINITY;
+    });
+    m.store(p, row, v, D);
   }
 }
 
@@ -1456,10 +1508,19 @@ template <int CACHE, int D, int MAXW, int MINB = 1>
 static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
                                  const TcParams& prm, const PrefixPieces& pre, cudaStream_t stream) {
   auto kern = decode_tc_kernel<CACHE, D, MAXW, MINB>;
+  auto merge = decode_merge_kernel<D>;
+  auto merge_all = decode_merge_all_kernel<D>;
   static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
   if ((int)plan.smem_bytes > configured_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    if (configured_bytes == 0) {
+      // the whole shared memory of an SM for the step's kernels (see prefer_max_smem)
+      e = prefer_max_smem(kern);
+      if (e == cudaSuccess) e = prefer_max_smem(merge);
+      if (e == cudaSuccess) e = prefer_max_smem(merge_all);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
+    }
     configured_bytes = (int)plan.smem_bytes;
   }
   cudaLaunchConfig_t cfg = {};
@@ -1500,7 +1561,10 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mp.HPC = plan.HPC;
   cudaLaunchConfig_t mcfg = {};
   mcfg.gridDim = dim3(plan.units);
-  mcfg.blockDim = dim3((unsigned)std::min(256, (mp.QH * (D / 4) + 31) / 32 * 32));
+  // a thread per (query head, 4 dims) up to 512; at most 64 registers a
+  // thread, so that 1024 threads of merge CTAs fit an SM (the units of a
+  // batch are one wave)
+  mcfg.blockDim = dim3((unsigned)std::min(512, (mp.QH * (D / 4) + 31) / 32 * 32));
   mcfg.dynamicSmemBytes = 0;
   mcfg.stream = stream;
   cudaLaunchAttribute mattr[1];
@@ -1508,8 +1572,7 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mattr[0].val.programmaticStreamSerializationAllowed = 1;
   mcfg.attrs = mattr;
   mcfg.numAttrs = 1;
-  e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, decode_merge_all_kernel<D>, mp)
-                    : cudaLaunchKernelEx(&mcfg, decode_merge_kernel<D>, mp);
+  e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, merge_all, mp) : cudaLaunchKernelEx(&mcfg, merge, mp);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_merge_kernel launch");
   return PKV_OK;

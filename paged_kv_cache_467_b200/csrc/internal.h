@@ -52,6 +52,16 @@ struct TcPlan {
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
 
+// The kernels of a decode step (prefix pass, decode, merge) ask for the
+// largest shared-memory carveout.  An SM's split between L1 and shared memory
+// is fixed while CTAs run on it, so a kernel configured for less shared memory
+// (the default picks the smallest split that fits its own CTA) would keep the
+// CTAs of the kernel running beside it off that SM.
+template <typename Kernel>
+inline cudaError_t prefer_max_smem(Kernel kern) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+}
+
 // Start state of a decode unit (kivi.cu's residual pass): per (KV head,
 // query row = s * G + head in group) the normalised output and its base-2 lse,
 // which the decode over the quantised blocks starts from.
@@ -69,8 +79,8 @@ struct PrefixState {
 // leaves its piece in unit_o / unit_lse.
 constexpr int kMaxPrefixSplits = 64;
 struct PrefixPieces {
-  const float* o = nullptr;    // [n_kv][rows][splits][head_dim]
-  const float* lse = nullptr;  // [n_kv][rows][splits]
+  const float* o = nullptr;    // [n_kv][splits][rows][head_dim]
+  const float* lse = nullptr;  // [n_kv][splits][rows]
   int splits = 0;
   int rows = 0;
   float* unit_o = nullptr;     // [num_seqs * n_q][head_dim]
