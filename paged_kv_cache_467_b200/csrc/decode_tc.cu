@@ -280,15 +280,21 @@ __device__ __forceinline__ float v_unscale(int mt, int hi) {
 // A unit split over several CTAs leaves one normalised partial output and its
 // base-2 log-sum-exp per CTA ("piece").  A second launch, queued behind the
 // decode kernel with programmatic serialisation, combines them: one CTA per
-// unit, a thread per (query head, 4 dims).  A thread loads the lse and its 4
-// dims of up to kMergeBatch pieces at once, so a merge of that many pieces
-// costs one L2 round trip, and combines them in a fixed order with a running
-// maximum: M' = max(M, lse_k), the sums so far scaled by 2^(M - M'), then
-// w_k = 2^(lse_k - M'); o = sum w_k o_k / sum w_k, lse = M + log2(sum w_k).
+// unit (or several, see below), a thread per (query head, 4 dims).  A thread
+// loads the lse and its 4 dims of up to kMergeBatch pieces at once, so a
+// merge of that many pieces costs one L2 round trip, and combines them in a
+// fixed order with a running maximum: M' = max(M, lse_k), the sums so far
+// scaled by 2^(M - M'), then w_k = 2^(lse_k - M'); o = sum w_k o_k / sum w_k,
+// lse = M + log2(sum w_k); with more pieces it takes the maximum first and
+// then one weighted pass.  When units are expected to have more pieces than
+// kMergeBatch, kMergeLanes lanes share a (query head, 4 dims): lane r takes
+// pieces r, r + kMergeLanes, ..., and the lanes' sums meet in a fixed shuffle
+// tree, over as many CTAs per unit as that takes.
 // Under a shared prefix every unit is merged (decode_merge_all_kernel): its
 // own piece(s) (CTA pieces, or the unit's whole piece) and then the prefix
 // pass's split pieces of the same query row.
 constexpr int kMergeBatch = 8;
+constexpr int kMergeLanes = 8;
 
 struct MergeParams {
   void* out;
@@ -310,15 +316,16 @@ struct MergeParams {
 struct MergeAcc {
   float M = -INFINITY, wsum = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  // piece(k, lse_ptr, o_ptr) names piece k's lse and this thread's 4 dims
+  // Pieces k = first, first + stride, ... below n; piece(k, lse_ptr, o_ptr)
+  // names piece k's lse and this thread's 4 dims.
   template <typename PieceFn>
-  __device__ __forceinline__ void add_pieces(int n, PieceFn piece) {
-    if (n > kMergeBatch) {
+  __device__ __forceinline__ void add_pieces(int n, int first, int stride, PieceFn piece) {
+    const int cnt = first < n ? (n - first + stride - 1) / stride : 0;
+    if (cnt > kMergeBatch) {
       // many pieces: the maximum over all lse first, then one pass of weights
-      // (two round trips whatever n is)
       float mb = M;
 #pragma unroll 8
-      for (int k = 0; k < n; ++k) {
+      for (int k = first; k < n; k += stride) {
         const float* lp;
         const float4* op;
         piece(k, lp, op);
@@ -332,7 +339,7 @@ struct MergeAcc {
       acc.z *= sc;
       acc.w *= sc;
 #pragma unroll 8
-      for (int k = 0; k < n; ++k) {
+      for (int k = first; k < n; k += stride) {
         const float* lp;
         const float4* op;
         piece(k, lp, op);
@@ -350,17 +357,17 @@ struct MergeAcc {
       M = mb;
       return;
     }
-    for (int k0 = 0; k0 < n; k0 += kMergeBatch) {
+    if (cnt > 0) {
       float lv[kMergeBatch];
       float4 ov[kMergeBatch];
 #pragma unroll
       for (int i = 0; i < kMergeBatch; ++i) {
         lv[i] = -INFINITY;
         ov[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (k0 + i < n) {
+        if (i < cnt) {
           const float* lp;
           const float4* op;
-          piece(k0 + i, lp, op);
+          piece(first + i * stride, lp, op);
           lv[i] = __ldcg(lp);
           ov[i] = __ldcg(op);
         }
@@ -368,7 +375,7 @@ struct MergeAcc {
       float mb = M;
 #pragma unroll
       for (int i = 0; i < kMergeBatch; ++i) mb = fmaxf(mb, lv[i]);
-      if (mb == -INFINITY) continue;  // no piece with any weight yet
+      if (mb == -INFINITY) return;  // no piece with any weight
       const float sc = ex2(M - mb);   // 0 while M is -inf
       wsum *= sc;
       acc.x *= sc;
@@ -389,6 +396,31 @@ struct MergeAcc {
       M = mb;
     }
   }
+  // The sums of the `lanes` lanes that share this thread's (query head, 4
+  // dims), combined in a fixed tree; every lane ends with the total.
+  template <int lanes>
+  __device__ __forceinline__ void reduce_lanes() {
+    if constexpr (lanes == 1) return;
+    float Mt = M;
+#pragma unroll
+    for (int o = 1; o < lanes; o <<= 1) Mt = fmaxf(Mt, __shfl_xor_sync(0xffffffffu, Mt, o));
+    if (Mt == -INFINITY) return;  // no lane has a piece with weight
+    const float sc = M == -INFINITY ? 0.f : ex2(M - Mt);
+    wsum *= sc;
+    acc.x *= sc;
+    acc.y *= sc;
+    acc.z *= sc;
+    acc.w *= sc;
+#pragma unroll
+    for (int o = 1; o < lanes; o <<= 1) {
+      wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+      acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+      acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+      acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+      acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    M = Mt;
+  }
   // out row (bf16 or f32) and lse (natural log; -inf and zeros if nothing had weight)
   __device__ __forceinline__ void store(const MergeParams& p, long long row, int v, int D) const {
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -404,7 +436,7 @@ struct MergeAcc {
   }
 };
 
-template <int D>
+template <int D, int L>
 __global__ void __launch_bounds__(512, 2) decode_merge_kernel(const MergeParams p) {
   grid_launch_dependents();
   grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
@@ -417,20 +449,25 @@ __global__ void __launch_bounds__(512, 2) decode_merge_kernel(const MergeParams 
   if (n < 2 || n > p.num_ctas || c0 >= p.num_ctas || c0 + n > p.num_ctas) return;
   const int s = u / p.HG, hg = u - s * p.HG;
   constexpr int V = D / 4;
-  for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
-    const int h = idx / V, v = idx - h * V;
+  const int r = threadIdx.x % L;  // L lanes per (query head, 4 dims); L divides the block
+  const int pairs = p.QH * V, step = gridDim.y * blockDim.x / L;
+  for (int idx = (blockIdx.y * blockDim.x + threadIdx.x) / L; idx - (int)(threadIdx.x / L) < pairs; idx += step) {
+    const bool live = idx < pairs;  // a lane group past the end still joins the shuffles
+    const int h = live ? idx / V : 0, v = live ? idx - h * V : 0;
     MergeAcc m;
     // CTA c0 + k's piece: slot 1 for k == 0 when the unit starts inside CTA c0's range
-    m.add_pieces(n, [&](int k, const float*& lp, const float4*& op) {
-      const size_t piece = ((size_t)(c0 + k) * 2 + ((k == 0 && c0_slot1) ? 1 : 0)) * p.QH + h;
-      lp = p.part_lse + piece;
-      op = reinterpret_cast<const float4*>(p.part_o + piece * D) + v;
-    });
-    m.store(p, (long long)s * p.n_q + hg * p.QH + h, v, D);
+    if (live)
+      m.add_pieces(n, r, L, [&](int k, const float*& lp, const float4*& op) {
+        const size_t piece = ((size_t)(c0 + k) * 2 + ((k == 0 && c0_slot1) ? 1 : 0)) * p.QH + h;
+        lp = p.part_lse + piece;
+        op = reinterpret_cast<const float4*>(p.part_o + piece * D) + v;
+      });
+    m.reduce_lanes<L>();
+    if (live && r == 0) m.store(p, (long long)s * p.n_q + hg * p.QH + h, v, D);
   }
 }
 
-template <int D>
+template <int D, int L>
 __global__ void __launch_bounds__(512, 2) decode_merge_all_kernel(const MergeParams p) {
   grid_launch_dependents();
   grid_wait_prerequisites();  // the decode kernel's pieces and descriptors are complete
@@ -445,8 +482,11 @@ __global__ void __launch_bounds__(512, 2) decode_merge_all_kernel(const MergePar
   const int npre = p.pre_splits;
   const int own = n;  // the unit's own pieces: n CTA pieces, its one whole piece (n == 1), or none
   constexpr int V = D / 4;
-  for (int idx = threadIdx.x; idx < p.QH * V; idx += blockDim.x) {
-    const int h = idx / V, v = idx - h * V;
+  const int r = threadIdx.x % L;  // L lanes per (query head, 4 dims); L divides the block
+  const int pairs = p.QH * V, step = gridDim.y * blockDim.x / L;
+  for (int idx = (blockIdx.y * blockDim.x + threadIdx.x) / L; idx - (int)(threadIdx.x / L) < pairs; idx += step) {
+    const bool live = idx < pairs;  // a lane group past the end still joins the shuffles
+    const int h = live ? idx / V : 0, v = live ? idx - h * V : 0;
     const long long row = (long long)s * p.n_q + hg * p.QH + h;
     // own piece k: the whole unit's (own == 1, written by one CTA), or CTA
     // c0 + k's slot (slot 1 of CTA c0 when the unit starts inside its range,
@@ -461,7 +501,8 @@ __global__ void __launch_bounds__(512, 2) decode_merge_all_kernel(const MergePar
     const float* pre_l = p.pre_lse + pre_row;
     const float* pre_o = p.pre_o + pre_row * D;
     MergeAcc m;
-    m.add_pieces(own + npre, [&](int k, const float*& lp, const float4*& op) {
+    if (live)
+      m.add_pieces(own + npre, r, L, [&](int k, const float*& lp, const float4*& op) {
       if (k < own) {
         const long long off = k == 0 ? 0 : (long long)k * 2 * p.QH - own_back;
         lp = own_l + off;
@@ -472,7 +513,8 @@ __global__ void __launch_bounds__(512, 2) decode_merge_all_kernel(const MergePar
         op = reinterpret_cast<const float4*>(pre_o + off * D) + v;
       }
     });
-    m.store(p, row, v, D);
+    m.reduce_lanes<L>();
+    if (live && r == 0) m.store(p, row, v, D);
   }
 }
 
@@ -1508,8 +1550,10 @@ template <int CACHE, int D, int MAXW, int MINB = 1>
 static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, const CUtensorMap& vm, const CUtensorMap& sm,
                                  const TcParams& prm, const PrefixPieces& pre, cudaStream_t stream) {
   auto kern = decode_tc_kernel<CACHE, D, MAXW, MINB>;
-  auto merge = decode_merge_kernel<D>;
-  auto merge_all = decode_merge_all_kernel<D>;
+  auto merge = decode_merge_kernel<D, 1>;
+  auto merge_all = decode_merge_all_kernel<D, 1>;
+  auto merge_wide = decode_merge_kernel<D, kMergeLanes>;
+  auto merge_all_wide = decode_merge_all_kernel<D, kMergeLanes>;
   static int configured_bytes = 0;  // max dynamic smem already granted to this instantiation
   if ((int)plan.smem_bytes > configured_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem_bytes);
@@ -1519,6 +1563,8 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
       e = prefer_max_smem(kern);
       if (e == cudaSuccess) e = prefer_max_smem(merge);
       if (e == cudaSuccess) e = prefer_max_smem(merge_all);
+      if (e == cudaSuccess) e = prefer_max_smem(merge_wide);
+      if (e == cudaSuccess) e = prefer_max_smem(merge_all_wide);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(carveout)");
     }
     configured_bytes = (int)plan.smem_bytes;
@@ -1559,12 +1605,19 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mp.pre_splits = pre.splits;
   mp.G = plan.G;
   mp.HPC = plan.HPC;
+  // Pieces a unit is expected to have, with every sequence at the longest
+  // length: about num_ctas / units + 1 (plus the prefix's splits).  Past
+  // kMergeBatch, kMergeLanes lanes share each (query head, 4 dims), if the
+  // threads that takes still fit the GPU at once (few, long units).
+  const int pieces_est = (plan.num_ctas + plan.units - 1) / std::max(1, plan.units) + 1 + (prm.merge_all ? pre.splits : 0);
+  const long long wide_threads = (long long)plan.units * mp.QH * (D / 4) * kMergeLanes;
+  const int lanes = pieces_est > kMergeBatch && wide_threads <= 1024LL * device_sm_count() ? kMergeLanes : 1;
+  const int threads = mp.QH * (D / 4) * lanes;
   cudaLaunchConfig_t mcfg = {};
-  mcfg.gridDim = dim3(plan.units);
-  // a thread per (query head, 4 dims) up to 512; at most 64 registers a
-  // thread, so that 1024 threads of merge CTAs fit an SM (the units of a
-  // batch are one wave)
-  mcfg.blockDim = dim3((unsigned)std::min(512, (mp.QH * (D / 4) + 31) / 32 * 32));
+  // up to 512 threads a CTA, as many CTAs per unit as the threads take; at
+  // most 64 registers a thread, so that 1024 threads of merge CTAs fit an SM
+  mcfg.blockDim = dim3((unsigned)std::min(512, (threads + 31) / 32 * 32));
+  mcfg.gridDim = dim3(plan.units, (unsigned)((threads + (int)mcfg.blockDim.x - 1) / (int)mcfg.blockDim.x));
   mcfg.dynamicSmemBytes = 0;
   mcfg.stream = stream;
   cudaLaunchAttribute mattr[1];
@@ -1572,7 +1625,10 @@ static pkv_status launch_variant(const TcPlan& plan, const CUtensorMap& km, cons
   mattr[0].val.programmaticStreamSerializationAllowed = 1;
   mcfg.attrs = mattr;
   mcfg.numAttrs = 1;
-  e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, merge_all, mp) : cudaLaunchKernelEx(&mcfg, merge, mp);
+  if (lanes == 1)
+    e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, merge_all, mp) : cudaLaunchKernelEx(&mcfg, merge, mp);
+  else
+    e = prm.merge_all ? cudaLaunchKernelEx(&mcfg, merge_all_wide, mp) : cudaLaunchKernelEx(&mcfg, merge_wide, mp);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "decode_merge_kernel launch");
   return PKV_OK;
