@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
       // ---- probabilities in bf16 into P tile c % 2 (row tid, K-major, 128-byte swizzle),
       // once the P V two chunks back is done with it
       if (c >= 2 && !mbar_wait(&p_free[c & 1], ((c - 2) >> 1) & 1, p.wait_limit)) ok = false;
+      fence_proxy_async_smem();  // the tensor core's reads of this P tile come before these stores
       uint8_t* pt = smem + Ly::kOffP + (c & 1) * Ly::kP;
       float ls4[4] = {0.f, 0.f, 0.f, 0.f};  // row sum over four independent chains
 #pragma unroll
@@ -412,6 +413,9 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
     named_barrier(2, kPfxSoftmaxThreads);  // every softmax warp knows whether one gave up
     if (!*reinterpret_cast<volatile int*>(soft_abort)) {
       tc_fence_after_sync();
+      // the staging reuses shared memory the TMA wrote and the tensor core
+      // read (async proxy): order those before these generic stores
+      fence_proxy_async_smem();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       uint8_t* ostage = smem + Ly::kOffO;
 #pragma unroll
