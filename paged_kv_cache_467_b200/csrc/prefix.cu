@@ -9,13 +9,12 @@
 // read by ceil(R / 128) CTAs instead of by every sequence.
 //
 // CTA = one KV head, 128 query rows (the MMA's M), one split of the prefix,
-// seven warps with fixed roles:
-//  * two loader warps stream K and V of 64 tokens (four 16-token blocks) per
-//    chunk, each through its own three-stage ring, in the pool's own row
-//    layout (K is the K-major B operand of S = Q K^T, V the MN-major B operand
-//    of O += P V).  K's stage is free again once S of its chunk is done, V's
-//    once P V is: K runs ahead of the softmax and V ahead of P V.  Their lanes
-//    read the split's block-table entries once, up front;
+// six warps with fixed roles:
+//  * a TMA warp streams K and V of 64 tokens (four 16-token blocks) per chunk
+//    through a three-stage ring, in the pool's own row layout (K is the K-major
+//    B operand of S = Q K^T, V the MN-major B operand of O += P V); its lanes
+//    read the split's block-table entries once, up front, and it starts while
+//    the softmax warps still load the queries;
 //  * an MMA warp issues the tcgen05.mma instructions from one thread: S of a
 //    chunk into one of two tensor-memory buffers while the softmax warps still
 //    read the other, and P V of the chunk before into the O accumulator
@@ -24,12 +23,11 @@
 //    64 scores come in by tcgen05.ld, its running max and sum are kept in
 //    base 2 (the max moved only past 2^8 of slack, its O row then rescaled in
 //    tensor memory), and its bf16 probabilities go to one of two P tiles
-//    (the K-major A operand of P V).  At the end they stage the normalised O
-//    rows in shared memory (128-byte swizzle), then store them row by row.
+//    (the K-major A operand of P V).
 //  * Q [128 x D] bf16 sits in shared memory, K-major with the 128-byte swizzle.
 // The split's result per row, normalised o and base-2 lse, is one piece of the
 // final merge, next to the pieces of the sequence's own blocks.
-// The CTAs also check the prefix contract, each a share of it: every
+// The CTAs that hold KV head 0 also check the prefix contract: every
 // sequence's first prefix_blocks table entries equal row 0's, and every
 // context is longer than the prefix.
 #include <cuda.h>
@@ -47,10 +45,10 @@ namespace pkv {
 constexpr int kPfxRows = 128;   // query rows per CTA (MMA M, TMEM lanes)
 constexpr int kPfxTok = 64;     // tokens per chunk (N of Q K^T, K of P V)
 constexpr int kPfxBlocks = kPfxTok / kBlockSize;
-constexpr int kPfxStages = 3;   // per ring (K, V)
+constexpr int kPfxStages = 3;
 constexpr int kPfxSoftmaxThreads = 128;  // warps 0-3: one query row each
-constexpr int kPfxMmaWarp = 4, kPfxKWarp = 5, kPfxVWarp = 6;
-constexpr int kPfxThreads = 224;
+constexpr int kPfxMmaWarp = 4, kPfxTmaWarp = 5;
+constexpr int kPfxThreads = 192;
 constexpr uint32_t kPfxTmemCols = 256;  // S buffers at columns [0, 64) and [64, 128), O at [128, 128 + D)
 constexpr uint32_t kPfxOCol = 128;
 
@@ -58,19 +56,14 @@ template <int D>
 struct PfxLayout {
   static constexpr int kDBlk = D / 64;                    // 128-byte column blocks of a bf16 row
   static constexpr uint32_t kQ = kPfxRows * D * 2;        // [dblk][128 rows][128 B]
-  static constexpr uint32_t kKV = kPfxTok * D * 2;        // one stage: [dblk][64 tokens][128 B]
+  static constexpr uint32_t kKV = kPfxTok * D * 2;        // [dblk][64 tokens][128 B]
+  static constexpr uint32_t kStage = 2 * kKV;             // K then V
   static constexpr uint32_t kP = kPfxRows * kPfxTok * 2;  // one P tile [128 rows][128 B]
-  static constexpr uint32_t kOffK = kQ;                   // K ring, then V ring
-  static constexpr uint32_t kOffV = kOffK + kPfxStages * kKV;
-  static constexpr uint32_t kOffP = kOffV + kPfxStages * kKV;  // two P tiles
+  static constexpr uint32_t kOffStage = kQ;
+  static constexpr uint32_t kOffP = kOffStage + kPfxStages * kStage;  // two P tiles
   static constexpr uint32_t kOffBar = kOffP + 2 * kP;
-  static constexpr uint32_t kOffTbl = kOffBar + 256;  // each loader warp's copy of the split's block numbers
-  static constexpr uint32_t kBytes = kOffTbl + 2 * 128 * 4;
+  static constexpr uint32_t kBytes = kOffBar + 256;
   static constexpr uint32_t kSmem = kBytes + 1024;        // slack for 1024-byte alignment
-  // the O rows staged for the row stores, fp32 [D / 32][128 rows][128 B],
-  // over the two rings (every load has landed and been read by then)
-  static constexpr uint32_t kOffO = kOffK;
-  static_assert(kPfxRows * D * 4 <= 2 * kPfxStages * kKV, "O staging fits the rings");
 };
 
 struct PrefixParams {
@@ -88,24 +81,22 @@ struct PrefixParams {
 };
 
 // Every sequence shares row 0's first prefix_blocks entries and is longer than
-// the prefix; violations set PKV_DEVERR_PREFIX / PKV_DEVERR_CONTEXT_LEN.  One
-// warp of each CTA checks the sequences s of its row tile with s % n_kv == kv
-// over its split's blocks (the splits starting at block 0: their lengths), so
-// the CTAs of all KV heads share the work.
-__device__ void check_prefix_contract(const PrefixParams& p, int tile, int kv, int b0, int nblk, int lane) {
+// the prefix; violations set PKV_DEVERR_PREFIX / PKV_DEVERR_CONTEXT_LEN.  The
+// CTAs of KV head 0 share the check: this CTA's tile of sequences over its
+// split's blocks.
+__device__ void check_prefix_contract(const PrefixParams& p, int tile, int b0, int nblk) {
   const int s_first = tile * kPfxRows / p.G;
   const int s_last = min(p.num_seqs - 1, (tile * kPfxRows + kPfxRows - 1) / p.G);
-  int s0 = s_first + ((kv - s_first % p.n_kv) + p.n_kv) % p.n_kv;  // first s >= s_first with s % n_kv == kv
-  const int nseq = s0 > s_last ? 0 : (s_last - s0) / p.n_kv + 1;
+  const int nseq = s_last - s_first + 1;
   bool bad_prefix = false, bad_len = false;
-  for (int idx = lane; idx < nseq * nblk; idx += 32) {
-    const int s = s0 + (idx / nblk) * p.n_kv, b = b0 + idx % nblk;
+  for (int idx = threadIdx.x; idx < nseq * nblk; idx += blockDim.x) {
+    const int s = s_first + idx / nblk, b = b0 + idx % nblk;
     if (s > 0 && __ldg(p.block_tables + (size_t)s * p.max_blocks_per_seq + b) != __ldg(p.block_tables + b))
       bad_prefix = true;
   }
   if (b0 == 0) {
-    for (int i = lane; i < nseq; i += 32)
-      if (__ldg(p.context_lens + s0 + i * p.n_kv) <= p.prefix_blocks * kBlockSize) bad_len = true;
+    for (int s = s_first + (int)threadIdx.x; s <= s_last; s += blockDim.x)
+      if (__ldg(p.context_lens + s) <= p.prefix_blocks * kBlockSize) bad_len = true;
   }
   if (bad_prefix) flag_error(p.err, DEVERR_PREFIX);
   if (bad_len) flag_error(p.err, DEVERR_CONTEXT_LEN);
@@ -120,19 +111,16 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* q_tile = smem;
-  uint64_t* full_k = reinterpret_cast<uint64_t*>(smem + Ly::kOffBar);  // [stages] K chunk landed
-  uint64_t* empty_k = full_k + kPfxStages;                               // [stages] S of the chunk done
-  uint64_t* full_v = empty_k + kPfxStages;                               // [stages] V chunk landed
-  uint64_t* empty_v = full_v + kPfxStages;                               // [stages] P V of the chunk done
-  uint64_t* s_full = empty_v + kPfxStages;                               // [2] S buffer written
-  uint64_t* s_free = s_full + 2;                                         // [2] S buffer read out
-  uint64_t* p_full = s_free + 2;                                         // [2] P tile written (O rescaled)
-  uint64_t* p_free = p_full + 2;                                         // [2] P V done with the P tile
-  uint64_t* o_done = p_free + 2;                                         // one phase per P V
-  uint64_t* bar_done = o_done + 1;                                       // every MMA of the CTA done
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Ly::kOffBar);  // [stages] K/V chunk landed
+  uint64_t* empty = full + kPfxStages;                                // [stages] P V of the chunk done
+  uint64_t* s_full = empty + kPfxStages;                              // [2] S buffer written
+  uint64_t* s_free = s_full + 2;                                      // [2] S buffer read out
+  uint64_t* p_full = s_free + 2;                                      // [2] P tile written (O rescaled)
+  uint64_t* p_free = p_full + 2;                                      // [2] P V done with the P tile
+  uint64_t* o_done = p_free + 2;                                      // one phase per P V
+  uint64_t* bar_done = o_done + 1;                                    // every MMA of the CTA done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_done + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);  // some wait gave up
-  int* soft_abort = abort_flag + 1;  // a softmax warp gave up (written by those warps only)
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = blockIdx.x, kv = blockIdx.y, split = blockIdx.z;
@@ -140,29 +128,16 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
   const int b1 = min(b0 + p.chunks_per_split * kPfxBlocks, p.prefix_blocks);
   const int nblk = max(0, b1 - b0);
   const int nchunks = (nblk + kPfxBlocks - 1) / kPfxBlocks;
-  const bool loader = warp == kPfxKWarp || warp == kPfxVWarp;
 
   // The previous kernel on the stream may still run: wait for it before
   // reading anything, then let the next kernel be scheduled.
   grid_wait_prerequisites();
   grid_launch_dependents();
 
-  // Loader lanes: the physical blocks of the split's blocks b0 + i, b0 + 32 + i, ...
-  // (read first, so that their latency overlaps the set-up below)
-  constexpr int kMaxHeld = 4;  // up to 128 blocks per split kept in shared memory
-  int held[kMaxHeld];
-#pragma unroll
-  for (int r = 0; r < kMaxHeld; ++r) {
-    const int b = b0 + r * 32 + lane;
-    held[r] = (loader && b < b1) ? __ldg(p.block_tables + b) : -1;
-  }
-
   if (tid == 0) {
     for (int k = 0; k < kPfxStages; ++k) {
-      mbar_init(&full_k[k], 1);
-      mbar_init(&empty_k[k], 1);
-      mbar_init(&full_v[k], 1);
-      mbar_init(&empty_v[k], 1);
+      mbar_init(&full[k], 1);
+      mbar_init(&empty[k], 1);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&s_full[k], 1);
@@ -173,7 +148,6 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
     mbar_init(o_done, 1);
     mbar_init(bar_done, 1);
     *abort_flag = 0;
-    *soft_abort = 0;
     fence_barrier_init();
   }
   if (warp == kPfxMmaWarp) {
@@ -202,75 +176,76 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
     fence_proxy_async_smem();
   }
   // the Q tile is complete once the softmax warps and the MMA warp meet here
-  // (the loader warps do not wait for it)
-  if (!loader) named_barrier(1, kPfxSoftmaxThreads + 32);
+  // (the TMA warp does not wait for it)
+  if (warp != kPfxTmaWarp) named_barrier(1, kPfxSoftmaxThreads + 32);
 
-  if (loader) {
-    // ---------------------------------------------------------- loader warps (K, V)
-    const bool is_k = warp == kPfxKWarp;
-    uint64_t* fullb = is_k ? full_k : full_v;
-    uint64_t* emptyb = is_k ? empty_k : empty_v;
-    const CUtensorMap* map = is_k ? &kmap : &vmap;
-    uint8_t* ring = smem + (is_k ? Ly::kOffK : Ly::kOffV);
-    // the split's physical blocks into this warp's table in shared memory
-    // (-1: past the split, or outside the pool: read as zeros, flagged)
-    int* tbl = reinterpret_cast<int*>(smem + Ly::kOffTbl) + (is_k ? 0 : kMaxHeld * 32);
+  if (warp == kPfxTmaWarp) {
+    // ---------------------------------------------------------- TMA warp
+    // lane i holds the physical block of the split's blocks b0 + i, b0 + 32 + i, ...
+    constexpr int kMaxHeld = 4;  // up to 128 blocks per split held in registers
+    int held[kMaxHeld];
 #pragma unroll
     for (int r = 0; r < kMaxHeld; ++r) {
-      const bool in_split = b0 + r * 32 + lane < b1;
-      int v = held[r];
-      if (in_split && (v < 0 || (long long)v >= p.num_blocks)) {
-        if (is_k) flag_error(p.err, DEVERR_BLOCK_RANGE);
-        v = -1;
+      const int b = b0 + r * 32 + lane;
+      held[r] = -1;
+      if (b < b1) {
+        held[r] = __ldg(p.block_tables + b);
+        if (held[r] < 0 || (long long)held[r] >= p.num_blocks) {
+          flag_error(p.err, DEVERR_BLOCK_RANGE);
+          held[r] = -1;
+        }
       }
-      tbl[r * 32 + lane] = v;
     }
-    __syncwarp();
-    if (lane == 0) prefetch_tensormap(map);
     int issued = 0;
+    if (lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+    }
     for (; issued < nchunks; ++issued) {
-      // the chunk's four physical blocks
+      // the chunk's four physical blocks (-1: past the split or outside the pool)
       int phys4[kPfxBlocks];
 #pragma unroll
       for (int i = 0; i < kPfxBlocks; ++i) {
         const int j = issued * kPfxBlocks + i;  // block index inside the split
-        if (j < kMaxHeld * 32) {
-          phys4[i] = tbl[j];
-        } else {  // a split longer than the table: read it here
-          phys4[i] = b0 + j < b1 ? __ldg(p.block_tables + b0 + j) : -1;
-          if (b0 + j < b1 && (phys4[i] < 0 || (long long)phys4[i] >= p.num_blocks)) {
-            if (lane == 0 && is_k) flag_error(p.err, DEVERR_BLOCK_RANGE);
+        int v = -1;
+#pragma unroll
+        for (int r = 0; r < kMaxHeld; ++r) v = (j >> 5) == r ? held[r] : v;
+        phys4[i] = __shfl_sync(0xffffffffu, v, j & 31);
+        if (j >= kMaxHeld * 32 && b0 + j < b1) {  // a split longer than the lanes hold: read it here
+          phys4[i] = __ldg(p.block_tables + b0 + j);
+          if (phys4[i] < 0 || (long long)phys4[i] >= p.num_blocks) {
+            if (lane == 0) flag_error(p.err, DEVERR_BLOCK_RANGE);
             phys4[i] = -1;
           }
         }
       }
       if (lane == 0) {
         const int k = issued, stage = k % kPfxStages;
-        // the stage's previous chunk (k - stages) must have been read by its MMA
-        if (k >= kPfxStages && !mbar_wait(&emptyb[stage], ((k / kPfxStages) - 1) & 1, p.wait_limit))
+        // the stage's previous chunk (k - stages) must have gone through P V
+        if (k >= kPfxStages && !mbar_wait(&empty[stage], ((k / kPfxStages) - 1) & 1, p.wait_limit))
           atomicExch(abort_flag, 1);
-        uint8_t* dst = ring + stage * Ly::kKV;
+        uint8_t* kst = smem + Ly::kOffStage + stage * Ly::kStage;
+        uint8_t* vst = kst + Ly::kKV;
         if (!*abort_flag) {
-          mbar_arrive_expect_tx(&fullb[stage], Ly::kKV);
+          mbar_arrive_expect_tx(&full[stage], Ly::kStage);
 #pragma unroll
           for (int i = 0; i < kPfxBlocks; ++i) {
             // blocks past the split, and table entries outside the pool, read as zeros (TMA fill)
 #pragma unroll
             for (int db = 0; db < Ly::kDBlk; ++db) {
               const uint32_t off = db * (kPfxTok * 128) + i * (kBlockSize * 128);
-              tma_load_3d(dst + off, map, 0, kv * Ly::kDBlk + db, phys4[i] * kBlockSize, &fullb[stage]);
+              tma_load_3d(kst + off, &kmap, 0, kv * Ly::kDBlk + db, phys4[i] * kBlockSize, &full[stage]);
+              tma_load_3d(vst + off, &vmap, 0, kv * Ly::kDBlk + db, phys4[i] * kBlockSize, &full[stage]);
             }
           }
         }
       }
       if (__shfl_sync(0xffffffffu, *abort_flag, 0)) break;
     }
-    // the K warp, done issuing, takes this CTA's share of the contract check
-    if (is_k) check_prefix_contract(p, tile, kv, b0, nblk, lane);
     // never leave with copies in flight: the last stages issued have landed
     if (lane == 0) {
       for (int k = max(0, issued - kPfxStages); k < issued; ++k)
-        mbar_wait(&fullb[k % kPfxStages], (k / kPfxStages) & 1);
+        mbar_wait(&full[k % kPfxStages], (k / kPfxStages) & 1);
     }
   } else if (warp == kPfxMmaWarp) {
     // ---------------------------------------------------------- MMA warp
@@ -278,13 +253,8 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
       constexpr uint32_t idesc_qk = umma_idesc_bf16(kPfxRows, kPfxTok, false, false);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(kPfxRows, D, false, true);
       const uint32_t q_addr = smem_addr(q_tile);
-      bool ok = true;
-      auto issue_pv = [&](int c) {  // O += P(c) V(c), then free the V stage and the P tile
-        ok = mbar_wait(&p_full[c & 1], (c >> 1) & 1, p.wait_limit) &&
-             mbar_wait(&full_v[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
-        if (!ok) return;
-        tc_fence_after_sync();
-        const uint32_t v_addr = smem_addr(smem + Ly::kOffV + (c % kPfxStages) * Ly::kKV);
+      auto issue_pv = [&](int c) {  // O += P(c) V(c), then free the stage and the P tile
+        const uint32_t v_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage + Ly::kKV);
         const uint32_t pt = smem_addr(smem + Ly::kOffP + (c & 1) * Ly::kP);
 #pragma unroll
         for (int kt = 0; kt < kPfxTok / 16; ++kt) {
@@ -292,17 +262,18 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
           const uint64_t b = umma_desc_sw128(v_addr + kt * 2048, kPfxTok * 128, 1024);
           umma_bf16(t_o, a, b, idesc_pv, (c > 0 || kt > 0) ? 1u : 0u);
         }
-        umma_commit(&empty_v[c % kPfxStages]);
+        umma_commit(&empty[c % kPfxStages]);
         umma_commit(&p_free[c & 1]);
         umma_commit(o_done);
       };
+      bool ok = true;
       for (int c = 0; c < nchunks && ok; ++c) {
-        ok = mbar_wait(&full_k[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
+        ok = mbar_wait(&full[c % kPfxStages], (c / kPfxStages) & 1, p.wait_limit);
         if (ok && c >= 2) ok = mbar_wait(&s_free[c & 1], ((c - 2) >> 1) & 1, p.wait_limit);
         if (!ok) break;
         tc_fence_after_sync();
         // S(c) = Q K(c)^T into S buffer c % 2
-        const uint32_t k_addr = smem_addr(smem + Ly::kOffK + (c % kPfxStages) * Ly::kKV);
+        const uint32_t k_addr = smem_addr(smem + Ly::kOffStage + (c % kPfxStages) * Ly::kStage);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           const uint64_t a = umma_desc_sw128(q_addr + (ks >> 2) * (kPfxRows * 128) + (ks & 3) * 32, 16, 1024);
@@ -310,11 +281,21 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
           umma_bf16(tmem + (c & 1) * kPfxTok, a, b, idesc_qk, ks > 0);
         }
         umma_commit(&s_full[c & 1]);
-        umma_commit(&empty_k[c % kPfxStages]);
         // P V of the chunk before, once its probabilities are written
-        if (c >= 1) issue_pv(c - 1);
+        if (c >= 1) {
+          ok = mbar_wait(&p_full[(c - 1) & 1], ((c - 1) >> 1) & 1, p.wait_limit);
+          if (!ok) break;
+          tc_fence_after_sync();
+          issue_pv(c - 1);
+        }
       }
-      if (ok && nchunks > 0) issue_pv(nchunks - 1);
+      if (ok && nchunks > 0) {
+        ok = mbar_wait(&p_full[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1, p.wait_limit);
+        if (ok) {
+          tc_fence_after_sync();
+          issue_pv(nchunks - 1);
+        }
+      }
       if (!ok) atomicExch(abort_flag, 1);
       // every MMA issued has completed before the CTA moves on
       umma_commit(bar_done);
@@ -401,53 +382,35 @@ __global__ void __launch_bounds__(kPfxThreads, 1)
       mbar_arrive(&p_full[c & 1]);
       if (!ok) break;
     }
-    // ---- the last P V done: normalised partial o of the 128 rows through
-    // shared memory (fp32, [D / 32][128 rows][128 B], 128-byte swizzle, each
-    // thread writes its row conflict-free) to coalesced row stores (rows past
-    // the batch are skipped), and the base-2 lse per row
+    // ---- the last P V done: normalised partial o and base-2 lse of this row
+    // and split (every lane takes part in the warp-wide loads; rows past the
+    // batch store nothing)
     if (ok && nchunks > 0 && !mbar_wait(o_done, (nchunks - 1) & 1, p.wait_limit)) ok = false;
-    if (!__all_sync(0xffffffffu, ok) && lane == 0) {
+    if (!__all_sync(0xffffffffu, ok)) {
       atomicExch(abort_flag, 1);
-      *soft_abort = 1;
-    }
-    named_barrier(2, kPfxSoftmaxThreads);  // every softmax warp knows whether one gave up
-    if (!*reinterpret_cast<volatile int*>(soft_abort)) {
+    } else {
       tc_fence_after_sync();
-      // the staging reuses shared memory the TMA wrote and the tensor core
-      // read (async proxy): order those before these generic stores
-      fence_proxy_async_smem();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint8_t* ostage = smem + Ly::kOffO;
+      float4* dst =
+          reinterpret_cast<float4*>(p.part_o + (((size_t)kv * p.splits + split) * p.rows + (row_ok ? row : 0)) * D);
 #pragma unroll
       for (int cb = 0; cb < D / 32; ++cb) {
         uint32_t orow[32];
         tmem_ld32(t_o + lane_base + cb * 32, orow);
         tmem_wait_ld();
-        uint8_t* dst = ostage + cb * (kPfxRows * 128) + tid * 128;
+        if (row_ok) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4*>(dst + ((j ^ (tid & 7)) << 4)) =
-              make_float4(__uint_as_float(orow[4 * j]) * inv, __uint_as_float(orow[4 * j + 1]) * inv,
-                          __uint_as_float(orow[4 * j + 2]) * inv, __uint_as_float(orow[4 * j + 3]) * inv);
-      }
-      named_barrier(2, kPfxSoftmaxThreads);
-      // row by row, a warp per row: lane e holds floats 4e .. 4e+3 (column
-      // block e / 8, 16-byte piece e % 8), one coalesced store of the row
-      float* o_plane = p.part_o + ((size_t)kv * p.splits + split) * p.rows * D;
-      const int nrows = min(kPfxRows, p.rows - tile * kPfxRows);
-      for (int r = warp; r < nrows; r += kPfxSoftmaxThreads / 32) {
-#pragma unroll
-        for (int e = lane; e < D / 4; e += 32) {
-          const float4 v = *reinterpret_cast<const float4*>(ostage + (e >> 3) * (kPfxRows * 128) + r * 128 +
-                                                            (((e & 7) ^ (r & 7)) << 4));
-          reinterpret_cast<float4*>(o_plane + (size_t)(tile * kPfxRows + r) * D)[e] = v;
+          for (int j = 0; j < 8; ++j)
+            dst[cb * 8 + j] = make_float4(__uint_as_float(orow[4 * j]) * inv, __uint_as_float(orow[4 * j + 1]) * inv,
+                                          __uint_as_float(orow[4 * j + 2]) * inv,
+                                          __uint_as_float(orow[4 * j + 3]) * inv);
         }
       }
-      if (row_ok)
-        p.part_lse[((size_t)kv * p.splits + split) * p.rows + row] = nchunks > 0 ? m + log2f(l) : -INFINITY;
+      if (row_ok) p.part_lse[((size_t)kv * p.splits + split) * p.rows + row] = nchunks > 0 ? m + log2f(l) : -INFINITY;
     }
   }
 
+  if (kv == 0) check_prefix_contract(p, tile, b0, nblk);
   tc_fence_before_sync();
   __syncthreads();  // nothing in flight, every TMEM read done
   if (tid == 0 && *abort_flag) flag_error(p.err, DEVERR_TIMEOUT);
@@ -489,7 +452,6 @@ static pkv_status run_prefix_kernel(dim3 grid, const CUtensorMap& km, const CUte
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(prefix_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess) e = prefer_max_smem(prefix_tc_kernel<D>);  // decode CTAs share the SM
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefix)");
     configured = true;
   }

@@ -121,6 +121,24 @@ def test_prefix_pass_beside_and_after_the_decode_agree():
         assert np.array_equal(results[(splits, False)][1], results[(splits, True)][1])
 
 
+def test_repeated_calls_are_bitwise_equal():
+    """The same call, repeated, gives the same bits (every piece is written by
+    one CTA at a fixed place and merged in a fixed order): per split setting
+    and order of the passes, four calls, outputs compared byte for byte."""
+    ops = _ops()
+    w = workloads.make_workload("p", seed=83, context_lens=[1100 + 61 * i for i in range(40)], n_q=32, n_kv=8,
+                                head_dim=128, extra_blocks=3, shared_prefix_tokens=1024)
+    st = fill_gpu(w)
+    for splits in (0, 1, 3):
+        for serial in (False, True):
+            tun = ops.DecodeTuning(0, 0, 0, ops.TUNE_PREFIX_SERIAL if serial else 0, splits)
+            first, first_lse = run_shared(w, st, tuning=tun)
+            for _ in range(3):
+                out, lse = run_shared(w, st, tuning=tun)
+                assert np.array_equal(out, first) and np.array_equal(lse, first_lse), (splits, serial)
+            assert int(st.device_error.item()) == 0
+
+
 def test_sequence_shorter_than_prefix_is_flagged():
     """A context that does not reach past the shared prefix sets the context-length
     bit; the other sequences are unaffected."""
