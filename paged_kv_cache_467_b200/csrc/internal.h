@@ -52,11 +52,10 @@ struct TcPlan {
 
 pkv_status plan_tc(const DecodeShape& s, const pkv_decode_tuning* tuning, TcPlan* plan);
 
-// The kernels of a decode step (prefix pass, decode, merge) ask for the
-// largest shared-memory carveout.  An SM's split between L1 and shared memory
-// is fixed while CTAs run on it, so a kernel configured for less shared memory
-// (the default picks the smallest split that fits its own CTA) would keep the
-// CTAs of the kernel running beside it off that SM.
+// The decode and merge kernels ask for the largest shared-memory carveout.
+// An SM's split between L1 and shared memory is fixed while CTAs run on it,
+// and the default picks the smallest split that fits a kernel's own CTA, which
+// would keep the CTAs of a kernel running beside it off that SM.
 template <typename Kernel>
 inline cudaError_t prefer_max_smem(Kernel kern) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
